@@ -1,0 +1,372 @@
+"""Throughput of the KronQ per-layer quantization path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kronq|reference]
+                    [--workload attn4096] [--bits 4,3,2]
+
+One step is the whole path for one Llama-2-7B attention-projection-shaped
+layer (W 4096x4096, 128 x 2048 = 262144 calibration tokens of bf16 X and G):
+both covariance SYRKs, the trace sensitivity, the BiIP rotations of W, H_X and
+H_G, the damped Cholesky factor of the inverse, and for each bit-width (W4, W3,
+W2 per-channel) the blocked OBS quantization and the Kronecker loss.  The
+metric counts the weights quantized: d_out * d_in per bit-width per step.
+Inputs are synthetic (seeded), resident in HBM before timing, and larger than
+L2 (X and G are 2 GiB each), so no L2 flush is needed between steps.
+
+With N > 1 (torchrun) every rank quantizes its own layer (weak scaling, no
+data-path collective); timing is the max over ranks.  Rank 0 prints one JSON
+line.  --impl reference times the float64 CPU oracle on a bounded sample of
+the same workload on the host cores and prints the same line for it.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "weights quantized/sec per layer"
+UNIT = "weights/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="kronq", choices=["kronq", "reference"])
+    ap.add_argument("--workload", default="attn4096")
+    ap.add_argument("--bits", default="4,3,2")
+    ap.add_argument("--group", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args()
+    a.warmup = max(a.warmup, 3)
+    return a
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during timing."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", str(self.idx)],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- GPU arm
+
+def run_kronq(a):
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    import post_weight_quantization_syrk_b200 as P
+    from post_weight_quantization_syrk_b200.pipeline import LayerQuantizer
+
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+    P.load()
+    spec = synth.WORKLOADS[a.workload]
+    bits = [int(b) for b in a.bits.split(",")]
+    settings = [(b, a.group) for b in bits]
+    seed = synth.layer_seed(2, rank)
+    with torch.no_grad():
+        W = synth.weights(spec, seed, dev)
+        X = synth.activations(spec, seed, dev)
+        G = synth.gradients(spec, seed, dev)
+    Ti, To = synth.rht_params(spec.d_in, seed * 2 + 11), synth.rht_params(spec.d_out, seed * 2 + 12)
+
+    def dev_rht(p):
+        return P.RHT(p.n, p.log2_p, p.m, p.signs.to(dev), None if p.Qm is None else p.Qm.to(dev))
+
+    T_in, T_out = dev_rht(Ti), dev_rht(To)
+    lq = LayerQuantizer(spec.d_out, spec.d_in, dev)
+    results = [lq.alloc_result(b, g) for b, g in settings]
+    stream = torch.cuda.current_stream()
+
+    syrk_events = []
+
+    def step(timed):
+        if timed:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e2 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            lq.statistics(X, G)   # the two SYRKs (H_X, then H_G)
+            e2.record(stream)
+            syrk_events.append((e0, e2))
+            _ = e1
+        else:
+            lq.statistics(X, G)
+        lq.sensitivity()
+        lq.rotate(W, T_in, T_out)
+        lq.factor(0.01)
+        for r in results:
+            lq.quantize(r)
+            lq.loss(r)
+
+    for _ in range(a.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    lq.check("warmup")
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    launches0 = P.kq_launch_count()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(a.steps):
+        step(True)
+    end.record(stream)
+    torch.cuda.synchronize()
+    launches = P.kq_launch_count() - launches0
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    lq.check("timed steps")
+    ms = start.elapsed_time(end)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    syrk_ms = [e0.elapsed_time(e2) / 2.0 for e0, e2 in syrk_events]   # two SYRK launches per step
+    weights_per_step = spec.d_out * spec.d_in * len(settings)
+    value = weights_per_step * a.steps * world / (ms_max / 1e3)
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not a.no_e2e:
+        e2e = run_e2e(a, lq, results, W, X, G, T_in, T_out, spec, settings, world, dev)
+
+    pk, src = peaks()
+    flops = spec.n_tokens * spec.d_in * (spec.d_in + 1)    # one SYRK launch on X (d_out == d_in here)
+    syrk_avg = statistics.mean(syrk_ms)
+    achieved = flops / (syrk_avg / 1e3) / 1e12
+    peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+        "ms_per_step": ms_max / a.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16->fp32 (SYRK), fp64 (Cholesky), fp32 (solver, loss)", "data": "synthetic",
+        "config": {"workload": f"{a.workload}: W {spec.d_out}x{spec.d_in}, N={spec.n_tokens} tokens, "
+                               f"{'+'.join('W%d' % b for b in bits)} {'per-channel' if not a.group else 'g%d' % a.group}",
+                   "layers_per_rank_per_step": 1, "bit_widths": bits, "group": a.group,
+                   "l2": "inputs larger than L2 (X, G 2 GiB each); no flush"},
+        "roofline": {"kernel": "kq_accum_cov (SYRK)", "bound": "tensor", "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                     "peak_source": f"{src} bf16 sustained", "algorithmic_flops_per_launch": flops,
+                     "avg_launch_ms": syrk_avg},
+        "gpu_launches": launches,
+        "clocks": clk,
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        out["cpu_baseline"] = oracle_sample(spec, settings)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def run_e2e(a, lq, results, W, X, G, T_in, T_out, spec, settings, world, dev):
+    """Same step through the public API from pinned host buffers: inputs are
+    copied host->device and the results (codes, grids, losses) device->host
+    inside the timed region."""
+    import torch
+    Wh, Xh, Gh = W.cpu().pin_memory(), X.cpu().pin_memory(), G.cpu().pin_memory()
+    Wd, Xd, Gd = torch.empty_like(W), torch.empty_like(X), torch.empty_like(G)
+    outs = [(torch.empty(r.codes.shape, dtype=torch.uint8, pin_memory=True),
+             torch.empty(r.scales.shape, pin_memory=True), torch.empty(r.zeros.shape, pin_memory=True),
+             torch.empty(1, dtype=torch.float64, pin_memory=True)) for r in results]
+    h2d = Wh.numel() * 4 + Xh.numel() * 2 + Gh.numel() * 2
+    d2h = sum(o[0].numel() + o[1].numel() * 4 + o[2].numel() * 4 + 8 for o in outs)
+    stream = torch.cuda.current_stream()
+    n = min(a.steps, 3)
+
+    def one():
+        Wd.copy_(Wh, non_blocking=True)
+        Xd.copy_(Xh, non_blocking=True)
+        Gd.copy_(Gh, non_blocking=True)
+        lq.run(Wd, Xd, Gd, T_in, T_out, settings, results=results)
+        for r, o in zip(results, outs):
+            o[0].copy_(r.codes, non_blocking=True)
+            o[1].copy_(r.scales, non_blocking=True)
+            o[2].copy_(r.zeros, non_blocking=True)
+            o[3].copy_(r.loss, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(n):
+        one()
+    e.record(stream)
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    return {"value": spec.d_out * spec.d_in * len(settings) * n * world / (ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms / n, "steps": n}
+
+
+# ----------------------------------------------------------------- CPU oracle
+
+def oracle_sample(spec, settings, seed=1234):
+    """Time the float64 oracle on a bounded sample of the workload and scale
+    each stage to the full layer by its work:
+      covariances: n_s of the N tokens (cost linear in tokens),
+      BiIP rotations, damped Cholesky factor: full size,
+      solver: r_s of the d_out rows (rows are independent given Uc),
+      Kronecker loss: full size, once, counted for every bit-width."""
+    import numpy as np
+    import torch
+
+    import oracle as O
+    import synth
+    n_s, r_s = 1024, 32
+    sp = synth.scaled(spec, n_tokens=n_s)
+    W = synth.weights(sp, seed).double().numpy()
+    X = synth.activations(sp, seed).float().numpy()
+    G = synth.gradients(sp, seed).float().numpy()
+    Ti, To = synth.rht_params(spec.d_in, 7), synth.rht_params(spec.d_out, 8)
+    Tin = O.rht_matrix(Ti.n, Ti.log2_p, Ti.signs.double().numpy(), None if Ti.Qm is None else Ti.Qm.double().numpy())
+    Tout = O.rht_matrix(To.n, To.log2_p, To.signs.double().numpy(), None if To.Qm is None else To.Qm.double().numpy())
+    t = {}
+    c0 = time.perf_counter()
+    HX = O.covariance(X)
+    HG = O.covariance(G)
+    t["cov"] = (time.perf_counter() - c0) * spec.n_tokens / n_s
+    c0 = time.perf_counter()
+    O.sensitivity(HX, HG)
+    Wp, HXp, HGp = O.biip(W, HX, HG, Tin, Tout)
+    t["rot"] = time.perf_counter() - c0
+    c0 = time.perf_counter()
+    Uc, dead, _ = O.chol_inv(HXp, 0.01)
+    t["chol"] = time.perf_counter() - c0
+    t["quant"] = 0.0
+    for b, g in settings:
+        c0 = time.perf_counter()
+        q = O.quantize_layer(Wp[:r_s], Uc, b, g, 128, dead)
+        t["quant"] += (time.perf_counter() - c0) * spec.d_out / r_s
+    Wh = np.array(Wp, copy=True)
+    Wh[:r_s] = q.W_hat
+    c0 = time.perf_counter()
+    O.kron_loss(Wp, Wh, HXp, HGp)
+    t["loss"] = (time.perf_counter() - c0) * len(settings)
+    total = sum(t.values())
+    threads = torch.get_num_threads()
+    return {"value": spec.d_out * spec.d_in * len(settings) / total, "unit": UNIT,
+            "cores": os.cpu_count(), "threads": threads, "kind": "oracle",
+            "seconds_per_step_extrapolated": total, "stage_seconds": t,
+            "sample": f"covariances on {n_s} of {spec.n_tokens} tokens (x{spec.n_tokens // n_s}); solver on "
+                      f"{r_s} of {spec.d_out} rows (x{spec.d_out // r_s}); rotations, Cholesky and one "
+                      f"Kronecker loss at full size (loss x{len(settings)}); NumPy float64 on the host cores"}
+
+
+def run_reference(a):
+    rank = int(os.environ.get("RANK", 0))
+    if rank != 0:
+        return
+    import synth
+    spec = synth.WORKLOADS[a.workload]
+    bits = [int(b) for b in a.bits.split(",")]
+    settings = [(b, a.group) for b in bits]
+    for _ in range(a.warmup if a.warmup <= 1 else 1):
+        oracle_sample(spec, settings)
+    vals, secs = [], []
+    for k in range(a.steps):
+        r = oracle_sample(spec, settings, seed=1234 + k)
+        vals.append(r["value"])
+        secs.append(r["seconds_per_step_extrapolated"])
+    value = len(vals) / sum(1.0 / v for v in vals)
+    last = r
+    out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup,
+           "ms_per_step": 1e3 * statistics.mean(secs), "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+           "config": {"workload": f"{a.workload}: W {spec.d_out}x{spec.d_in}, N={spec.n_tokens} tokens, "
+                                  f"{'+'.join('W%d' % b for b in bits)} "
+                                  f"{'per-channel' if not a.group else 'g%d' % a.group}",
+                      "bit_widths": bits, "group": a.group},
+           "cpu_baseline": {"value": value, "unit": UNIT, "cores": last["cores"], "kind": "oracle",
+                            "sample": last["sample"]},
+           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    a = parse()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_kronq(a)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,261 @@
+/*
+ * kronq.h - C ABI of the KronQ per-linear-layer quantization path on B200.
+ *
+ * The path (one linear layer y = W x, W [d_out, d_in] row-major):
+ *   1. H_X = X^T X / N and H_G = G^T G / N from bf16 calibration activations
+ *      X [N, d_in] and output gradients G [N, d_out]        -> kq_accum_cov
+ *   2. sensitivity tr(H_X), tr(H_G), tr(H_G) tr(H_X)          -> kq_sensitivity
+ *   3. bidirectional incoherence processing: W' = V W U^T,
+ *      H_X' = U H_X U^T, H_G' = V H_G V^T with randomised
+ *      Hadamard rotations U (input side) and V (output side) -> kq_rotate
+ *   4. damping, dead columns and the upper Cholesky factor of
+ *      the damped inverse of H_X'                            -> kq_chol_inv
+ *   5. blocked column-wise OBS (GPTQ) quantization of W' on a
+ *      b-bit asymmetric grid                                  -> kq_quantize_layer
+ *   6. Kronecker loss tr(dW H_X' dW^T H_G')                   -> kq_kron_loss
+ *   7. sublayer bit allocation from the sensitivities (host)  -> kq_allocate_bits
+ *
+ * Sources (page title and section):
+ *   - KronQ paper page (Hugging Face papers 2607.07964), Abstract: H ~ H_X kron
+ *     H_G; bidirectional incoherence processing; trace sensitivity for
+ *     mixed precision.  Authors' reply (Community thread): H_G from one
+ *     backward pass, reused across bit-widths.
+ *   - Paper review "KronQ: LLM Quantization via Kronecker-Factored Hessian"
+ *     (romaanj.github.io/reviews/kronq), sections Background, Prior
+ *     limitations, Goal, Method, Comparison, Limitations.
+ *   - "A Unified Hessian-Guided Framework for Post-Training Quantization"
+ *     (hub.valency.io/works/W_r72x54u6), Background (grid step and shift;
+ *     transformations), Appendix A.1 (trace form of the Kronecker norm).
+ *
+ * Conventions for every entry point:
+ *   - Matrices are row-major with an explicit leading dimension (elements).
+ *   - Every pointer is CALLER-OWNED DEVICE memory unless stated otherwise;
+ *     the library allocates and frees nothing.  Scratch memory is sized by the
+ *     matching kq_*_workspace_size() and passed in as (ws, ws_bytes); ws must
+ *     be 256-byte aligned.
+ *   - Work is enqueued on `stream` (NULL = legacy default stream) and the
+ *     call returns without synchronising.  Host-side validation errors are
+ *     returned synchronously and nothing is enqueued.
+ *   - Device-detected errors are written to `info`, a caller-owned device
+ *     int32 that the library never clears: the first error sticks (code in
+ *     bits 24..31, an index in bits 0..23, see KQ_INFO_*).  Zero it before a
+ *     chain of calls and read it after the stream has synchronised.
+ *   - Every device wait is bounded; on expiry the kernel records
+ *     KQ_ERR_TIMEOUT in `info` and returns.
+ *   - The library is stateless apart from a thread-local last-error string
+ *     and is safe to call from several host threads.  No C++ exception
+ *     crosses this ABI.
+ */
+#ifndef KRONQ_H
+#define KRONQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The same handle type as cudaStream_t. */
+typedef struct CUstream_st* kq_stream_t;
+
+typedef enum kq_status {
+  KQ_OK = 0,
+  KQ_ERR_INVALID_ARG = 1,       /* NULL pointer, negative size, bad enum value        */
+  KQ_ERR_UNSUPPORTED_SHAPE = 2, /* a size outside the limits stated per call          */
+  KQ_ERR_ALIGNMENT = 3,         /* pointer or leading dimension misaligned            */
+  KQ_ERR_WORKSPACE = 4,         /* ws too small or misaligned                          */
+  KQ_ERR_CUDA = 5,              /* a CUDA runtime call failed (see kq_last_error)     */
+  KQ_ERR_NOT_PD = 6,            /* device: damped matrix not positive definite        */
+  KQ_ERR_NONFINITE = 7,         /* device: NaN or Inf met in an input                  */
+  KQ_ERR_TIMEOUT = 8            /* device: a bounded wait expired                      */
+} kq_status;
+
+#define KQ_INFO_CODE(info) ((int32_t)(((uint32_t)(info)) >> 24))
+#define KQ_INFO_INDEX(info) ((int32_t)((info) & 0xFFFFFF))
+
+enum { KQ_AXIS_ROWS = 0, KQ_AXIS_COLS = 1 };
+enum { KQ_GEMM_FP32 = 0, KQ_GEMM_3XTF32 = 1 };
+
+/* Human-readable name of a status code (static string). */
+const char* kq_status_string(kq_status s);
+/* Detail of the last non-OK status returned on this host thread ("" if none). */
+const char* kq_last_error(void);
+/* Library version, major * 10000 + minor * 100 + patch. */
+int kq_version(void);
+/* Number of CUDA kernel launches this library has enqueued in this process
+ * (all host threads); a diagnostic for counting device work per step. */
+unsigned long long kq_launch_count(void);
+
+/* --------------------------------------------------------------------------
+ * kq_accum_cov - covariance accumulation (steps a1/a2).
+ *
+ * Computes C = alpha * A^T A (accumulate == 0) or C += alpha * A^T A
+ * (accumulate != 0), the input-activation covariance H_X = E[x x^T] or the
+ * output-gradient covariance H_G = E[g g^T] (KronQ review, Background: the
+ * Kronecker factors of the layer Hessian; research thread: H_G = E[g g^T]).
+ * Pass alpha = 1 / N_total to obtain the mean over all calls' tokens.
+ *
+ *   A      bf16 bit patterns, [n, d] row-major (tokens x channels), lda >= d;
+ *          lda % 8 == 0 and A 16-byte aligned (TMA requirements); may be
+ *          NULL when n == 0.
+ *   n      number of tokens, >= 0 (n == 0 leaves C = 0 or unchanged).
+ *   d      channels, 1 <= d <= 65536.
+ *   C      fp32 [d, d] row-major, ldc >= d; the full symmetric matrix is
+ *          written (lower triangle computed and mirrored).
+ *   ws     workspace of kq_accum_cov_workspace_size(n, d) bytes.
+ *   info   device word; KQ_ERR_NONFINITE (index = row) if C gets NaN/Inf,
+ *          KQ_ERR_TIMEOUT if a pipeline wait expired.
+ * Tensor cores: bf16 x bf16 products accumulated in fp32.
+ * ------------------------------------------------------------------------ */
+size_t kq_accum_cov_workspace_size(int64_t n, int64_t d);
+kq_status kq_accum_cov(const uint16_t* A, int64_t n, int64_t d, int64_t lda,
+                       float* C, int64_t ldc, float alpha, int accumulate,
+                       void* ws, size_t ws_bytes, int32_t* info, kq_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * kq_sensitivity - trace sensitivity (step a3).
+ *
+ * out3[0] = tr(H_X), out3[1] = tr(H_G), out3[2] = tr(H_G) * tr(H_X), each
+ * summed in fp64 (KronQ review, Method (2): the joint score tr(H_G) tr(H_X)
+ * separates sublayers with identical inputs; tr(H_X) alone is the H_X-only
+ * score of the Comparison section).
+ *
+ *   H_X  fp32 [d_in, d_in], ldhx >= d_in;  H_G fp32 [d_out, d_out], ldhg >= d_out.
+ *   out3 device fp64[3].
+ * ------------------------------------------------------------------------ */
+kq_status kq_sensitivity(const float* H_X, int64_t d_in, int64_t ldhx,
+                         const float* H_G, int64_t d_out, int64_t ldhg,
+                         double* out3, kq_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * kq_rotate - randomised Hadamard rotation (steps a4/a5, BiIP).
+ *
+ * T = (Q_m kron H_p / sqrt(p)) . diag(signs), n = m * p, p = 2^log2_p, with
+ * H_p the Sylvester Walsh-Hadamard matrix (KronQ review, Method (1): the
+ * input-side random rotation extended to the output side; Unified
+ * Hessian-Guided PTQ, Background / Transformations: randomised Hadamard
+ * transforms are orthogonal and preserve the layer output).  Element a*p + b
+ * of a vector is (row a of Q_m, row b of H_p).
+ *
+ *   axis == KQ_AXIS_ROWS : M <- T . M    (T acts on the row index; T->n == rows)
+ *   axis == KQ_AXIS_COLS : M <- M . T^T  (T acts on the column index; T->n == cols)
+ *   inverse != 0 applies T^T instead of T.
+ * In place on fp32 M [rows, cols], ld >= cols, 16-byte aligned, ld % 4 == 0.
+ * Limits: 1 <= m <= 64, 0 <= log2_p <= 15, n <= 65536; T->signs device
+ * fp32[n] of +-1; T->Qm device fp32[m*m] row-major orthogonal, may be NULL
+ * only when m == 1.  BiIP of a layer is:
+ *   W:   kq_rotate(W,  KQ_AXIS_COLS, U) then kq_rotate(W, KQ_AXIS_ROWS, V)
+ *   H_X: kq_rotate(HX, KQ_AXIS_COLS, U) then kq_rotate(HX, KQ_AXIS_ROWS, U)
+ *   H_G: kq_rotate(HG, KQ_AXIS_COLS, V) then kq_rotate(HG, KQ_AXIS_ROWS, V)
+ * ------------------------------------------------------------------------ */
+typedef struct kq_rht {
+  int64_t n;
+  int32_t log2_p;
+  int32_t m;
+  const float* signs;
+  const float* Qm;
+} kq_rht;
+
+kq_status kq_rotate(float* M, int64_t rows, int64_t cols, int64_t ld, int axis,
+                    const kq_rht* T, int inverse, kq_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * kq_chol_inv - damping, dead columns and Cholesky factor of the inverse (a6).
+ *
+ * GPTQ solver set-up on H (KronQ review, Prior limitations: GPTQ's
+ * column-wise OBS update uses H_X as the Hessian proxy).  A column j with
+ * H[j][j] == 0 is dead: dead_mask[j] = 1 and its diagonal becomes 1.  Then
+ * lambda = damp_frac * mean(diag) is added to the diagonal and the upper
+ * triangular Uc with Uc^T Uc = (H + lambda I)^-1 is formed, via H = R R^T
+ * (R upper) and Uc = R^-1, in fp64 throughout; Uc is written as fp32 with
+ * zeros below the diagonal.
+ *
+ *   H         fp32 [n, n] symmetric (only the upper triangle is read), ldh >= n.
+ *   Uc        fp32 [n, n], lduc >= n.   dead_mask uint8[n] or NULL.
+ *   ws        kq_chol_inv_workspace_size(n) bytes.
+ *   info      KQ_ERR_NOT_PD (index = column whose pivot failed),
+ *             KQ_ERR_NONFINITE (index = row holding NaN/Inf).
+ * Limits: 1 <= n <= 65536, 0 <= damp_frac.
+ * ------------------------------------------------------------------------ */
+size_t kq_chol_inv_workspace_size(int64_t n);
+kq_status kq_chol_inv(const float* H, int64_t n, int64_t ldh, float damp_frac,
+                      float* Uc, int64_t lduc, uint8_t* dead_mask,
+                      void* ws, size_t ws_bytes, int32_t* info, kq_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * kq_quantize_layer - blocked column-wise OBS quantization (a7, a8, a9).
+ *
+ * For each block [i, i+block) and each column j in it (natural order):
+ *   q = clamp(rint(w_j / scale + zero), 0, 2^bits - 1),  w_hat = scale (q - zero),
+ *   e = (w_j - w_hat) / Uc[j][j],  W[:, j+1:i+block] -= e Uc[j, j+1:i+block];
+ * after the block W[:, i+block:] -= E Uc[i:i+block, i+block:] (the lazy
+ * trailing update).  H_G does not enter: it cancels from the update (KronQ
+ * review, Method (1), Proposition 1).  Grid: asymmetric min/max, scale =
+ * (max - min) / (2^bits - 1), zero = rint(-min / scale) (degenerate range:
+ * scale 1, zero rint(-min)); per output channel (group == 0, fitted on the
+ * initial rows) or per `group` columns (fitted on the current values when the
+ * group's first column is reached).  Dead columns (dead_mask[j] != 0) are
+ * zeroed first.  All arithmetic is IEEE fp32 (true division, rint half-even).
+ *
+ *   W        fp32 [d_out, d_in] rotated weights, ldw >= d_in (read only).
+ *   Uc       fp32 [d_in, d_in] from kq_chol_inv, lduc >= d_in.
+ *   bits     2..8.   group 0 or a divisor of block that is a multiple of 32.
+ *   block    128 (the only block size built).
+ *   gemm_mode KQ_GEMM_FP32 (SIMT fp32) or KQ_GEMM_3XTF32 (tensor cores).
+ *   codes    uint8 [d_out, d_in], ldq >= d_in.
+ *   scales, zeros  fp32 [d_out, n_groups], n_groups = 1 or ceil(d_in / group).
+ *   W_hat    fp32 [d_out, d_in] dequantized weights (rotated coordinates),
+ *            ldwh >= d_in; also used as the running copy of W.
+ *   ws       kq_quantize_layer_workspace_size(d_out, d_in, block) bytes.
+ *   info     KQ_ERR_NONFINITE (index = row) if W holds NaN/Inf.
+ * Limits: 1 <= d_out, 1 <= d_in <= 65536.
+ * ------------------------------------------------------------------------ */
+size_t kq_quantize_layer_workspace_size(int64_t d_out, int64_t d_in, int block);
+kq_status kq_quantize_layer(const float* W, int64_t d_out, int64_t d_in, int64_t ldw,
+                            const float* Uc, int64_t lduc, const uint8_t* dead_mask,
+                            int bits, int group, int block, int gemm_mode,
+                            uint8_t* codes, int64_t ldq, float* scales, float* zeros,
+                            float* W_hat, int64_t ldwh,
+                            void* ws, size_t ws_bytes, int32_t* info, kq_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * kq_kron_loss - Kronecker loss (a10).
+ *
+ * loss = tr(dW H_X dW^T H_G), dW = W - W_hat (KronQ review, Background: the
+ * layer Hessian H ~ H_X kron H_G; Unified Hessian-Guided PTQ, Appendix A.1:
+ * the Kronecker-weighted norm as a trace).  H_G == NULL means the identity
+ * (the H_X-only GPTQ objective).  Products in fp32, final sum in fp64.
+ *
+ *   W, W_hat fp32 [d_out, d_in];  H_X fp32 [d_in, d_in];  H_G fp32 [d_out, d_out].
+ *   loss     device fp64[1].
+ *   ws       kq_kron_loss_workspace_size(d_out, d_in) bytes.
+ * ------------------------------------------------------------------------ */
+size_t kq_kron_loss_workspace_size(int64_t d_out, int64_t d_in);
+kq_status kq_kron_loss(const float* W, int64_t ldw, const float* W_hat, int64_t ldwh,
+                       int64_t d_out, int64_t d_in,
+                       const float* H_X, int64_t ldhx, const float* H_G, int64_t ldhg,
+                       double* loss, void* ws, size_t ws_bytes, kq_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * kq_allocate_bits - sublayer bit allocation (a11).  HOST memory, synchronous.
+ *
+ * Greedy upgrade ordering by the trace sensitivity (KronQ review, Method (2)
+ * and Comparison / Table 6 ablation).  Every sublayer starts at the lowest
+ * choice; the integer budget is floor(sum(n_params) * (avg_bits - lowest)
+ * * (1 + 1e-12)) in bit*parameter units; sublayers are visited by descending
+ * score (ties: lower index first) and each takes the highest choice whose
+ * extra cost n_params[k] * (b - lowest) still fits the remaining budget.
+ *
+ *   sens[n_layers], n_params[n_layers] (> 0), choices[n_choices] distinct,
+ *   in 1..16; bits_out[n_layers].  All host pointers.
+ * ------------------------------------------------------------------------ */
+kq_status kq_allocate_bits(const double* sens, const int64_t* n_params, int n_layers,
+                           const int* choices, int n_choices, double avg_bits,
+                           int* bits_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KRONQ_H */

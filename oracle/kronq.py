@@ -174,9 +174,12 @@ def damp_and_dead(H, damp_frac=0.01):
     Reading R6 (GPTQ convention): a column j with H[j, j] == 0 carries no
     signal; its diagonal is set to 1 (and its weights are zeroed in the
     solver).  The damping lambda = damp_frac * mean(diag H) is taken after that
-    replacement and added to every diagonal entry.
+    replacement and added to every diagonal entry.  H is symmetric by
+    definition; a computed H can differ from its transpose by rounding, so the
+    upper triangle is taken as the definition (mirrored onto the lower).
     """
-    H = np.array(H, dtype=np.float64, copy=True)
+    H = np.asarray(H, dtype=np.float64)
+    H = np.triu(H) + np.triu(H, 1).T
     dead = np.diag(H) == 0
     idx = np.flatnonzero(dead)
     H[idx, idx] = 1.0

@@ -1,0 +1,273 @@
+"""ctypes binding of libkronq.so (the C ABI declared in include/kronq.h).
+
+Argument marshalling only: every computation runs in the library's CUDA
+kernels.  Each wrapper takes torch CUDA tensors, checks dtype, device and
+layout, passes raw pointers, leading dimensions and the current CUDA stream,
+and raises KronqError on a non-OK status.  The library is loaded from the
+package directory; if it is missing the import fails loudly (there is no
+other implementation of these operations in the package).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkronq.so")
+
+KQ_OK = 0
+STATUS_NAMES = {
+    0: "KQ_OK", 1: "KQ_ERR_INVALID_ARG", 2: "KQ_ERR_UNSUPPORTED_SHAPE", 3: "KQ_ERR_ALIGNMENT",
+    4: "KQ_ERR_WORKSPACE", 5: "KQ_ERR_CUDA", 6: "KQ_ERR_NOT_PD", 7: "KQ_ERR_NONFINITE", 8: "KQ_ERR_TIMEOUT",
+}
+KQ_AXIS_ROWS, KQ_AXIS_COLS = 0, 1
+KQ_GEMM_FP32, KQ_GEMM_3XTF32 = 0, 1
+
+# Every symbol the header declares.
+EXPORTS = (
+    "kq_status_string", "kq_last_error", "kq_version", "kq_launch_count",
+    "kq_accum_cov_workspace_size", "kq_accum_cov",
+    "kq_sensitivity",
+    "kq_rotate",
+    "kq_chol_inv_workspace_size", "kq_chol_inv",
+    "kq_quantize_layer_workspace_size", "kq_quantize_layer",
+    "kq_kron_loss_workspace_size", "kq_kron_loss",
+    "kq_allocate_bits",
+)
+
+
+class KronqError(RuntimeError):
+    def __init__(self, status, detail, where=""):
+        self.status = int(status)
+        self.name = STATUS_NAMES.get(int(status), f"status {status}")
+        super().__init__(f"{where}: {self.name}: {detail}" if where else f"{self.name}: {detail}")
+
+
+class kq_rht(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_int64), ("log2_p", ctypes.c_int32), ("m", ctypes.c_int32),
+                ("signs", ctypes.c_void_p), ("Qm", ctypes.c_void_p)]
+
+
+_i64, _i32, _f32, _f64, _vp, _sz = (ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_double,
+                                    ctypes.c_void_p, ctypes.c_size_t)
+
+_SIGS = {
+    "kq_status_string": (ctypes.c_char_p, [_i32]),
+    "kq_last_error": (ctypes.c_char_p, []),
+    "kq_version": (_i32, []),
+    "kq_launch_count": (ctypes.c_ulonglong, []),
+    "kq_accum_cov_workspace_size": (_sz, [_i64, _i64]),
+    "kq_accum_cov": (_i32, [_vp, _i64, _i64, _i64, _vp, _i64, _f32, _i32, _vp, _sz, _vp, _vp]),
+    "kq_sensitivity": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _vp, _vp]),
+    "kq_rotate": (_i32, [_vp, _i64, _i64, _i64, _i32, ctypes.POINTER(kq_rht), _i32, _vp]),
+    "kq_chol_inv_workspace_size": (_sz, [_i64]),
+    "kq_chol_inv": (_i32, [_vp, _i64, _i64, _f32, _vp, _i64, _vp, _vp, _sz, _vp, _vp]),
+    "kq_quantize_layer_workspace_size": (_sz, [_i64, _i64, _i32]),
+    "kq_quantize_layer": (_i32, [_vp, _i64, _i64, _i64, _vp, _i64, _vp, _i32, _i32, _i32, _i32,
+                                 _vp, _i64, _vp, _vp, _vp, _i64, _vp, _sz, _vp, _vp]),
+    "kq_kron_loss_workspace_size": (_sz, [_i64, _i64]),
+    "kq_kron_loss": (_i32, [_vp, _i64, _vp, _i64, _i64, _i64, _vp, _i64, _vp, _i64, _vp, _vp, _sz, _vp]),
+    "kq_allocate_bits": (_i32, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), _i32,
+                                ctypes.POINTER(ctypes.c_int), _i32, _f64, ctypes.POINTER(ctypes.c_int)]),
+}
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libkronq.so (once) and declare every entry point's signature."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `python -m post_weight_quantization_syrk_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in _SIGS.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(status, where):
+    if status != KQ_OK:
+        detail = load().kq_last_error().decode(errors="replace")
+        raise KronqError(status, detail, where)
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _mat(t, dtype, name):
+    """Row-major matrix check; returns the leading dimension."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name} must be a 2-D row-major tensor (unit column stride)")
+    return t.stride(0) if t.shape[0] > 1 else max(t.shape[1], t.stride(0))
+
+
+def _buf(ws):
+    return (ctypes.c_void_p(0), 0) if ws is None else (ctypes.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size())
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """A device byte buffer for a kq_* workspace (torch allocations are 256-byte aligned)."""
+    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+def new_info(device) -> torch.Tensor:
+    return torch.zeros(1, dtype=torch.int32, device=device)
+
+
+def check_info(info: torch.Tensor, where: str = "device"):
+    """Raise KronqError if a kernel recorded an error in `info` (synchronises)."""
+    v = int(info.item())
+    if v != 0:
+        code, index = (v >> 24) & 0xFF, v & 0xFFFFFF
+        raise KronqError(code, f"recorded by a kernel at index {index}", where)
+
+
+# ----------------------------------------------------------------- wrappers
+
+def kq_version() -> int:
+    return int(load().kq_version())
+
+
+def kq_launch_count() -> int:
+    return int(load().kq_launch_count())
+
+
+def kq_status_string(s: int) -> str:
+    return load().kq_status_string(int(s)).decode()
+
+
+def kq_accum_cov_workspace_size(n: int, d: int) -> int:
+    return int(load().kq_accum_cov_workspace_size(int(n), int(d)))
+
+
+def kq_accum_cov(A, C, alpha, accumulate=False, ws=None, info=None, stream=None):
+    """C (+)= alpha * A^T A, A bf16 [n, d], C fp32 [d, d]."""
+    lda = _mat(A, torch.bfloat16, "A")
+    ldc = _mat(C, torch.float32, "C")
+    n, d = A.shape
+    if C.shape != (d, d):
+        raise ValueError("C must be [d, d]")
+    if ws is None:
+        ws = workspace(kq_accum_cov_workspace_size(n, d), A.device)
+    wp, wb = _buf(ws)
+    _check(load().kq_accum_cov(_ptr(A), n, d, lda, _ptr(C), ldc, float(alpha), int(bool(accumulate)),
+                               wp, wb, _ptr(info), _stream(stream)), "kq_accum_cov")
+
+
+def kq_sensitivity(H_X, H_G, out3, stream=None):
+    """out3 (fp64[3]) = tr H_X, tr H_G, their product."""
+    ldx = _mat(H_X, torch.float32, "H_X")
+    ldg = _mat(H_G, torch.float32, "H_G")
+    if out3.dtype != torch.float64 or out3.numel() < 3 or not out3.is_cuda:
+        raise TypeError("out3 must be a CUDA float64 tensor of 3 elements")
+    _check(load().kq_sensitivity(_ptr(H_X), H_X.shape[0], ldx, _ptr(H_G), H_G.shape[0], ldg, _ptr(out3),
+                                 _stream(stream)), "kq_sensitivity")
+
+
+class RHT:
+    """Device-side parameters of T = (Q_m kron H_p / sqrt(p)) diag(signs)."""
+
+    def __init__(self, n, log2_p, m, signs, Qm=None):
+        if signs.dtype != torch.float32 or not signs.is_cuda or signs.numel() != n:
+            raise TypeError("signs must be a CUDA float32 tensor of n elements")
+        if m > 1 and (Qm is None or Qm.dtype != torch.float32 or not Qm.is_cuda or Qm.numel() != m * m):
+            raise TypeError("Qm must be a CUDA float32 [m, m] tensor when m > 1")
+        self.signs = signs.contiguous()
+        self.Qm = None if Qm is None else Qm.contiguous()
+        self.c = kq_rht(int(n), int(log2_p), int(m), self.signs.data_ptr(),
+                        0 if self.Qm is None else self.Qm.data_ptr())
+
+
+def kq_rotate(M, axis, T: RHT, inverse=False, stream=None):
+    """In place: axis ROWS: M <- T M; axis COLS: M <- M T^T (T^T when inverse)."""
+    ld = _mat(M, torch.float32, "M")
+    _check(load().kq_rotate(_ptr(M), M.shape[0], M.shape[1], ld, int(axis), ctypes.byref(T.c), int(bool(inverse)),
+                            _stream(stream)), "kq_rotate")
+
+
+def kq_chol_inv_workspace_size(n: int) -> int:
+    return int(load().kq_chol_inv_workspace_size(int(n)))
+
+
+def kq_chol_inv(H, damp_frac, Uc, dead_mask=None, ws=None, info=None, stream=None):
+    ldh = _mat(H, torch.float32, "H")
+    ldu = _mat(Uc, torch.float32, "Uc")
+    n = H.shape[0]
+    if dead_mask is not None and (dead_mask.dtype != torch.uint8 or dead_mask.numel() < n):
+        raise TypeError("dead_mask must be uint8 [n]")
+    if ws is None:
+        ws = workspace(kq_chol_inv_workspace_size(n), H.device)
+    wp, wb = _buf(ws)
+    _check(load().kq_chol_inv(_ptr(H), n, ldh, float(damp_frac), _ptr(Uc), ldu, _ptr(dead_mask), wp, wb,
+                              _ptr(info), _stream(stream)), "kq_chol_inv")
+
+
+def kq_quantize_layer_workspace_size(d_out: int, d_in: int, block: int = 128) -> int:
+    return int(load().kq_quantize_layer_workspace_size(int(d_out), int(d_in), int(block)))
+
+
+def kq_quantize_layer(W, Uc, dead_mask, bits, group, codes, scales, zeros, W_hat, block=128,
+                      gemm_mode=KQ_GEMM_FP32, ws=None, info=None, stream=None):
+    ldw = _mat(W, torch.float32, "W")
+    ldu = _mat(Uc, torch.float32, "Uc")
+    ldq = _mat(codes, torch.uint8, "codes")
+    ldh = _mat(W_hat, torch.float32, "W_hat")
+    d_out, d_in = W.shape
+    ng = 1 if not group else -(-d_in // group)
+    for t, nm in ((scales, "scales"), (zeros, "zeros")):
+        if t.dtype != torch.float32 or not t.is_contiguous() or t.numel() < d_out * ng:
+            raise TypeError(f"{nm} must be contiguous float32 [d_out, n_groups]")
+    if ws is None:
+        ws = workspace(kq_quantize_layer_workspace_size(d_out, d_in, block), W.device)
+    wp, wb = _buf(ws)
+    _check(load().kq_quantize_layer(_ptr(W), d_out, d_in, ldw, _ptr(Uc), ldu, _ptr(dead_mask), int(bits), int(group),
+                                    int(block), int(gemm_mode), _ptr(codes), ldq, _ptr(scales), _ptr(zeros),
+                                    _ptr(W_hat), ldh, wp, wb, _ptr(info), _stream(stream)), "kq_quantize_layer")
+
+
+def kq_kron_loss_workspace_size(d_out: int, d_in: int) -> int:
+    return int(load().kq_kron_loss_workspace_size(int(d_out), int(d_in)))
+
+
+def kq_kron_loss(W, W_hat, H_X, H_G, loss, ws=None, stream=None):
+    ldw = _mat(W, torch.float32, "W")
+    ldh = _mat(W_hat, torch.float32, "W_hat")
+    ldx = _mat(H_X, torch.float32, "H_X")
+    ldg = 0 if H_G is None else _mat(H_G, torch.float32, "H_G")
+    d_out, d_in = W.shape
+    if loss.dtype != torch.float64 or not loss.is_cuda:
+        raise TypeError("loss must be a CUDA float64 tensor")
+    if ws is None:
+        ws = workspace(kq_kron_loss_workspace_size(d_out, d_in), W.device)
+    wp, wb = _buf(ws)
+    _check(load().kq_kron_loss(_ptr(W), ldw, _ptr(W_hat), ldh, d_out, d_in, _ptr(H_X), ldx, _ptr(H_G), ldg,
+                               _ptr(loss), wp, wb, _stream(stream)), "kq_kron_loss")
+
+
+def kq_allocate_bits(sens, n_params, choices=(2, 3, 4), avg_bits=3.0):
+    """Host call: greedy bit allocation; returns a list of ints."""
+    k = len(sens)
+    s = (ctypes.c_double * k)(*[float(x) for x in sens])
+    n = (ctypes.c_int64 * k)(*[int(x) for x in n_params])
+    c = (ctypes.c_int * len(choices))(*[int(x) for x in choices])
+    out = (ctypes.c_int * max(k, 1))()
+    _check(load().kq_allocate_bits(s, n, k, c, len(choices), float(avg_bits), out), "kq_allocate_bits")
+    return [int(out[i]) for i in range(k)]

@@ -1,0 +1,129 @@
+// kq_kron_loss: Kronecker loss tr(dW H_X dW^T H_G), dW = W - W_hat (a10).
+//
+// KronQ review (romaanj.github.io/reviews/kronq), Background: H ~ H_X kron H_G;
+// Unified Hessian-Guided PTQ (hub.valency.io/works/W_r72x54u6), Appendix A.1:
+// the Kronecker-weighted norm of a perturbation is a trace of this form.
+// Using the symmetry of H_G, tr(dW H_X dW^T H_G) = sum_ij (dW H_X)_ij (H_G dW)_ij.
+// Each CTA forms one 64x64 tile of both products (dW is formed on the fly from
+// W and W_hat), reduces their elementwise product to an fp64 partial, and a
+// final one-CTA pass sums the partials in a fixed order (deterministic).
+#include "kq_internal.cuh"
+
+namespace {
+
+constexpr int T = 64, TK = 32;
+
+// acc[4][4] += sum_k A(r,k) B(k,c) over k in [0, K), tile rows r0.., cols c0..
+// A(r,k) = fa(r, k), B(k,c) = fb(k, c), both fp32 loaded through smem.
+template <typename FA, typename FB>
+__device__ __forceinline__ void tile_product(float (&acc)[4][4], int64_t K, FA fa, FB fb) {
+  __shared__ __align__(16) float As[TK][T];
+  __shared__ __align__(16) float Bs[TK][T];
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  for (int64_t k0 = 0; k0 < K; k0 += TK) {
+    for (int idx = threadIdx.x; idx < TK * T; idx += 256) {
+      int r = idx % T, k = idx / T;
+      As[k][r] = (k0 + k < K) ? fa(r, k0 + k) : 0.f;
+    }
+    for (int idx = threadIdx.x; idx < TK * T; idx += 256) {
+      int c = idx % T, k = idx / T;
+      Bs[k][c] = (k0 + k < K) ? fb(k0 + k, c) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int k = 0; k < TK; ++k) {
+      float4 a = *reinterpret_cast<const float4*>(&As[k][ty * 4]);
+      float4 b = *reinterpret_cast<const float4*>(&Bs[k][tx * 4]);
+      float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+}
+
+__global__ void __launch_bounds__(256) loss_tile_kernel(const float* __restrict__ W, int64_t ldw,
+                                                        const float* __restrict__ Wh, int64_t ldwh, int64_t d_out,
+                                                        int64_t d_in, const float* __restrict__ HX, int64_t ldhx,
+                                                        const float* __restrict__ HG, int64_t ldhg,
+                                                        double* __restrict__ partial) {
+  const int64_t r0 = (int64_t)blockIdx.y * T, c0 = (int64_t)blockIdx.x * T;
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  auto D = [&](int64_t r, int64_t c) -> float {
+    return (r < d_out && c < d_in) ? W[r * ldw + c] - Wh[r * ldwh + c] : 0.f;
+  };
+  float A[4][4], B[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) A[i][j] = B[i][j] = 0.f;
+  // A = dW H_X (K = d_in)
+  tile_product(A, d_in, [&](int r, int64_t k) { return D(r0 + r, k); },
+               [&](int64_t k, int c) { return (c0 + c < d_in) ? HX[k * ldhx + c0 + c] : 0.f; });
+  if (HG) {
+    // B = H_G dW (K = d_out)
+    tile_product(B, d_out, [&](int r, int64_t k) { return (r0 + r < d_out) ? HG[(r0 + r) * ldhg + k] : 0.f; },
+                 [&](int64_t k, int c) { return D(k, c0 + c); });
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) B[i][j] = D(r0 + ty * 4 + i, c0 + tx * 4 + j);
+  }
+  double s = 0.0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) s += (double)A[i][j] * (double)B[i][j];
+  __shared__ double red[256];
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) partial[(int64_t)blockIdx.y * gridDim.x + blockIdx.x] = red[0];
+}
+
+__global__ void sum_kernel(const double* __restrict__ partial, int64_t n, double* __restrict__ out) {
+  __shared__ double red[1024];
+  double s = 0.0;
+  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) s += partial[i];
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *out = red[0];
+}
+
+}  // namespace
+
+extern "C" size_t kq_kron_loss_workspace_size(int64_t d_out, int64_t d_in) {
+  if (d_out < 1 || d_in < 1) return 0;
+  return kq::align_up((size_t)kq::cdiv(d_out, T) * kq::cdiv(d_in, T) * sizeof(double), 256);
+}
+
+extern "C" kq_status kq_kron_loss(const float* W, int64_t ldw, const float* W_hat, int64_t ldwh, int64_t d_out,
+                                  int64_t d_in, const float* H_X, int64_t ldhx, const float* H_G, int64_t ldhg,
+                                  double* loss, void* ws, size_t ws_bytes, kq_stream_t stream) {
+  if (!W || !W_hat || !H_X || !loss) return kq::fail(KQ_ERR_INVALID_ARG, "kq_kron_loss: NULL pointer");
+  if (d_out < 1 || d_in < 1) return kq::fail(KQ_ERR_INVALID_ARG, "kq_kron_loss: sizes must be >= 1");
+  if (ldw < d_in || ldwh < d_in || ldhx < d_in || (H_G && ldhg < d_out))
+    return kq::fail(KQ_ERR_INVALID_ARG, "kq_kron_loss: leading dimension too small");
+  if (!ws || !kq::aligned(ws, 256) || ws_bytes < kq_kron_loss_workspace_size(d_out, d_in))
+    return kq::fail(KQ_ERR_WORKSPACE, "kq_kron_loss: workspace too small or not 256-byte aligned");
+  if (kq::cdiv(d_out, T) > 65535) return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_kron_loss: d_out too large");
+  cudaStream_t st = (cudaStream_t)stream;
+  double* partial = static_cast<double*>(ws);
+  dim3 grid((unsigned)kq::cdiv(d_in, T), (unsigned)kq::cdiv(d_out, T));
+  loss_tile_kernel<<<grid, 256, 0, st>>>(W, ldw, W_hat, ldwh, d_out, d_in, H_X, ldhx, H_G, ldhg, partial);
+  KQ_TRY(kq::launch_check("kq_kron_loss tiles"));
+  sum_kernel<<<1, 1024, 0, st>>>(partial, (int64_t)grid.x * grid.y, loss);
+  KQ_TRY(kq::launch_check("kq_kron_loss sum"));
+  kq::clear_error();
+  return KQ_OK;
+}

@@ -1,0 +1,117 @@
+"""One linear layer through the whole KronQ path, driven through the C ABI.
+
+Order of the steps (KronQ paper page, Abstract; KronQ review, Method):
+  H_X, H_G (covariance SYRKs) -> sensitivity -> BiIP rotations of W, H_X, H_G
+  -> damped Cholesky factor of the inverse of H_X' (once per layer)
+  -> for each bit-width: blocked OBS quantization + Kronecker loss.
+H_G is computed once and reused across bit-widths, as the authors' reply on
+the paper page describes.  All buffers are allocated once per layer shape
+(torch provides device memory and the stream); every computation is a kq_*
+call into libkronq.so.
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import torch
+
+from . import _lib as K
+
+
+@dataclasses.dataclass
+class BitResult:
+    bits: int
+    group: int
+    codes: torch.Tensor
+    scales: torch.Tensor
+    zeros: torch.Tensor
+    W_hat: torch.Tensor
+    loss: torch.Tensor      # fp64[1] device
+
+
+class LayerQuantizer:
+    """Device buffers for one (d_out, d_in) layer and the calls that fill them."""
+
+    def __init__(self, d_out, d_in, device="cuda", block=128, gemm_mode=K.KQ_GEMM_FP32):
+        self.d_out, self.d_in, self.block, self.gemm_mode = d_out, d_in, block, gemm_mode
+        dev = torch.device(device)
+        self.device = dev
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.H_X = torch.empty((d_in, d_in), **f32)
+        self.H_G = torch.empty((d_out, d_out), **f32)
+        self.Wp = torch.empty((d_out, d_in), **f32)
+        self.Uc = torch.empty((d_in, d_in), **f32)
+        self.dead = torch.zeros(d_in, dtype=torch.uint8, device=dev)
+        self.sens = torch.zeros(3, dtype=torch.float64, device=dev)
+        self.info = K.new_info(dev)
+        self._ws = K.workspace(256, dev)
+        self._ws_bytes = 256
+
+    def workspace(self, nbytes):
+        """One scratch buffer shared by the calls (they run in stream order)."""
+        if nbytes > self._ws_bytes:
+            self._ws = K.workspace(nbytes, self.device)
+            self._ws_bytes = nbytes
+        return self._ws
+
+    def alloc_result(self, bits, group):
+        ng = 1 if not group else -(-self.d_in // group)
+        dev = self.device
+        return BitResult(bits, group,
+                         torch.empty((self.d_out, self.d_in), dtype=torch.uint8, device=dev),
+                         torch.empty((self.d_out, ng), dtype=torch.float32, device=dev),
+                         torch.empty((self.d_out, ng), dtype=torch.float32, device=dev),
+                         torch.empty((self.d_out, self.d_in), dtype=torch.float32, device=dev),
+                         torch.zeros(1, dtype=torch.float64, device=dev))
+
+    # -- steps -----------------------------------------------------------
+    def statistics(self, X, G, n_total=None, accumulate=False, stream=None):
+        """H_X (+)= X^T X / N, H_G (+)= G^T G / N; sensitivity of the result."""
+        n_total = X.shape[0] if n_total is None else n_total
+        alpha = 1.0 / n_total if n_total else 0.0
+        ws = self.workspace(max(K.kq_accum_cov_workspace_size(X.shape[0], self.d_in),
+                                K.kq_accum_cov_workspace_size(G.shape[0], self.d_out)))
+        K.kq_accum_cov(X, self.H_X, alpha, accumulate, ws, self.info, stream)
+        K.kq_accum_cov(G, self.H_G, alpha, accumulate, ws, self.info, stream)
+
+    def sensitivity(self, stream=None):
+        K.kq_sensitivity(self.H_X, self.H_G, self.sens, stream)
+
+    def rotate(self, W, T_in: K.RHT, T_out: K.RHT, stream=None):
+        """W' = V W U^T, H_X' = U H_X U^T, H_G' = V H_G V^T (in the layer's buffers)."""
+        self.Wp.copy_(W)
+        K.kq_rotate(self.Wp, K.KQ_AXIS_COLS, T_in, False, stream)
+        K.kq_rotate(self.Wp, K.KQ_AXIS_ROWS, T_out, False, stream)
+        K.kq_rotate(self.H_X, K.KQ_AXIS_COLS, T_in, False, stream)
+        K.kq_rotate(self.H_X, K.KQ_AXIS_ROWS, T_in, False, stream)
+        K.kq_rotate(self.H_G, K.KQ_AXIS_COLS, T_out, False, stream)
+        K.kq_rotate(self.H_G, K.KQ_AXIS_ROWS, T_out, False, stream)
+
+    def factor(self, damp_frac=0.01, stream=None):
+        ws = self.workspace(K.kq_chol_inv_workspace_size(self.d_in))
+        K.kq_chol_inv(self.H_X, damp_frac, self.Uc, self.dead, ws, self.info, stream)
+
+    def quantize(self, res: BitResult, stream=None):
+        ws = self.workspace(K.kq_quantize_layer_workspace_size(self.d_out, self.d_in, self.block))
+        K.kq_quantize_layer(self.Wp, self.Uc, self.dead, res.bits, res.group, res.codes, res.scales, res.zeros,
+                            res.W_hat, self.block, self.gemm_mode, ws, self.info, stream)
+
+    def loss(self, res: BitResult, stream=None):
+        ws = self.workspace(K.kq_kron_loss_workspace_size(self.d_out, self.d_in))
+        K.kq_kron_loss(self.Wp, res.W_hat, self.H_X, self.H_G, res.loss, ws, stream)
+
+    def run(self, W, X, G, T_in, T_out, settings, damp_frac=0.01, results=None, stream=None):
+        """The whole path; settings = [(bits, group), ...].  Asynchronous."""
+        self.statistics(X, G, stream=stream)
+        self.sensitivity(stream)
+        self.rotate(W, T_in, T_out, stream)
+        self.factor(damp_frac, stream)
+        if results is None:
+            results = [self.alloc_result(b, g) for b, g in settings]
+        for r in results:
+            self.quantize(r, stream)
+            self.loss(r, stream)
+        return results
+
+    def check(self, where="kronq"):
+        K.check_info(self.info, where)

@@ -1,0 +1,140 @@
+"""The C ABI without a GPU: the library loads, exports every declared symbol,
+validates arguments on the host, and its host-only entry point (bit
+allocation) matches the oracle bit for bit."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle as O
+import post_weight_quantization_syrk_b200 as P
+from post_weight_quantization_syrk_b200 import _lib as K
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kronq.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_path():
+    names = declared_functions()
+    for fn in ("kq_accum_cov", "kq_rotate", "kq_chol_inv", "kq_quantize_layer", "kq_kron_loss",
+               "kq_sensitivity", "kq_allocate_bits"):
+        assert fn in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = K.load()
+    names = declared_functions()
+    for n in names:
+        assert hasattr(lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", K.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (kq_\w+)", out))
+    assert set(names) <= exported
+    assert set(K.EXPORTS) == set(names)
+
+
+def test_status_strings_and_version():
+    assert P.kq_version() >= 100
+    for code, name in K.STATUS_NAMES.items():
+        assert P.kq_status_string(code) == name
+
+
+def test_allocation_matches_oracle_bit_exact():
+    rng = np.random.default_rng(0)
+    for _ in range(200):
+        k = int(rng.integers(1, 40))
+        s = rng.uniform(0, 10, k)
+        if rng.random() < 0.3:
+            s = np.round(s)          # ties
+        n = rng.integers(1, 50, k) * int(rng.choice([1, 4096, 4096 * 11008]))
+        avg = float(rng.choice([2.0, 2.5, 3.0, 3.25, 4.0]))
+        ch = (2, 3, 4) if rng.random() < 0.7 else (2, 4, 8)
+        assert P.kq_allocate_bits(s, n, ch, avg) == list(O.allocate_bits(s, n, ch, avg))
+
+
+def test_allocation_llama7b_shapes():
+    """The 7B-shaped model: 32 blocks x (q, k, v, o, gate, up, down)."""
+    rng = np.random.default_rng(1)
+    n = np.array([4096 * 4096] * 4 + [4096 * 11008] * 3, dtype=np.int64)
+    n = np.tile(n, 32)
+    s = rng.lognormal(0, 2, n.size)
+    b = np.array(P.kq_allocate_bits(s, n, (2, 3, 4), 3.0))
+    assert list(b) == list(O.allocate_bits(s, n, (2, 3, 4), 3.0))
+    assert (b * n).sum() <= 3.0 * n.sum()
+    assert (b * n).sum() > 2.99 * n.sum()
+
+
+def test_allocation_validation():
+    with pytest.raises(P.KronqError) as e:
+        P.kq_allocate_bits([1.0], [0], (2, 3))
+    assert e.value.status == 1
+    with pytest.raises(P.KronqError):
+        P.kq_allocate_bits([float("nan")], [5], (2, 3))
+    with pytest.raises(P.KronqError):
+        P.kq_allocate_bits([1.0], [5], (2, 2))
+    assert P.kq_allocate_bits([], [], (2, 3)) == []
+
+
+def _raw():
+    return K.load()
+
+
+def test_host_validation_without_gpu():
+    """Argument checks return before any CUDA call: NULL pointers, bad sizes,
+    misalignment and short workspaces are reported synchronously."""
+    lib = _raw()
+    NULL = ctypes.c_void_p(0)
+    fake = ctypes.c_void_p(0x10000)        # never dereferenced: validation fails first
+    odd = ctypes.c_void_p(0x10002)
+    s = lib.kq_accum_cov(NULL, 10, 8, 8, fake, 8, 1.0, 0, NULL, 0, fake, NULL)
+    assert s == 1
+    s = lib.kq_accum_cov(fake, 10, 0, 8, fake, 8, 1.0, 0, NULL, 0, fake, NULL)
+    assert s == 2
+    s = lib.kq_accum_cov(odd, 10, 8, 8, fake, 8, 1.0, 0, NULL, 0, fake, NULL)
+    assert s == 3
+    assert b"aligned" in lib.kq_last_error()
+    s = lib.kq_accum_cov(fake, 10, 8, 9, fake, 8, 1.0, 0, NULL, 0, fake, NULL)
+    assert s == 3
+    s = lib.kq_chol_inv(fake, 16, 16, ctypes.c_float(0.01), fake, 16, NULL, fake, 8, fake, NULL)
+    assert s == 4                           # workspace too small
+    s = lib.kq_chol_inv(fake, 16, 8, ctypes.c_float(0.01), fake, 16, NULL, fake, 1 << 30, fake, NULL)
+    assert s == 1                           # ldh < n
+    s = lib.kq_chol_inv(fake, 0, 8, ctypes.c_float(0.01), fake, 16, NULL, fake, 1 << 30, fake, NULL)
+    assert s == 2
+    s = lib.kq_quantize_layer(fake, 8, 8, 8, fake, 8, NULL, 1, 0, 128, 0, fake, 8, fake, fake,
+                              ctypes.c_void_p(0x20000), 8, fake, 1 << 20, fake, NULL)
+    assert s == 1                           # bits outside 2..8
+    s = lib.kq_quantize_layer(fake, 8, 8, 8, fake, 8, NULL, 3, 48, 128, 0, fake, 8, fake, fake,
+                              ctypes.c_void_p(0x20000), 8, fake, 1 << 20, fake, NULL)
+    assert s == 2                           # group not a multiple of 32 dividing 128
+    s = lib.kq_quantize_layer(fake, 8, 8, 8, fake, 8, NULL, 3, 0, 64, 0, fake, 8, fake, fake,
+                              ctypes.c_void_p(0x20000), 8, fake, 1 << 20, fake, NULL)
+    assert s == 2                           # block != 128
+    rht = K.kq_rht(12, 2, 3, 0x10000, 0)    # m = 3 needs Qm
+    s = lib.kq_rotate(fake, 4, 12, 12, 1, ctypes.byref(rht), 0, NULL)
+    assert s == 1
+    rht = K.kq_rht(12, 2, 3, 0x10000, 0x10000)
+    s = lib.kq_rotate(fake, 4, 16, 16, 1, ctypes.byref(rht), 0, NULL)
+    assert s == 1                           # n does not match cols
+    rht = K.kq_rht(13, 2, 3, 0x10000, 0x10000)
+    s = lib.kq_rotate(fake, 4, 13, 16, 1, ctypes.byref(rht), 0, NULL)
+    assert s == 2                           # n != m * 2^log2_p
+    s = lib.kq_kron_loss(fake, 8, fake, 8, 8, 8, fake, 8, NULL, 0, fake, NULL, 0, NULL)
+    assert s == 4
+    s = lib.kq_sensitivity(fake, 0, 8, fake, 8, 8, fake, NULL)
+    assert s == 1
+
+
+def test_workspace_sizes():
+    assert P.kq_chol_inv_workspace_size(4096) >= 2 * 4096 * 4096 * 8
+    assert P.kq_quantize_layer_workspace_size(4096, 4096) >= 4096 * 128 * 4
+    assert P.kq_kron_loss_workspace_size(4096, 4096) >= 64 * 64 * 8
+    assert P.kq_chol_inv_workspace_size(0) == 0
