@@ -238,6 +238,36 @@ kq_status kq_kron_loss(const float* W, int64_t ldw, const float* W_hat, int64_t 
                        double* loss, void* ws, size_t ws_bytes, kq_stream_t stream);
 
 /* --------------------------------------------------------------------------
+ * kq_kron_loss_noalloc - kq_kron_loss without a caller workspace.
+ *
+ * The paper has no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory: code embedded in a host application
+ * that owns every device allocation through its own pool, or a latency-bound
+ * loop where the implicit synchronisation of cudaMalloc/cudaFree is not
+ * acceptable.  It computes the same loss with the same kernels as
+ * kq_kron_loss, but keeps the per-tile partial sums in a fixed array inside
+ * the library (static device memory: KQ_KRON_LOSS_NOALLOC_MAX_TILES fp64
+ * values, 512 KiB, held by every GPU that loads the library until the
+ * process exits).  It calls no cudaMalloc, cudaFree or allocating routine.
+ *
+ *   Arguments as kq_kron_loss, without ws/ws_bytes.
+ *   Limit: ceil(d_out / 64) * ceil(d_in / 64) <= KQ_KRON_LOSS_NOALLOC_MAX_TILES
+ *          (e.g. 8192 x 28672 fits); larger layers get KQ_ERR_UNSUPPORTED_SHAPE.
+ *   The stream must belong to the current device.  The first call on a
+ *   device looks up the array's device address (cudaGetSymbolAddress) with
+ *   that device current; make that first call before any stream capture.
+ *   All calls on a device share the one array and it keeps the last call's
+ *   contents (nothing in it needs clearing: each call overwrites the slots
+ *   it reads).  Calls whose work overlaps on the GPU (other streams, other
+ *   host threads) race on the array: serialise them.
+ * ------------------------------------------------------------------------ */
+#define KQ_KRON_LOSS_NOALLOC_MAX_TILES 65536
+kq_status kq_kron_loss_noalloc(const float* W, int64_t ldw, const float* W_hat, int64_t ldwh,
+                               int64_t d_out, int64_t d_in,
+                               const float* H_X, int64_t ldhx, const float* H_G, int64_t ldhg,
+                               double* loss, kq_stream_t stream);
+
+/* --------------------------------------------------------------------------
  * kq_allocate_bits - sublayer bit allocation (a11).  HOST memory, synchronous.
  *
  * Greedy upgrade ordering by the trace sensitivity (KronQ review, Method (2)

@@ -33,7 +33,7 @@ EXPORTS = (
     "kq_rotate",
     "kq_chol_inv_workspace_size", "kq_chol_inv",
     "kq_quantize_layer_workspace_size", "kq_quantize_layer",
-    "kq_kron_loss_workspace_size", "kq_kron_loss",
+    "kq_kron_loss_workspace_size", "kq_kron_loss", "kq_kron_loss_noalloc",
     "kq_allocate_bits",
 )
 
@@ -69,6 +69,7 @@ _SIGS = {
                                  _vp, _i64, _vp, _vp, _vp, _i64, _vp, _sz, _vp, _vp]),
     "kq_kron_loss_workspace_size": (_sz, [_i64, _i64]),
     "kq_kron_loss": (_i32, [_vp, _i64, _vp, _i64, _i64, _i64, _vp, _i64, _vp, _i64, _vp, _vp, _sz, _vp]),
+    "kq_kron_loss_noalloc": (_i32, [_vp, _i64, _vp, _i64, _i64, _i64, _vp, _i64, _vp, _i64, _vp, _vp]),
     "kq_allocate_bits": (_i32, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), _i32,
                                 ctypes.POINTER(ctypes.c_int), _i32, _f64, ctypes.POINTER(ctypes.c_int)]),
 }
@@ -260,6 +261,19 @@ def kq_kron_loss(W, W_hat, H_X, H_G, loss, ws=None, stream=None):
     wp, wb = _buf(ws)
     _check(load().kq_kron_loss(_ptr(W), ldw, _ptr(W_hat), ldh, d_out, d_in, _ptr(H_X), ldx, _ptr(H_G), ldg,
                                _ptr(loss), wp, wb, _stream(stream)), "kq_kron_loss")
+
+
+def kq_kron_loss_noalloc(W, W_hat, H_X, H_G, loss, stream=None):
+    """kq_kron_loss with the library's own fixed scratch (no workspace argument)."""
+    ldw = _mat(W, torch.float32, "W")
+    ldh = _mat(W_hat, torch.float32, "W_hat")
+    ldx = _mat(H_X, torch.float32, "H_X")
+    ldg = 0 if H_G is None else _mat(H_G, torch.float32, "H_G")
+    d_out, d_in = W.shape
+    if loss.dtype != torch.float64 or not loss.is_cuda:
+        raise TypeError("loss must be a CUDA float64 tensor")
+    _check(load().kq_kron_loss_noalloc(_ptr(W), ldw, _ptr(W_hat), ldh, d_out, d_in, _ptr(H_X), ldx, _ptr(H_G), ldg,
+                                       _ptr(loss), _stream(stream)), "kq_kron_loss_noalloc")
 
 
 def kq_allocate_bits(sens, n_params, choices=(2, 3, 4), avg_bits=3.0):

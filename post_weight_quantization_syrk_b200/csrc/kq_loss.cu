@@ -7,6 +7,8 @@
 // Each CTA forms one 64x64 tile of both products (dW is formed on the fly from
 // W and W_hat), reduces their elementwise product to an fp64 partial, and a
 // final one-CTA pass sums the partials in a fixed order (deterministic).
+#include <mutex>
+
 #include "kq_internal.cuh"
 
 namespace {
@@ -124,6 +126,68 @@ extern "C" kq_status kq_kron_loss(const float* W, int64_t ldw, const float* W_ha
   KQ_TRY(kq::launch_check("kq_kron_loss tiles"));
   sum_kernel<<<1, 1024, 0, st>>>(partial, (int64_t)grid.x * grid.y, loss);
   KQ_TRY(kq::launch_check("kq_kron_loss sum"));
+  kq::clear_error();
+  return KQ_OK;
+}
+
+// ---------------------------------------------------------------------------
+// kq_kron_loss_noalloc: the same loss with the per-tile partial sums kept in a
+// fixed device array that belongs to this library, for callers that must not
+// allocate device memory themselves (see kronq.h).
+// ---------------------------------------------------------------------------
+namespace {
+
+// Per-tile partial sums, one fp64 per 64x64 tile; every GPU that loads the
+// library holds this array until the process exits.
+static __device__ __align__(256) double g_loss_partials[KQ_KRON_LOSS_NOALLOC_MAX_TILES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_partials_mutex;
+double* g_partials_ptr[kMaxDevices] = {nullptr};
+
+// Device address of g_loss_partials on the current device, looked up once per
+// device with that device current.  A host-side use of the symbol itself
+// would name a host stand-in, not device memory.
+kq_status partials_address(double** out) {
+  int dev = -1;
+  KQ_TRY(kq::cuda_check(cudaGetDevice(&dev), "kq_kron_loss_noalloc: cudaGetDevice"));
+  if (dev < 0 || dev >= kMaxDevices)
+    return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_kron_loss_noalloc: device ordinal %d above %d", dev, kMaxDevices - 1);
+  std::lock_guard<std::mutex> lock(g_partials_mutex);
+  if (!g_partials_ptr[dev]) {
+    void* p = nullptr;
+    KQ_TRY(kq::cuda_check(cudaGetSymbolAddress(&p, g_loss_partials), "kq_kron_loss_noalloc: cudaGetSymbolAddress"));
+    g_partials_ptr[dev] = static_cast<double*>(p);
+  }
+  *out = g_partials_ptr[dev];
+  return KQ_OK;
+}
+
+}  // namespace
+
+extern "C" kq_status kq_kron_loss_noalloc(const float* W, int64_t ldw, const float* W_hat, int64_t ldwh,
+                                          int64_t d_out, int64_t d_in, const float* H_X, int64_t ldhx,
+                                          const float* H_G, int64_t ldhg, double* loss, kq_stream_t stream) {
+  if (!W || !W_hat || !H_X || !loss) return kq::fail(KQ_ERR_INVALID_ARG, "kq_kron_loss_noalloc: NULL pointer");
+  if (d_out < 1 || d_in < 1) return kq::fail(KQ_ERR_INVALID_ARG, "kq_kron_loss_noalloc: sizes must be >= 1");
+  if (ldw < d_in || ldwh < d_in || ldhx < d_in || (H_G && ldhg < d_out))
+    return kq::fail(KQ_ERR_INVALID_ARG, "kq_kron_loss_noalloc: leading dimension too small");
+  const int64_t tiles = kq::cdiv(d_out, T) * kq::cdiv(d_in, T);
+  if (tiles > KQ_KRON_LOSS_NOALLOC_MAX_TILES)
+    return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE,
+                    "kq_kron_loss_noalloc: ceil(d_out/64) * ceil(d_in/64) = %lld tiles exceeds the fixed scratch of %d "
+                    "tiles; use kq_kron_loss with a caller workspace",
+                    (long long)tiles, (int)KQ_KRON_LOSS_NOALLOC_MAX_TILES);
+  double* partial = nullptr;
+  KQ_TRY(partials_address(&partial));
+  cudaStream_t st = (cudaStream_t)stream;
+  dim3 grid((unsigned)kq::cdiv(d_in, T), (unsigned)kq::cdiv(d_out, T));
+  // Every tile overwrites its own slot and the sum reads only those slots, so
+  // nothing left in the array by an earlier call needs clearing.
+  loss_tile_kernel<<<grid, 256, 0, st>>>(W, ldw, W_hat, ldwh, d_out, d_in, H_X, ldhx, H_G, ldhg, partial);
+  KQ_TRY(kq::launch_check("kq_kron_loss_noalloc tiles"));
+  sum_kernel<<<1, 1024, 0, st>>>(partial, tiles, loss);
+  KQ_TRY(kq::launch_check("kq_kron_loss_noalloc sum"));
   kq::clear_error();
   return KQ_OK;
 }
