@@ -4,96 +4,555 @@
 // activations) and H_G (output gradients, E[g g^T] per the research thread)
 // are the two Kronecker factors of the layer Hessian.
 //
-// Lower-triangle 64x64 tiles only; each tile is mirrored on write-out.
-#include "kq_internal.cuh"
-
+// B200 design (tcgen05 + TMEM + TMA):
+//  * Output tiles are 256x256 blocks of the lower triangle (diagonal blocks
+//    are computed whole, only their lower half is written).  A tile is two
+//    M=128 x N=256 bf16 MMAs per 16 tokens, accumulating in fp32 in TMEM: the
+//    two accumulators fill all 512 TMEM columns of the SM.
+//  * X is [tokens, channels] row-major, so both MMA operands are MN-major:
+//    TMA copies boxes of 64 tokens x 64 channels (128-byte rows, 128-byte
+//    swizzle) and the shared-memory descriptors walk 64-channel atoms with the
+//    leading offset and 8-token groups with the stride offset.  A diagonal tile
+//    loads its channels once and uses them for both operands.
+//  * One persistent CTA per SM walks work units (tile, token split); the
+//    splits of one tile are far apart in the walk while tiles sharing a token
+//    range run side by side, so X streams through L2 about once per wave.
+//  * Warp roles: warp 0 issues TMA (3-stage ring of 64 KB stages guarded by
+//    mbarriers), warp 1 allocates TMEM and one of its threads issues the
+//    MMAs, warps 2-5 drain TMEM with tcgen05.ld and write C (or an fp32
+//    partial tile when the tokens are split; a second kernel then sums the
+//    splits in a fixed order, so results do not depend on scheduling).
+//  * Every mbarrier wait is bounded by a time limit; on expiry the kernel
+//    records KQ_ERR_TIMEOUT, lets its own copies and MMAs drain (again
+//    bounded), frees TMEM and returns.
+#include <cuda.h>
 #include <cuda_bf16.h>
+
+#include <algorithm>
+#include <cmath>
+#include <mutex>
+
+#include "kq_internal.cuh"
 
 namespace {
 
-constexpr int T = 64, TK = 32;
+constexpr int TILE = 256;                 // output tile (rows and columns)
+constexpr int BK = 64;                    // tokens per pipeline stage
+constexpr int STAGES = 3;
+constexpr int BOX_BYTES = 64 * 64 * 2;    // one TMA box: 64 tokens x 64 channels bf16
+constexpr int OPER_BYTES = 4 * BOX_BYTES; // 256 channels x 64 tokens
+constexpr int STAGE_BYTES = 2 * OPER_BYTES;
+constexpr int THREADS = 192;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int ASSUMED_SMS = 148;          // the B200's SM count, used to size splits
+constexpr unsigned long long kTimeoutNs = 4000000000ull;
 
-__device__ __forceinline__ void tri_index(int64_t l, int64_t* ti, int64_t* tj) {
+// Instruction descriptor, kind::f16: D fp32, A/B bf16, both MN-major, M=128, N=256.
+constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) | ((256u >> 3) << 17) |
+                           ((128u >> 4) << 24);
+
+struct Params {
+  int64_t n, d;
+  int T;            // tiles per dimension
+  int num_tiles;    // T (T + 1) / 2
+  int splits;       // token splits per tile
+  int kb_per_split; // 64-token blocks per split
+  int kblocks;      // total 64-token blocks
+  int num_units;    // num_tiles * splits
+  float alpha;
+  int accumulate;
+  float* C;
+  int64_t ldc;
+  float* partial;   // [splits][num_tiles][256][256] when splits > 1
+  int32_t* info;
+};
+
+// ------------------------------------------------------------------ PTX
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity.  Returns false (and sets
+// the CTA's abort flag, recording a timeout once) when the limit expires or
+// another role already aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int32_t* info,
+                                          int where) {
+  unsigned long long t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0) {
+      if (*abort_flag) return false;
+      unsigned long long now = globaltimer();
+      if (it == 0) {
+        t0 = now;
+      } else if (now - t0 > kTimeoutNs) {
+        *abort_flag = 1;
+        kq::report(info, KQ_ERR_TIMEOUT, where);
+        return false;
+      }
+    }
+  }
+}
+
+// Wait used only while draining after an abort: bounded, never reports.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+  unsigned long long t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > kTimeoutNs) return;
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: MN-major operand, 128-byte swizzle.
+// start address >> 4 in bits 0..13; leading byte offset (between 64-element
+// MN atoms) >> 4 in bits 16..29; stride byte offset (between 8-row K groups)
+// >> 4 in bits 32..45; descriptor version 1 in bits 46..47; layout 2
+// (SWIZZLE_128B) in bits 61..63.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
+  const uint64_t lbo = BOX_BYTES >> 4;  // next 64 channels: next TMA box
+  const uint64_t sbo = 1024 >> 4;       // next 8 tokens: 8 rows of 128 bytes
+  return (uint64_t)((addr >> 4) & 0x3FFF) | (lbo << 16) | (sbo << 32) | (1ull << 46) | (2ull << 61);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(IDESC), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tri_index(int64_t l, int* ti, int* tj) {
   int64_t t = (int64_t)((sqrt(8.0 * (double)l + 1.0) - 1.0) * 0.5);
   while (t * (t + 1) / 2 > l) --t;
   while ((t + 1) * (t + 2) / 2 <= l) ++t;
-  *ti = t;
-  *tj = l - t * (t + 1) / 2;
+  *ti = (int)t;
+  *tj = (int)(l - t * (t + 1) / 2);
 }
 
-__global__ void __launch_bounds__(256) syrk_simt_kernel(const __nv_bfloat16* __restrict__ A, int64_t n, int64_t d,
-                                                        int64_t lda, float* __restrict__ C, int64_t ldc, float alpha,
-                                                        int accumulate, int32_t* info) {
-  __shared__ __align__(16) float As[TK][T];
-  __shared__ __align__(16) float Bs[TK][T];
-  int64_t ti, tj;
-  tri_index(blockIdx.x, &ti, &tj);
-  const int64_t i0 = ti * T, j0 = tj * T;
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  float acc[4][4];
+// unit -> (tile, split); units of the same split are adjacent.
+__device__ __forceinline__ void unit_coords(const Params& p, int u, int* ti, int* tj, int* split) {
+  *split = u / p.num_tiles;
+  tri_index(u % p.num_tiles, ti, tj);
+}
+
+// ------------------------------------------------------------------ kernel
+
+__global__ void __launch_bounds__(THREADS, 1) syrk_tc_kernel(const __grid_constant__ CUtensorMap tmap, Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  // bars[0..S): full, [S..2S): empty, [2S]: acc full, [2S+1]: acc empty, [2S+2]: mma drained
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 3);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES);
+  const uint32_t accfull = smem_u32(bars + 2 * STAGES), accempty = smem_u32(bars + 2 * STAGES + 1);
+  const uint32_t drained = smem_u32(bars + 2 * STAGES + 2);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    mbar_init(accfull, 1);
+    mbar_init(accempty, 128);
+    mbar_init(drained, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap)) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(tmem_slot))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_phase[STAGES];
+      bool issued[STAGES];
+      for (int s = 0; s < STAGES; ++s) issued[s] = false;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+        int ti, tj, sp;
+        unit_coords(p, u, &ti, &tj, &sp);
+        const int kb0 = sp * p.kb_per_split;
+        const int kb1 = min(p.kblocks, kb0 + p.kb_per_split);
+        const bool diag = (ti == tj);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.info, 1)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = full0 + 8 * stage;
+          mbar_arrive_expect_tx(fb, diag ? OPER_BYTES : STAGE_BYTES);
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+          const int y = kb * BK;
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+          for (int q = 0; q < 4; ++q) tma_load_2d(sa + q * BOX_BYTES, &tmap, ti * TILE + 64 * q, y, fb);
+          if (!diag) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-  for (int64_t t0 = 0; t0 < n; t0 += TK) {
-    for (int idx = threadIdx.x; idx < TK * T; idx += 256) {
-      int c = idx % T, k = idx / T;
-      bool kin = t0 + k < n;
-      As[k][c] = (kin && i0 + c < d) ? __bfloat162float(A[(t0 + k) * lda + i0 + c]) : 0.f;
-      Bs[k][c] = (kin && j0 + c < d) ? __bfloat162float(A[(t0 + k) * lda + j0 + c]) : 0.f;
+            for (int q = 0; q < 4; ++q) tma_load_2d(sa + OPER_BYTES + q * BOX_BYTES, &tmap, tj * TILE + 64 * q, y, fb);
+          }
+          issued[stage] = true;
+          issued_phase[stage] = phase;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // let this CTA's own copies land before the CTA can exit
+        for (int s = 0; s < STAGES; ++s)
+          if (issued[s]) mbar_drain(full0 + 8 * s, issued_phase[s]);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true, any = false;
+      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+        int ti, tj, sp;
+        unit_coords(p, u, &ti, &tj, &sp);
+        const int kb0 = sp * p.kb_per_split;
+        const int kb1 = min(p.kblocks, kb0 + p.kb_per_split);
+        const bool diag = (ti == tj);
+        if (!mbar_wait(accempty, acc_phase ^ 1u, abort_flag, p.info, 2)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, p.info, 3)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+          const uint32_t sb = diag ? sa : sa + OPER_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint32_t acc = (kb > kb0 || k > 0) ? 1u : 0u;
+            const uint64_t db = smem_desc(sb + k * 2048);
+            mma_bf16(tmem, smem_desc(sa + k * 2048), db, acc);                    // rows 0..127
+            mma_bf16(tmem + 256, smem_desc(sa + 2 * BOX_BYTES + k * 2048), db, acc);  // rows 128..255
+          }
+          any = true;
+          mma_commit(empty0 + 8 * stage);   // stage is free once these MMAs have read it
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(accfull);               // accumulators complete for this unit
+        acc_phase ^= 1u;
+      }
+      if (any) {
+        // every MMA this thread issued has completed before TMEM is released
+        mma_commit(drained);
+        mbar_drain(drained, 0);
+      }
+    }
+  } else {
+    // ---------------- epilogue: warps 2..5 drain TMEM lanes 32*(warp%4) ..
+    const int wq = warp & 3;
+    const int row_in_half = 32 * wq + lane;
+    uint32_t acc_phase = 0;
+    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+      int ti, tj, sp;
+      unit_coords(p, u, &ti, &tj, &sp);
+      if (!mbar_wait(accfull, acc_phase, abort_flag, p.info, 4)) break;
+      tc_fence_after();
+      const int64_t i0 = (int64_t)ti * TILE, j0 = (int64_t)tj * TILE;
+      const bool diag = (ti == tj);
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        const int r = half * 128 + row_in_half;
+        const int64_t gi = i0 + r;
+#pragma unroll 1
+        for (int c0 = 0; c0 < TILE; c0 += 16) {
+          float v[16];
+          tmem_ld16(tmem + ((uint32_t)(32 * wq) << 16) + (uint32_t)(half * 256 + c0), v);
+          if (p.splits > 1) {
+            float* dst = p.partial + (((int64_t)sp * p.num_tiles + (u % p.num_tiles)) * TILE + r) * TILE + c0;
+#pragma unroll
+            for (int q = 0; q < 16; q += 4)
+              *reinterpret_cast<float4*>(dst + q) = make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
+          } else if (gi < p.d && (!diag || c0 <= r)) {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              const int64_t gj = j0 + c0 + q;
+              if (gj >= p.d || gj > gi) continue;
+              float val = p.alpha * v[q];
+              if (p.accumulate) val += p.C[gi * p.ldc + gj];
+              if (!isfinite(val)) kq::report(p.info, KQ_ERR_NONFINITE, gi);
+              p.C[gi * p.ldc + gj] = val;
+              p.C[gj * p.ldc + gi] = val;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(accempty);
+      acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+  }
+}
+
+// Sum the token splits of every lower tile in split order, apply alpha (and
+// the old C when accumulating), write the lower element and its mirror.
+// One CTA per (tile, 32-row band); 32x8 threads; the mirror goes through a
+// shared-memory transpose so both writes are coalesced.
+__global__ void __launch_bounds__(256) split_reduce_kernel(Params p) {
+  __shared__ float t[32][33];
+  const int tile = blockIdx.x / 8;
+  const int band = blockIdx.x % 8;  // 32-row band within the 256-row tile
+  int ti, tj;
+  tri_index(tile, &ti, &tj);
+  const int64_t i0 = (int64_t)ti * TILE + band * 32, j0 = (int64_t)tj * TILE;
+  const int tx = threadIdx.x % 32, ty = threadIdx.x / 32;
+  for (int cb = 0; cb < TILE; cb += 32) {
+    const int64_t gj = j0 + cb + tx;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int rr = ty + 8 * k;
+      const int64_t gi = i0 + rr;
+      float s = 0.f;
+      for (int sp = 0; sp < p.splits; ++sp)
+        s += p.partial[(((int64_t)sp * p.num_tiles + tile) * TILE + band * 32 + rr) * TILE + cb + tx];
+      float val = p.alpha * s;
+      const bool keep = gi < p.d && gj < p.d && gj <= gi;
+      if (keep) {
+        if (p.accumulate) val += p.C[gi * p.ldc + gj];
+        if (!isfinite(val)) kq::report(p.info, KQ_ERR_NONFINITE, gi);
+        p.C[gi * p.ldc + gj] = val;
+      }
+      t[rr][tx] = val;
     }
     __syncthreads();
-#pragma unroll 8
-    for (int k = 0; k < TK; ++k) {
-      float4 a = *reinterpret_cast<const float4*>(&As[k][ty * 4]);
-      float4 b = *reinterpret_cast<const float4*>(&Bs[k][tx * 4]);
-      float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    for (int k = 0; k < 4; ++k) {
+      const int cc = ty + 8 * k;          // column within the 32-wide block
+      const int64_t gj2 = j0 + cb + cc;   // mirror row
+      const int64_t gi2 = i0 + tx;        // mirror column
+      if (gi2 < p.d && gj2 < p.d && gj2 < gi2) p.C[gj2 * p.ldc + gi2] = t[tx][cc];
     }
     __syncthreads();
   }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int64_t gi = i0 + ty * 4 + i;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int64_t gj = j0 + tx * 4 + j;
-      if (gi >= d || gj >= d || gj > gi) continue;
-      float v = alpha * acc[i][j];
-      if (accumulate) v += C[gi * ldc + gj];
-      if (!isfinite(v)) kq::report(info, KQ_ERR_NONFINITE, gi);
-      C[gi * ldc + gj] = v;
-      C[gj * ldc + gi] = v;
+}
+
+__global__ void scale_or_zero_kernel(float* C, int64_t d, int64_t ldc, int accumulate) {
+  // n == 0: C = 0 (overwrite) or unchanged (accumulate)
+  if (accumulate) return;
+  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < d * d;
+       idx += (int64_t)gridDim.x * blockDim.x)
+    C[(idx / d) * ldc + idx % d] = 0.f;
+}
+
+// ------------------------------------------------------------------ host
+
+struct Plan {
+  int T, num_tiles, kblocks, splits, kb_per_split, num_units;
+};
+
+// Token splits per tile: minimise (waves / splits) x full-tile MMA time plus
+// the partial-tile round trip through HBM, with waves counted on 148 SMs.
+Plan make_plan(int64_t n, int64_t d) {
+  Plan pl;
+  pl.T = (int)kq::cdiv(d, TILE);
+  pl.num_tiles = pl.T * (pl.T + 1) / 2;
+  pl.kblocks = (int)kq::cdiv(n, BK);
+  const double tile_s = 2.0 * TILE * TILE * (double)n / (1.4e15 / ASSUMED_SMS);
+  double best = 1e300;
+  int best_s = 1;
+  const int smax = std::min(16, std::max(1, pl.kblocks));
+  for (int s = 1; s <= smax; ++s) {
+    const int per = (int)kq::cdiv(pl.kblocks, s);
+    const int s_eff = (int)kq::cdiv(pl.kblocks, per);
+    if (s_eff != s) continue;
+    const double units = (double)pl.num_tiles * s;
+    const double waves = std::ceil(units / ASSUMED_SMS);
+    double t = waves * tile_s / s;
+    if (s > 1) t += units * TILE * TILE * 8.0 / 6.4e12;
+    if (t < best * 0.995) {
+      best = t;
+      best_s = s;
     }
   }
+  pl.splits = best_s;
+  pl.kb_per_split = (int)kq::cdiv(pl.kblocks, best_s);
+  pl.num_units = pl.num_tiles * best_s;
+  return pl;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+kq_status get_encoder(EncodeTiledFn* fn) {
+  static std::mutex mu;
+  static EncodeTiledFn cached = nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cached) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !f)
+      return kq::fail(KQ_ERR_CUDA, "kq_accum_cov: cuTensorMapEncodeTiled unavailable");
+    cached = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  *fn = cached;
+  return KQ_OK;
 }
 
 }  // namespace
 
 extern "C" size_t kq_accum_cov_workspace_size(int64_t n, int64_t d) {
-  (void)n;
-  (void)d;
-  return 0;
+  if (n <= 0 || d < 1) return 0;
+  Plan pl = make_plan(n, d);
+  if (pl.splits == 1) return 0;
+  return kq::align_up((size_t)pl.num_units * TILE * TILE * sizeof(float), 256);
 }
 
 extern "C" kq_status kq_accum_cov(const uint16_t* A, int64_t n, int64_t d, int64_t lda, float* C, int64_t ldc,
                                   float alpha, int accumulate, void* ws, size_t ws_bytes, int32_t* info,
                                   kq_stream_t stream) {
-  (void)ws;
-  (void)ws_bytes;
   if ((!A && n > 0) || !C || !info) return kq::fail(KQ_ERR_INVALID_ARG, "kq_accum_cov: NULL pointer");
   if (n < 0 || d < 1 || d > 65536) return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_accum_cov: need n >= 0, 1 <= d <= 65536");
+  if (n > ((int64_t)1 << 31) - BK) return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_accum_cov: n above 2^31 - 64");
   if (lda < d || ldc < d) return kq::fail(KQ_ERR_INVALID_ARG, "kq_accum_cov: leading dimension too small");
-  if ((n > 0 && !kq::aligned(A, 16)) || (lda & 7)) return kq::fail(KQ_ERR_ALIGNMENT, "kq_accum_cov: A 16-byte aligned, lda % 8 == 0");
+  if ((n > 0 && !kq::aligned(A, 16)) || (lda & 7))
+    return kq::fail(KQ_ERR_ALIGNMENT, "kq_accum_cov: A 16-byte aligned, lda % 8 == 0");
   if (!isfinite(alpha)) return kq::fail(KQ_ERR_INVALID_ARG, "kq_accum_cov: alpha not finite");
   cudaStream_t st = (cudaStream_t)stream;
-  const int64_t nt = kq::cdiv(d, T);
-  syrk_simt_kernel<<<(unsigned)(nt * (nt + 1) / 2), 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(A), n, d,
-                                                                 lda, C, ldc, alpha, accumulate, info);
+  if (n == 0) {
+    scale_or_zero_kernel<<<256, 256, 0, st>>>(C, d, ldc, accumulate);
+    KQ_TRY(kq::launch_check("kq_accum_cov zero"));
+    kq::clear_error();
+    return KQ_OK;
+  }
+  Plan pl = make_plan(n, d);
+  const size_t need = kq_accum_cov_workspace_size(n, d);
+  if (need && (!ws || !kq::aligned(ws, 256) || ws_bytes < need))
+    return kq::fail(KQ_ERR_WORKSPACE, "kq_accum_cov: workspace of %zu bytes needed", need);
+
+  EncodeTiledFn encode;
+  KQ_TRY(get_encoder(&encode));
+  CUtensorMap tmap;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)n};
+  cuuint64_t strides[1] = {(cuuint64_t)lda * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult cr = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(A), dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return kq::fail(KQ_ERR_CUDA, "kq_accum_cov: cuTensorMapEncodeTiled failed (%d)", (int)cr);
+
+  Params p;
+  p.n = n;
+  p.d = d;
+  p.T = pl.T;
+  p.num_tiles = pl.num_tiles;
+  p.splits = pl.splits;
+  p.kb_per_split = pl.kb_per_split;
+  p.kblocks = pl.kblocks;
+  p.num_units = pl.num_units;
+  p.alpha = alpha;
+  p.accumulate = accumulate ? 1 : 0;
+  p.C = C;
+  p.ldc = ldc;
+  p.partial = static_cast<float*>(ws);
+  p.info = info;
+
+  int dev = 0, sms = ASSUMED_SMS;
+  KQ_TRY(kq::cuda_check(cudaGetDevice(&dev), "kq_accum_cov: cudaGetDevice"));
+  KQ_TRY(kq::cuda_check(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev), "kq_accum_cov: SM count"));
+  KQ_TRY(kq::cuda_check(cudaFuncSetAttribute(syrk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES),
+                        "kq_accum_cov: smem attribute"));
+  const int grid = std::min(pl.num_units, sms);
+  syrk_tc_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(tmap, p);
   KQ_TRY(kq::launch_check("kq_accum_cov"));
+  if (pl.splits > 1) {
+    split_reduce_kernel<<<pl.num_tiles * 8, 256, 0, st>>>(p);
+    KQ_TRY(kq::launch_check("kq_accum_cov reduce"));
+  }
   kq::clear_error();
   return KQ_OK;
 }
