@@ -145,26 +145,33 @@ def run_kronq(a):
     results = [lq.alloc_result(b, g) for b, g in settings]
     stream = torch.cuda.current_stream()
 
-    syrk_events = []
+    stage_events = []   # per timed step: [(name, start_event, end_event), ...]
 
     def step(timed):
-        if timed:
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e2 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            lq.statistics(X, G)   # the two SYRKs (H_X, then H_G)
-            e2.record(stream)
-            syrk_events.append((e0, e2))
-            _ = e1
-        else:
-            lq.statistics(X, G)
+        marks = []
+
+        def mark(name):
+            if timed:
+                e = torch.cuda.Event(enable_timing=True)
+                e.record(stream)
+                marks.append((name, e))
+
+        mark("start")
+        lq.statistics(X, G)   # the two covariance SYRKs (H_X, then H_G)
+        mark("syrk_x2")
         lq.sensitivity()
+        mark("sensitivity")
         lq.rotate(W, T_in, T_out)
+        mark("rotate")
         lq.factor(0.01)
+        mark("chol_inv")
         for r in results:
             lq.quantize(r)
+            mark(f"quantize_w{r.bits}")
             lq.loss(r)
+            mark(f"loss_w{r.bits}")
+        if timed:
+            stage_events.append(marks)
 
     for _ in range(a.warmup):
         step(False)
@@ -193,7 +200,12 @@ def run_kronq(a):
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms_max = float(t.item())
-    syrk_ms = [e0.elapsed_time(e2) / 2.0 for e0, e2 in syrk_events]   # two SYRK launches per step
+    stages = {}
+    for marks in stage_events:
+        for (_, e0), (name, e1) in zip(marks[:-1], marks[1:]):
+            stages.setdefault(name, []).append(e0.elapsed_time(e1))
+    stages_ms = {k: statistics.mean(v) for k, v in stages.items()}
+    syrk_ms = [v / 2.0 for v in stages["syrk_x2"]]   # two SYRK launches per step
     weights_per_step = spec.d_out * spec.d_in * len(settings)
     value = weights_per_step * a.steps * world / (ms_max / 1e3)
 
@@ -219,6 +231,7 @@ def run_kronq(a):
                      "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
                      "peak_source": f"{src} bf16 sustained", "algorithmic_flops_per_launch": flops,
                      "avg_launch_ms": syrk_avg},
+        "stages_ms": stages_ms,
         "gpu_launches": launches,
         "clocks": clk,
         "e2e": e2e,

@@ -66,6 +66,10 @@ WORKLOADS = {
     "mlp_up11008": LayerSpec("mlp_up11008", 11008, 4096, 262144, x_sigma=1.0, g_lo=1e-3),
     "mlp_down11008": LayerSpec("mlp_down11008", 4096, 11008, 262144, x_kind="silu_gated",
                                x_sigma=1.0, g_lo=1e-3),
+    # The attention-projection layer with a quarter of the tokens (profiling
+    # captures: inputs still larger than L2, a few GB on the device).
+    "attn4096_n65536": LayerSpec("attn4096_n65536", 4096, 4096, 65536, w_std=0.02, x_sigma=1.5,
+                                 x_massive=8, g_lo=1e-4),
     # Llama-70B-shaped down projection: 28672 -> 8192, 65536 tokens, Student-t(3).
     "down28672": LayerSpec("down28672", 8192, 28672, 65536, w_std=0.01,
                            x_kind="student_t3", g_lo=1e-4),
