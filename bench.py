@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--workload", default="attn4096")
     ap.add_argument("--bits", default="4,3,2")
     ap.add_argument("--group", type=int, default=0)
+    ap.add_argument("--gemm", default="3xtf32", choices=["3xtf32", "fp32"],
+                    help="precision mode of the solver's trailing update")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     a = ap.parse_args()
@@ -141,7 +143,8 @@ def run_kronq(a):
         return P.RHT(p.n, p.log2_p, p.m, p.signs.to(dev), None if p.Qm is None else p.Qm.to(dev))
 
     T_in, T_out = dev_rht(Ti), dev_rht(To)
-    lq = LayerQuantizer(spec.d_out, spec.d_in, dev)
+    gemm_mode = P.KQ_GEMM_3XTF32 if a.gemm == "3xtf32" else P.KQ_GEMM_FP32
+    lq = LayerQuantizer(spec.d_out, spec.d_in, dev, gemm_mode=gemm_mode)
     results = [lq.alloc_result(b, g) for b, g in settings]
     stream = torch.cuda.current_stream()
 
@@ -226,6 +229,7 @@ def run_kronq(a):
         "config": {"workload": f"{a.workload}: W {spec.d_out}x{spec.d_in}, N={spec.n_tokens} tokens, "
                                f"{'+'.join('W%d' % b for b in bits)} {'per-channel' if not a.group else 'g%d' % a.group}",
                    "layers_per_rank_per_step": 1, "bit_widths": bits, "group": a.group,
+                   "trailing_update": a.gemm,
                    "l2": "inputs larger than L2 (X, G 2 GiB each); no flush"},
         "roofline": {"kernel": "kq_accum_cov (SYRK)", "bound": "tensor", "achieved": achieved, "peak": peak,
                      "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,

@@ -202,7 +202,9 @@ kq_status kq_chol_inv(const float* H, int64_t n, int64_t ldh, float damp_frac,
  *   Uc       fp32 [d_in, d_in] from kq_chol_inv, lduc >= d_in.
  *   bits     2..8.   group 0 or a divisor of block that is a multiple of 32.
  *   block    128 (the only block size built).
- *   gemm_mode KQ_GEMM_FP32 (SIMT fp32) or KQ_GEMM_3XTF32 (tensor cores).
+ *   gemm_mode trailing-update precision: KQ_GEMM_FP32 (SIMT fp32) or
+ *            KQ_GEMM_3XTF32 (tcgen05 tensor cores, operands split into tf32 +
+ *            remainder, fp32-level accuracy).
  *   codes    uint8 [d_out, d_in], ldq >= d_in.
  *   scales, zeros  fp32 [d_out, n_groups], n_groups = 1 or ceil(d_in / group).
  *   W_hat    fp32 [d_out, d_in] dequantized weights (rotated coordinates),
@@ -225,7 +227,8 @@ kq_status kq_quantize_layer(const float* W, int64_t d_out, int64_t d_in, int64_t
  * loss = tr(dW H_X dW^T H_G), dW = W - W_hat (KronQ review, Background: the
  * layer Hessian H ~ H_X kron H_G; Unified Hessian-Guided PTQ, Appendix A.1:
  * the Kronecker-weighted norm as a trace).  H_G == NULL means the identity
- * (the H_X-only GPTQ objective).  Products in fp32, final sum in fp64.
+ * (the H_X-only GPTQ objective).  Products on the tensor cores in 3xTF32
+ * (fp32-level accuracy), elementwise products and sums in fp64.
  *
  *   W, W_hat fp32 [d_out, d_in];  H_X fp32 [d_in, d_in];  H_G fp32 [d_out, d_out].
  *   loss     device fp64[1].

@@ -1,0 +1,383 @@
+// 3xTF32 GEMM on tcgen05 tensor cores, with TMA-fed operands and TMEM
+// accumulators (internal; see kq_gemm.cuh).
+//
+// fp32 accuracy at tensor-core speed: each fp32 operand x is split into its
+// tf32 rounding b = tf32(x) and the remainder s = x - b (exact in fp32), and
+// A B ~ Ab Bb + Ab Bs + As Bb: the dropped As Bs term and the tf32 reading of
+// the remainders are ~2^-22 relative.  The products the path needs (dW H_X,
+// H_G dW for the Kronecker loss, E Uc for the solver's trailing update) lose
+// up to ~60x to cancellation, which rules out plain TF32 or bf16 there.
+//
+// Structure (same as the covariance SYRK): persistent CTAs, one per SM, walk
+// 256 x 256 output tiles; each tile is two M=128 x N=256 accumulators (all
+// 512 TMEM columns).  Warp 0 streams 16-deep K slices of A and B (both
+// K-major, 64-byte swizzle; tcgen05 kind::tf32 produced no result with an
+// MN-major operand on B200 when measured, so callers pass B transposed), big
+// and small parts, through a 3-stage ring; one thread of warp 1 issues 12
+// tcgen05.mma kind::tf32 per stage; warps 2-5 run the epilogue from TMEM.
+// Waits are time-bounded.
+#include <cuda.h>
+
+#include <algorithm>
+
+#include "kq_gemm.cuh"
+#include "kq_tc.cuh"
+
+namespace kq {
+namespace {
+
+using namespace kq::tc;
+
+constexpr int BM = 256, BN = 256, BKF = 16;         // tile rows, cols, K per stage (fp32)
+constexpr int A_BYTES = BM * BKF * 4;               // 16 KB per part
+constexpr int B_BYTES = BN * BKF * 4;               // 16 KB per part
+constexpr int STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;
+constexpr int STAGES = 3;
+constexpr int THREADS = 192;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+
+struct Params {
+  int64_t M, N, K;
+  int tiles_m, tiles_n, num_tiles, kblocks;
+  int a_x0, a_y0, b_x0, b_y0;   // tensor-map coordinates of A(0,0) and B(0,0)
+  int epilogue;
+  float* C;
+  int64_t ldc;
+  const float* src;
+  int64_t ld_src;
+  const uint8_t* dead;
+  const float* other;
+  int64_t ld_other;
+  double* partial;
+  int32_t* info;
+};
+
+// Operand layout in shared memory (K-major): one 16 (k) x 256 TMA box per
+// part and stage, rows of 16 fp32 = 64 B with the 64-byte swizzle; 8-row
+// groups 512 B apart; a 128-row half starts 8 KB on; the second 8-deep K step
+// of the slice starts 32 B on.
+__device__ __forceinline__ uint64_t desc_op(uint32_t addr) { return smem_desc(addr, 16, 512, kSwizzle64); }
+
+struct Maps {
+  CUtensorMap ab, as, bb, bs;
+};
+
+__global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant__ Maps maps, Params p) {
+  constexpr uint32_t IDESC = idesc(kFmtTF32, /*A K-major*/ 0, /*B K-major*/ 0, 128, 256);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 3);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES);
+  const uint32_t accfull = smem_u32(bars + 2 * STAGES), accempty = smem_u32(bars + 2 * STAGES + 1);
+  const uint32_t drained = smem_u32(bars + 2 * STAGES + 2);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    mbar_init(accfull, 1);
+    mbar_init(accempty, 128);
+    mbar_init(drained, 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+    prefetch_map(&maps.ab);
+    prefetch_map(&maps.as);
+    prefetch_map(&maps.bb);
+    prefetch_map(&maps.bs);
+  }
+  if (warp == 1) tmem_alloc<512>(smem_u32(tmem_slot));
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_phase[STAGES];
+      bool issued[STAGES] = {false, false, false};
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        const int m0 = (t / p.tiles_n) * BM, n0 = (t % p.tiles_n) * BN;
+        for (int kb = 0; kb < p.kblocks; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.info, 11)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = full0 + 8 * stage;
+          mbar_arrive_expect_tx(fb, STAGE_BYTES);
+          const uint32_t s0 = smem_u32(smem + stage * STAGE_BYTES);
+          const int k0 = kb * BKF;
+          tma_load_2d(s0, &maps.ab, p.a_x0 + k0, p.a_y0 + m0, fb);
+          tma_load_2d(s0 + A_BYTES, &maps.as, p.a_x0 + k0, p.a_y0 + m0, fb);
+          tma_load_2d(s0 + 2 * A_BYTES, &maps.bb, p.b_x0 + k0, p.b_y0 + n0, fb);
+          tma_load_2d(s0 + 2 * A_BYTES + B_BYTES, &maps.bs, p.b_x0 + k0, p.b_y0 + n0, fb);
+          issued[stage] = true;
+          issued_phase[stage] = phase;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok)
+        for (int s = 0; s < STAGES; ++s)
+          if (issued[s]) mbar_drain(full0 + 8 * s, issued_phase[s]);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true, any = false;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        if (!mbar_wait(accempty, acc_phase ^ 1u, abort_flag, p.info, 12)) break;
+        fence_after();
+        for (int kb = 0; kb < p.kblocks; ++kb) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, p.info, 13)) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          const uint32_t s0 = smem_u32(smem + stage * STAGE_BYTES);
+          const uint32_t ab = s0, as = s0 + A_BYTES, bb = s0 + 2 * A_BYTES, bs = bb + B_BYTES;
+#pragma unroll
+          for (int ks = 0; ks < BKF / 8; ++ks) {
+            const uint64_t dbb = desc_op(bb + ks * 32), dbs = desc_op(bs + ks * 32);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint32_t d = tmem + 256 * h;
+              const uint32_t first = (kb == 0 && ks == 0) ? 0u : 1u;
+              const uint64_t dab = desc_op(ab + h * (A_BYTES / 2) + ks * 32);
+              const uint64_t das = desc_op(as + h * (A_BYTES / 2) + ks * 32);
+              mma_tf32<IDESC>(d, dab, dbs, first);   // big x small
+              mma_tf32<IDESC>(d, das, dbb, 1u);      // small x big
+              mma_tf32<IDESC>(d, dab, dbb, 1u);      // big x big
+            }
+          }
+          any = true;
+          mma_commit(empty0 + 8 * stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(accfull);
+        acc_phase ^= 1u;
+      }
+      if (any) {
+        mma_commit(drained);
+        mbar_drain(drained, 0);
+      }
+    }
+  } else {
+    const int wq = warp & 3;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+      const int64_t m0 = (int64_t)(t / p.tiles_n) * BM, n0 = (int64_t)(t % p.tiles_n) * BN;
+      // one lane waits, the warp follows: every lane leaves together on abort
+      bool ready = true;
+      if (lane == 0) ready = mbar_wait(accfull, acc_phase, abort_flag, p.info, 14);
+      if (!__shfl_sync(0xffffffffu, ready ? 1 : 0, 0)) break;
+      __syncwarp();
+      fence_after();
+      double dot = 0.0;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        const int64_t gi = m0 + h * 128 + 32 * wq + lane;
+        const bool row_ok = gi < p.M;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          float v[16];
+          tmem_ld16(tmem + ((uint32_t)(32 * wq) << 16) + (uint32_t)(256 * h + c0), v);
+          const int64_t gj0 = n0 + c0;
+          if (!row_ok || gj0 >= p.N) continue;
+          const bool full16 = gj0 + 16 <= p.N;
+          if (p.epilogue == kEpiDot) {
+            const float* o = p.other + gi * p.ld_other + gj0;
+            if (full16) {
+#pragma unroll
+              for (int q = 0; q < 16; q += 4) {
+                const float4 w = *reinterpret_cast<const float4*>(o + q);
+                dot += (double)v[q] * w.x + (double)v[q + 1] * w.y + (double)v[q + 2] * w.z + (double)v[q + 3] * w.w;
+              }
+            } else {
+              for (int q = 0; gj0 + q < p.N && q < 16; ++q) dot += (double)v[q] * o[q];
+            }
+          } else {
+            float* c = p.C + gi * p.ldc + gj0;
+            if (p.epilogue == kEpiSubtract) {
+              const float* s = p.src + gi * p.ld_src + gj0;
+              if (full16 && !p.dead) {
+#pragma unroll
+                for (int q = 0; q < 16; q += 4) {
+                  float4 w = *reinterpret_cast<const float4*>(s + q);
+                  w.x -= v[q];
+                  w.y -= v[q + 1];
+                  w.z -= v[q + 2];
+                  w.w -= v[q + 3];
+                  *reinterpret_cast<float4*>(c + q) = w;
+                }
+              } else {
+                for (int q = 0; gj0 + q < p.N && q < 16; ++q) {
+                  const float sv = (p.dead && p.dead[gj0 + q]) ? 0.f : s[q];
+                  c[q] = sv - v[q];
+                }
+              }
+            } else {
+              if (full16) {
+#pragma unroll
+                for (int q = 0; q < 16; q += 4)
+                  *reinterpret_cast<float4*>(c + q) = make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
+              } else {
+                for (int q = 0; gj0 + q < p.N && q < 16; ++q) c[q] = v[q];
+              }
+            }
+          }
+        }
+      }
+      fence_before();
+      mbar_arrive(accempty);
+      if (p.epilogue == kEpiDot) {
+        // fixed-order reduction within the warp (xor butterfly); one partial
+        // per (tile, warp), summed later in index order: no CTA barrier here
+        for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        if (lane == 0) p.partial[4 * (int64_t)t + wq] = dot;
+      }
+      acc_phase ^= 1u;
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    fence_after();
+    tmem_dealloc<512>(tmem);
+  }
+}
+
+__device__ __forceinline__ float tf32_round(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
+// big = tf32(x - y), small = (x - y) - big at (r, c), or at (c, r) when
+// transposing (through a 32 x 32 shared-memory tile so both sides coalesce).
+__global__ void __launch_bounds__(256) split_kernel(const float* __restrict__ x, int64_t ldx,
+                                                    const float* __restrict__ y, int64_t ldy, int64_t rows,
+                                                    int64_t cols, float* __restrict__ big, float* __restrict__ small,
+                                                    int64_t ldo, int transpose) {
+  __shared__ float tb[32][33];
+  __shared__ float ts[32][33];
+  const int64_t tiles_c = (cols + 31) / 32;
+  const int64_t r0 = (int64_t)(blockIdx.x / tiles_c) * 32, c0 = (int64_t)(blockIdx.x % tiles_c) * 32;
+  const int tx = threadIdx.x % 32, ty = threadIdx.x / 32;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int64_t r = r0 + ty + 8 * k, c = c0 + tx;
+    if (r < rows && c < cols) {
+      float v = x[r * ldx + c];
+      if (y) v -= y[r * ldy + c];
+      const float b = tf32_round(v);
+      if (transpose) {
+        tb[ty + 8 * k][tx] = b;
+        ts[ty + 8 * k][tx] = v - b;
+      } else {
+        big[r * ldo + c] = b;
+        small[r * ldo + c] = v - b;
+      }
+    }
+  }
+  if (!transpose) return;
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int64_t c = c0 + ty + 8 * k, r = r0 + tx;   // output row c, column r
+    if (r < rows && c < cols) {
+      big[c * ldo + r] = tb[tx][ty + 8 * k];
+      small[c * ldo + r] = ts[tx][ty + 8 * k];
+    }
+  }
+}
+
+}  // namespace
+
+int64_t gemm_tiles(int64_t M, int64_t N) { return cdiv(M, BM) * cdiv(N, BN); }
+
+kq_status split_tf32(const float* x, int64_t ldx, const float* y, int64_t ldy, int64_t rows, int64_t cols, float* big,
+                     float* small, int64_t ldo, bool transpose, cudaStream_t st) {
+  if (rows <= 0 || cols <= 0) return KQ_OK;
+  const int64_t blocks = cdiv(rows, 32) * cdiv(cols, 32);
+  if (blocks > 0x7fffffff) return fail(KQ_ERR_UNSUPPORTED_SHAPE, "split_tf32: too large");
+  split_kernel<<<(unsigned)blocks, 256, 0, st>>>(x, ldx, y, ldy, rows, cols, big, small, ldo, transpose ? 1 : 0);
+  return launch_check("split_tf32");
+}
+
+kq_status gemm_3xtf32(const Gemm3xTF32& g, cudaStream_t st) {
+  if (g.M <= 0 || g.N <= 0 || g.K <= 0) return KQ_OK;
+  const void* ptrs[] = {g.a_big, g.a_small, g.bt_big, g.bt_small};
+  for (const void* q : ptrs)
+    if (!q || !aligned(q, 16)) return fail(KQ_ERR_ALIGNMENT, "gemm: operands must be 16-byte aligned");
+  if ((g.lda & 3) || (g.ldbt & 3) || (g.a_col0 & 3) || (g.bt_col0 & 3))
+    return fail(KQ_ERR_ALIGNMENT, "gemm: leading dimensions and column offsets must be multiples of 4");
+  const int64_t big = (int64_t)1 << 31;
+  if (g.a_row0 + g.M >= big || g.a_col0 + g.K >= big || g.bt_row0 + g.N >= big || g.bt_col0 + g.K >= big)
+    return fail(KQ_ERR_UNSUPPORTED_SHAPE, "gemm: coordinates beyond 2^31");
+  // Tensor maps end exactly at the used region, so every read past M, N or K
+  // (ragged tiles, a K tail) is filled with zeros by the TMA unit.
+  Maps maps;
+  auto map_op = [&](CUtensorMap* m, const float* base, int64_t ld, int64_t row0, int64_t col0, int64_t rows)
+      -> kq_status {
+    return tc::make_map_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, col0 + g.K, row0 + rows, ld, BKF, BM,
+                           CU_TENSOR_MAP_SWIZZLE_64B);
+  };
+  KQ_TRY(map_op(&maps.ab, g.a_big, g.lda, g.a_row0, g.a_col0, g.M));
+  KQ_TRY(map_op(&maps.as, g.a_small, g.lda, g.a_row0, g.a_col0, g.M));
+  KQ_TRY(map_op(&maps.bb, g.bt_big, g.ldbt, g.bt_row0, g.bt_col0, g.N));
+  KQ_TRY(map_op(&maps.bs, g.bt_small, g.ldbt, g.bt_row0, g.bt_col0, g.N));
+  Params p;
+  p.M = g.M;
+  p.N = g.N;
+  p.K = g.K;
+  p.tiles_m = (int)cdiv(g.M, BM);
+  p.tiles_n = (int)cdiv(g.N, BN);
+  p.num_tiles = p.tiles_m * p.tiles_n;
+  p.kblocks = (int)cdiv(g.K, BKF);
+  p.a_x0 = (int)g.a_col0;
+  p.a_y0 = (int)g.a_row0;
+  p.b_x0 = (int)g.bt_col0;
+  p.b_y0 = (int)g.bt_row0;
+  p.epilogue = g.epilogue;
+  p.C = g.C;
+  p.ldc = g.ldc;
+  p.src = g.src;
+  p.ld_src = g.ld_src;
+  p.dead = g.dead;
+  p.other = g.other;
+  p.ld_other = g.ld_other;
+  p.partial = g.partial;
+  p.info = g.info;
+  if (g.epilogue == kEpiDot) {
+    if (!g.other || !g.partial || !aligned(g.other, 16) || (g.ld_other & 3))
+      return fail(KQ_ERR_ALIGNMENT, "gemm: dot epilogue needs an aligned `other` and `partial`");
+  } else {
+    if (!g.C || !aligned(g.C, 16) || (g.ldc & 3)) return fail(KQ_ERR_ALIGNMENT, "gemm: C must be 16-byte aligned");
+    if (g.epilogue == kEpiSubtract && (!g.src || !aligned(g.src, 16) || (g.ld_src & 3)))
+      return fail(KQ_ERR_ALIGNMENT, "gemm: src must be 16-byte aligned");
+  }
+  int dev = 0, sms = 148;
+  KQ_TRY(cuda_check(cudaGetDevice(&dev), "gemm: cudaGetDevice"));
+  KQ_TRY(cuda_check(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev), "gemm: SM count"));
+  KQ_TRY(cuda_check(cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES),
+                    "gemm: smem attribute"));
+  gemm_kernel<<<std::min(p.num_tiles, sms), THREADS, SMEM_BYTES, st>>>(maps, p);
+  return launch_check("gemm_3xtf32");
+}
+
+}  // namespace kq

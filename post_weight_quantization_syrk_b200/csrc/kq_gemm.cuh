@@ -1,0 +1,51 @@
+// fp32-accurate GEMM on the tcgen05 tensor cores (3xTF32), internal to the
+// library: used by the Kronecker loss and the solver's lazy trailing update.
+#pragma once
+
+#include "kq_internal.cuh"
+
+namespace kq {
+
+// Epilogues: C = AB;  partial[tile] = sum_ij (AB)_ij other_ij;  C = src - AB.
+enum GemmEpilogue { kEpiStore = 0, kEpiDot = 1, kEpiSubtract = 2 };
+
+// C[M, N] = A[M, K] B[K, N], each operand given as a tf32 "big" part and an
+// fp32 remainder "small" (see split_tf32), as AB ~ Ab Bb + Ab Bs + As Bb
+// with fp32 accumulation in TMEM.  Both operands are read K-major (the
+// layout tcgen05 kind::tf32 takes): A as stored, B through its transpose Bt:
+//   (m, k) of A at a[(a_row0 + m) * lda + a_col0 + k]
+//   (k, n) of B at bt[(bt_row0 + n) * ldbt + bt_col0 + k]
+// All base pointers 16-byte aligned; leading dimensions and column offsets
+// multiples of 4.
+struct Gemm3xTF32 {
+  int64_t M = 0, N = 0, K = 0;
+  const float* a_big = nullptr;
+  const float* a_small = nullptr;
+  int64_t lda = 0, a_row0 = 0, a_col0 = 0;
+  const float* bt_big = nullptr;
+  const float* bt_small = nullptr;
+  int64_t ldbt = 0, bt_row0 = 0, bt_col0 = 0;
+  int epilogue = kEpiStore;
+  float* C = nullptr;              // (m, n) at C[m * ldc + n]      (store, subtract)
+  int64_t ldc = 0;
+  const float* src = nullptr;      // (m, n) at src[m * ld_src + n] (subtract)
+  int64_t ld_src = 0;
+  const uint8_t* dead = nullptr;   // subtract: src column n reads as 0 when dead[n]
+  const float* other = nullptr;    // (m, n) at other[m * ld_other + n] (dot)
+  int64_t ld_other = 0;
+  double* partial = nullptr;       // dot: 4 fp64 per output tile (one per epilogue warp)
+  int32_t* info = nullptr;
+};
+
+// Output tiles of an M x N product (`partial` holds 4 per tile for kEpiDot).
+int64_t gemm_tiles(int64_t M, int64_t N);
+
+kq_status gemm_3xtf32(const Gemm3xTF32& g, cudaStream_t st);
+
+// big = tf32(x - y) (round to nearest), small = (x - y) - big, elementwise over
+// rows x cols; y may be NULL.  Outputs have leading dimension ldo and are
+// written transposed ([cols][rows]) when `transpose`.
+kq_status split_tf32(const float* x, int64_t ldx, const float* y, int64_t ldy, int64_t rows, int64_t cols,
+                     float* big, float* small, int64_t ldo, bool transpose, cudaStream_t st);
+
+}  // namespace kq

@@ -4,11 +4,20 @@
 // Unified Hessian-Guided PTQ (hub.valency.io/works/W_r72x54u6), Appendix A.1:
 // the Kronecker-weighted norm of a perturbation is a trace of this form.
 // Using the symmetry of H_G, tr(dW H_X dW^T H_G) = sum_ij (dW H_X)_ij (H_G dW)_ij.
-// Each CTA forms one 64x64 tile of both products (dW is formed on the fly from
-// W and W_hat), reduces their elementwise product to an fp64 partial, and a
-// final one-CTA pass sums the partials in a fixed order (deterministic).
+//
+// kq_kron_loss runs the two products on the tensor cores in 3xTF32 (fp32
+// accuracy; plain TF32 or bf16 lose too much to cancellation here): split
+// dW, H_X, H_G into tf32 + remainder, A1 = dW H_X stored, then H_G dW with
+// the elementwise product against A1 reduced in the GEMM epilogue to fp64
+// partials, summed in a fixed order.
+//
+// kq_kron_loss_noalloc (below) keeps a SIMT fp32 path whose only scratch is
+// one fp64 per 64x64 tile: each CTA forms one tile of both products and
+// reduces their elementwise product.
+#include <algorithm>
 #include <mutex>
 
+#include "kq_gemm.cuh"
 #include "kq_internal.cuh"
 
 namespace {
@@ -104,9 +113,77 @@ __global__ void sum_kernel(const double* __restrict__ partial, int64_t n, double
 
 }  // namespace
 
+namespace {
+
+// sum_ij A1_ij (Db + Ds)_ij: the H_G = I case (dW = Db + Ds exactly).
+__global__ void __launch_bounds__(256) dot_rows_kernel(const float* __restrict__ A1, const float* __restrict__ Db,
+                                                       const float* __restrict__ Ds, int64_t ld, int64_t rows,
+                                                       int64_t cols, double* __restrict__ partial) {
+  __shared__ double red[256];
+  double s = 0.0;
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x)
+    for (int64_t c = threadIdx.x; c < cols; c += blockDim.x) {
+      const int64_t i = r * ld + c;
+      s += (double)A1[i] * (double)(Db[i] + Ds[i]);
+    }
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) partial[blockIdx.x] = red[0];
+}
+
+constexpr int kDotBlocks = 1024;
+
+// dW (as A of dW H_X), dW^T (as the transposed B of H_G dW), H_X^T, H_G, each
+// split into tf32 + remainder, then A1 = dW H_X and the partial sums.
+struct LossWs {
+  float *Db, *Ds, *Dtb, *Dts, *Xb, *Xs, *Gb, *Gs, *A1;
+  double* partial;
+  int64_t ldd, ldt, ldx, ldg;
+};
+
+size_t loss_layout(int64_t d_out, int64_t d_in, LossWs* w, void* base) {
+  const int64_t ldd = (d_in + 3) / 4 * 4, ldx = ldd, ldg = (d_out + 3) / 4 * 4, ldt = ldg;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = kq::align_up(off + bytes, 256);
+    return o;
+  };
+  const size_t sd = (size_t)d_out * ldd * 4, st_ = (size_t)d_in * ldt * 4, sx = (size_t)d_in * ldx * 4,
+               sg = (size_t)d_out * ldg * 4;
+  size_t oDb = take(sd), oDs = take(sd), oTb = take(st_), oTs = take(st_), oXb = take(sx), oXs = take(sx),
+         oGb = take(sg), oGs = take(sg), oA = take(sd);
+  const int64_t np = std::max<int64_t>(4 * kq::gemm_tiles(d_out, d_in), kDotBlocks);
+  size_t oP = take((size_t)np * 8);
+  if (w && base) {
+    char* b = static_cast<char*>(base);
+    w->Db = reinterpret_cast<float*>(b + oDb);
+    w->Ds = reinterpret_cast<float*>(b + oDs);
+    w->Dtb = reinterpret_cast<float*>(b + oTb);
+    w->Dts = reinterpret_cast<float*>(b + oTs);
+    w->Xb = reinterpret_cast<float*>(b + oXb);
+    w->Xs = reinterpret_cast<float*>(b + oXs);
+    w->Gb = reinterpret_cast<float*>(b + oGb);
+    w->Gs = reinterpret_cast<float*>(b + oGs);
+    w->A1 = reinterpret_cast<float*>(b + oA);
+    w->partial = reinterpret_cast<double*>(b + oP);
+    w->ldd = ldd;
+    w->ldt = ldt;
+    w->ldx = ldx;
+    w->ldg = ldg;
+  }
+  return off;
+}
+
+}  // namespace
+
 extern "C" size_t kq_kron_loss_workspace_size(int64_t d_out, int64_t d_in) {
   if (d_out < 1 || d_in < 1) return 0;
-  return kq::align_up((size_t)kq::cdiv(d_out, T) * kq::cdiv(d_in, T) * sizeof(double), 256);
+  return loss_layout(d_out, d_in, nullptr, nullptr);
 }
 
 extern "C" kq_status kq_kron_loss(const float* W, int64_t ldw, const float* W_hat, int64_t ldwh, int64_t d_out,
@@ -114,17 +191,56 @@ extern "C" kq_status kq_kron_loss(const float* W, int64_t ldw, const float* W_ha
                                   double* loss, void* ws, size_t ws_bytes, kq_stream_t stream) {
   if (!W || !W_hat || !H_X || !loss) return kq::fail(KQ_ERR_INVALID_ARG, "kq_kron_loss: NULL pointer");
   if (d_out < 1 || d_in < 1) return kq::fail(KQ_ERR_INVALID_ARG, "kq_kron_loss: sizes must be >= 1");
+  if (d_out > 65536 || d_in > 65536) return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_kron_loss: sizes above 65536");
   if (ldw < d_in || ldwh < d_in || ldhx < d_in || (H_G && ldhg < d_out))
     return kq::fail(KQ_ERR_INVALID_ARG, "kq_kron_loss: leading dimension too small");
   if (!ws || !kq::aligned(ws, 256) || ws_bytes < kq_kron_loss_workspace_size(d_out, d_in))
     return kq::fail(KQ_ERR_WORKSPACE, "kq_kron_loss: workspace too small or not 256-byte aligned");
-  if (kq::cdiv(d_out, T) > 65535) return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_kron_loss: d_out too large");
   cudaStream_t st = (cudaStream_t)stream;
-  double* partial = static_cast<double*>(ws);
-  dim3 grid((unsigned)kq::cdiv(d_in, T), (unsigned)kq::cdiv(d_out, T));
-  loss_tile_kernel<<<grid, 256, 0, st>>>(W, ldw, W_hat, ldwh, d_out, d_in, H_X, ldhx, H_G, ldhg, partial);
-  KQ_TRY(kq::launch_check("kq_kron_loss tiles"));
-  sum_kernel<<<1, 1024, 0, st>>>(partial, (int64_t)grid.x * grid.y, loss);
+  LossWs w;
+  loss_layout(d_out, d_in, &w, ws);
+  KQ_TRY(kq::split_tf32(W, ldw, W_hat, ldwh, d_out, d_in, w.Db, w.Ds, w.ldd, false, st));
+  KQ_TRY(kq::split_tf32(H_X, ldhx, nullptr, 0, d_in, d_in, w.Xb, w.Xs, w.ldx, true, st));
+  kq::Gemm3xTF32 g1;                 // A1 = dW H_X   (B^T = H_X^T)
+  g1.M = d_out;
+  g1.N = d_in;
+  g1.K = d_in;
+  g1.a_big = w.Db;
+  g1.a_small = w.Ds;
+  g1.lda = w.ldd;
+  g1.bt_big = w.Xb;
+  g1.bt_small = w.Xs;
+  g1.ldbt = w.ldx;
+  g1.epilogue = kq::kEpiStore;
+  g1.C = w.A1;
+  g1.ldc = w.ldd;
+  KQ_TRY(kq::gemm_3xtf32(g1, st));
+  int64_t np;
+  if (H_G) {
+    KQ_TRY(kq::split_tf32(W, ldw, W_hat, ldwh, d_out, d_in, w.Dtb, w.Dts, w.ldt, true, st));
+    KQ_TRY(kq::split_tf32(H_G, ldhg, nullptr, 0, d_out, d_out, w.Gb, w.Gs, w.ldg, false, st));
+    kq::Gemm3xTF32 g2;               // sum (H_G dW) .* A1   (B^T = dW^T)
+    g2.M = d_out;
+    g2.N = d_in;
+    g2.K = d_out;
+    g2.a_big = w.Gb;
+    g2.a_small = w.Gs;
+    g2.lda = w.ldg;
+    g2.bt_big = w.Dtb;
+    g2.bt_small = w.Dts;
+    g2.ldbt = w.ldt;
+    g2.epilogue = kq::kEpiDot;
+    g2.other = w.A1;
+    g2.ld_other = w.ldd;
+    g2.partial = w.partial;
+    KQ_TRY(kq::gemm_3xtf32(g2, st));
+    np = 4 * kq::gemm_tiles(d_out, d_in);
+  } else {
+    dot_rows_kernel<<<kDotBlocks, 256, 0, st>>>(w.A1, w.Db, w.Ds, w.ldd, d_out, d_in, w.partial);
+    KQ_TRY(kq::launch_check("kq_kron_loss dot"));
+    np = kDotBlocks;
+  }
+  sum_kernel<<<1, 1024, 0, st>>>(w.partial, np, loss);
   KQ_TRY(kq::launch_check("kq_kron_loss sum"));
   kq::clear_error();
   return KQ_OK;

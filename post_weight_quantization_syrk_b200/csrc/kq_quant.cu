@@ -4,31 +4,33 @@
 // KronQ review (romaanj.github.io/reviews/kronq), Goal and Method (1): the
 // solver stays the H_X-only column-wise OBS update (H_G cancels from it,
 // Proposition 1).  For each block of 128 columns:
-//   in-block recursion (latency bound, 128 dependent steps): one thread owns
-//     one output row; the rows of a CTA keep their 128-column slab in shared
-//     memory and the block's Uc rows (transposed) beside it; columns are taken
-//     in sub-blocks of 32 held in registers, and the rest of the block is
-//     brought up to date with the sub-block's 32 errors at once (same
-//     left-to-right order of the subtractions as column by column);
-//   lazy trailing update W[:, end:] -= E Uc[blk, end:] (a dense GEMM).
+//   in-block recursion (latency bound, 128 dependent steps): eight lanes
+//     share one output row, each holding 16 of the block's columns in
+//     registers; the column's owner quantizes it and broadcasts its error by
+//     warp shuffle, and every lane applies the rank-1 update to its own
+//     columns with the block's Uc rows read from shared memory.  The
+//     subtractions into each column happen in the same left-to-right order
+//     as column by column;
+//   lazy trailing update W[:, end:] -= E Uc[blk, end:] (a dense GEMM): fp32
+//     SIMT (KQ_GEMM_FP32) or 3xTF32 on the tcgen05 tensor cores
+//     (KQ_GEMM_3XTF32, the block's errors split into tf32 + remainder as they
+//     are written, Uc split once per call).
 // W_hat doubles as the running copy of W: column j of W_hat is overwritten by
 // its dequantized value once the column has been quantized.
 //
 // Grid (asymmetric min/max): scale = (max - min) / (2^b - 1),
 // zero = rint(-min / scale); degenerate range: scale 1, zero rint(-min).
-// Codes q = clamp(rint(w / scale + zero), 0, 2^b - 1).  IEEE fp32 throughout
-// (true division, round half to even).
+// Codes q = clamp(rint(v), 0, 2^b - 1) with v = fma(w, 1/scale, zero) in fp32
+// (round half to even); errors e = (w - w_hat) * (1/Uc[j][j]).  The grid
+// itself (scale, zero) uses IEEE fp32 division.
 #include <algorithm>
 
+#include "kq_gemm.cuh"
 #include "kq_internal.cuh"
 
 namespace {
 
 constexpr int BLK = 128;      // solver block
-constexpr int SUB = 32;       // register sub-block
-constexpr int RPC = 32;       // rows (threads) per CTA in the in-block kernel
-constexpr int UT_LD = 132;    // padded row of the transposed Uc block
-constexpr int WS_LD = 129;    // padded row of the W slab
 
 __device__ __forceinline__ void fit_grid(float mn, float mx, float nl, float* scale, float* zero) {
   float s = (mx - mn) / nl;
@@ -94,114 +96,183 @@ struct InblockArgs {
   int64_t n_groups;
   uint8_t* codes;
   int64_t ldq;
-  float* ET;   // [128, d_out]: the block's errors, transposed
+  float* ET;   // [128, d_out]: the block's errors, transposed (fp32 SIMT trailing update)
+  float* Eb;   // [d_out, 128]: tf32 part of the errors (3xTF32 trailing update), or NULL
+  float* Es;   // [d_out, 128]: remainder
   int32_t* info;
 };
 
-__global__ void __launch_bounds__(RPC) inblock_kernel(InblockArgs a) {
+// Eight lanes share a row: lane L of a row group owns the 16 columns
+// 32 m + 4 L + t (m, t in 0..3), kept in registers.  Column j is quantized by
+// its owner, whose error e_j reaches the row's other lanes by one warp
+// shuffle; every lane then updates its own columns right of j.  This
+// interleaved ownership makes each lane's four float4 reads of Uc row j hit
+// distinct shared-memory banks.
+constexpr int LPR = 8;                  // lanes per row
+constexpr int IB_THREADS = 256;
+constexpr int IB_ROWS = IB_THREADS / LPR;  // 32 rows per CTA
+constexpr int IB_SMEM = BLK * BLK * 4 + BLK * 4;
+
+__device__ __forceinline__ int col_of(int L, int r) { return 32 * (r >> 2) + 4 * L + (r & 3); }
+
+__global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
   extern __shared__ float sm[];
-  float* UT = sm;                        // [128][UT_LD], UT[k][j] = Uc[i0+j][i0+k]
-  float* Ws = UT + BLK * UT_LD;          // [RPC][WS_LD] slab, later W_hat
-  float* Es = Ws + RPC * WS_LD;          // [RPC][WS_LD] errors
-  uint8_t* Qs = reinterpret_cast<uint8_t*>(Es + RPC * WS_LD);  // [RPC][BLK]
+  float* Us = sm;                 // [128][128]: Uc[i0 + j][i0 + k]
+  float* inv_d = sm + BLK * BLK;  // 1 / Uc[i0 + j][i0 + j]
   const int t = threadIdx.x;
-  const int64_t row0 = (int64_t)blockIdx.x * RPC;
+  const int lane = t & 31, L = lane & (LPR - 1);
+  const int64_t row = (int64_t)blockIdx.x * IB_ROWS + t / LPR;
+  const bool row_ok = row < a.d_out;
   const int bw = a.bw;
   const int64_t i0 = a.i0;
 
-  for (int idx = t; idx < BLK * BLK; idx += RPC) {
-    int j = idx / BLK, k = idx % BLK;
-    UT[k * UT_LD + j] = (k >= j && j < bw && k < bw) ? a.Uc[(i0 + j) * a.lduc + i0 + k] : 0.f;
-  }
-  for (int idx = t; idx < RPC * BLK; idx += RPC) {
-    int r = idx / BLK, c = idx % BLK;
-    float v = 0.f;
-    if (row0 + r < a.d_out && c < bw) {
-      v = load_w(a.src, a.ld_src, row0 + r, i0 + c, a.dead);
-      if (!isfinite(v)) kq::report(a.info, KQ_ERR_NONFINITE, row0 + r);
+  for (int idx = t; idx < BLK * (BLK / 4); idx += IB_THREADS) {
+    const int j = idx / (BLK / 4), k = 4 * (idx % (BLK / 4));
+    float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (j < bw) {
+      const float* g = a.Uc + (i0 + j) * a.lduc + i0 + k;
+      if (k + 3 < bw) {
+        u = *reinterpret_cast<const float4*>(g);
+      } else {
+        if (k + 0 < bw) u.x = g[0];
+        if (k + 1 < bw) u.y = g[1];
+        if (k + 2 < bw) u.z = g[2];
+      }
     }
-    Ws[r * WS_LD + c] = v;
+    *reinterpret_cast<float4*>(Us + j * BLK + k) = u;
+  }
+
+  // this lane's 16 columns of the row
+  float w[16];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const int c = 32 * m + 4 * L;
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    if (row_ok) {
+      if (c + 3 < bw && !a.dead) {
+        const float4 q = *reinterpret_cast<const float4*>(a.src + row * a.ld_src + i0 + c);
+        v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+      } else {
+        for (int e = 0; e < 4; ++e)
+          if (c + e < bw) v[e] = load_w(a.src, a.ld_src, row, i0 + c + e, a.dead);
+      }
+      if (!(isfinite(v[0]) && isfinite(v[1]) && isfinite(v[2]) && isfinite(v[3])))
+        kq::report(a.info, KQ_ERR_NONFINITE, row);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) w[4 * m + e] = v[e];
   }
   __syncthreads();
+  if (t < BLK) inv_d[t] = (t < bw) ? 1.f / Us[t * BLK + t] : 0.f;
+  __syncthreads();
 
-  const int64_t r = row0 + t;
   float scale = 1.f, zero = 0.f;
-  if (!a.group && r < a.d_out) {
-    scale = a.scales[r * a.n_groups];
-    zero = a.zeros[r * a.n_groups];
+  if (!a.group && row_ok) {
+    scale = a.scales[row * a.n_groups];
+    zero = a.zeros[row * a.n_groups];
   }
-  float* wrow = Ws + t * WS_LD;
-  float* erow = Es + t * WS_LD;
-  for (int s0 = 0; s0 < bw; s0 += SUB) {
-    float w[SUB], e[SUB];
+  float inv_scale = 1.f / scale;
+  float qv[16], ev[16];
+  const int gbase = lane & ~(LPR - 1);
+
 #pragma unroll
-    for (int jj = 0; jj < SUB; ++jj) {
-      w[jj] = (s0 + jj < bw) ? wrow[s0 + jj] : 0.f;
-      e[jj] = 0.f;
-    }
+  for (int m = 0; m < 4; ++m) {
+#pragma unroll 1
+    for (int Lo = 0; Lo < LPR; ++Lo) {
 #pragma unroll
-    for (int jj = 0; jj < SUB; ++jj) {
-      const int j = s0 + jj;
-      if (j < bw) {
-        if (a.group && ((i0 + j) % a.group) == 0) {
-          // Group grid on the current values of the group's columns; they are
-          // all in this block and up to date (group divides the block, and
-          // groups start on sub-block boundaries, so w[] == wrow here).
+      for (int tt = 0; tt < 4; ++tt) {
+        const int j = 32 * m + 4 * Lo + tt;   // column quantized in this step
+        if (j >= bw) break;
+        if (a.group && tt == 0 && ((i0 + j) % a.group) == 0) {
+          // group grid on the current values of columns [j, j + group): every
+          // lane folds its own columns in range, then the row's 8 lanes meet
           const int64_t lim = a.d_in - i0;
           const int gend = (int)((int64_t)(j + a.group) < lim ? (int64_t)(j + a.group) : lim);
           float mn = INFINITY, mx = -INFINITY;
-          for (int c = j; c < gend; ++c) {
-            mn = fminf(mn, wrow[c]);
-            mx = fmaxf(mx, wrow[c]);
+#pragma unroll
+          for (int r = 0; r < 16; ++r) {
+            const int c = col_of(L, r);
+            if (c >= j && c < gend) {
+              mn = fminf(mn, w[r]);
+              mx = fmaxf(mx, w[r]);
+            }
+          }
+#pragma unroll
+          for (int o = 1; o < LPR; o <<= 1) {
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
           }
           fit_grid(mn, mx, a.nl, &scale, &zero);
-          if (r < a.d_out) {
+          inv_scale = 1.f / scale;
+          if (row_ok && L == 0) {
             const int64_t g = (i0 + j) / a.group;
-            a.scales[r * a.n_groups + g] = scale;
-            a.zeros[r * a.n_groups + g] = zero;
+            a.scales[row * a.n_groups + g] = scale;
+            a.zeros[row * a.n_groups + g] = zero;
           }
         }
-        const float v = w[jj] / scale + zero;
+        // every lane runs the owner's arithmetic on its own register 4m+tt;
+        // only the owner's (L == Lo) result is kept and broadcast
+        const int r = 4 * m + tt;
+        const float x = w[r];
+        const float v = fmaf(x, inv_scale, zero);
         const float q = fminf(fmaxf(rintf(v), 0.f), a.nl);
         const float wh = scale * (q - zero);
-        const float ej = (w[jj] - wh) / UT[j * UT_LD + j];
-        e[jj] = ej;
+        const float e_own = (x - wh) * inv_d[j];
+        if (L == Lo) {
+          qv[r] = q;
+          w[r] = wh;   // the column is final: keep its dequantized value
+          ev[r] = e_own;
+        }
+        const float e = __shfl_sync(0xffffffffu, e_own, gbase + Lo);
+        const float4* urow = reinterpret_cast<const float4*>(Us + j * BLK);
 #pragma unroll
-        for (int kk = jj + 1; kk < SUB; ++kk) w[kk] = fmaf(-ej, UT[(s0 + kk) * UT_LD + j], w[kk]);
-        wrow[j] = wh;
-        erow[j] = ej;
-        Qs[t * BLK + j] = (uint8_t)q;
+        for (int m2 = 0; m2 < 4; ++m2) {
+          const float4 u = urow[8 * m2 + L];
+          const float uu[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int t2 = 0; t2 < 4; ++t2) {
+            const int r2 = 4 * m2 + t2;
+            if (col_of(L, r2) > j) w[r2] = fmaf(-e, uu[t2], w[r2]);
+          }
+        }
       }
     }
-    // bring the rest of the block up to date with this sub-block's errors
-    for (int k = s0 + SUB; k < bw; ++k) {
-      float acc = wrow[k];
-      const float4* u4 = reinterpret_cast<const float4*>(UT + k * UT_LD + s0);
+  }
+
+  if (!row_ok) return;
+  // this lane's 16 columns: W_hat, codes, and the errors for the trailing update
 #pragma unroll
-      for (int q4 = 0; q4 < SUB / 4; ++q4) {
-        float4 u = u4[q4];
-        acc = fmaf(-e[4 * q4 + 0], u.x, acc);
-        acc = fmaf(-e[4 * q4 + 1], u.y, acc);
-        acc = fmaf(-e[4 * q4 + 2], u.z, acc);
-        acc = fmaf(-e[4 * q4 + 3], u.w, acc);
-      }
-      wrow[k] = acc;
+  for (int m = 0; m < 4; ++m) {
+    const int c = 32 * m + 4 * L;
+    if (c + 3 < bw) {
+      *reinterpret_cast<float4*>(a.W_hat + row * a.ldwh + i0 + c) = make_float4(w[4 * m], w[4 * m + 1], w[4 * m + 2],
+                                                                               w[4 * m + 3]);
+      uchar4 qq = make_uchar4((unsigned char)qv[4 * m], (unsigned char)qv[4 * m + 1], (unsigned char)qv[4 * m + 2],
+                              (unsigned char)qv[4 * m + 3]);
+      *reinterpret_cast<uchar4*>(a.codes + row * a.ldq + i0 + c) = qq;
+    } else {
+      for (int e = 0; e < 4; ++e)
+        if (c + e < bw) {
+          a.W_hat[row * a.ldwh + i0 + c + e] = w[4 * m + e];
+          a.codes[row * a.ldq + i0 + c + e] = (uint8_t)qv[4 * m + e];
+        }
     }
-  }
-  __syncthreads();
-  // coalesced write-back of codes and W_hat (row-major) and of E^T ([128][d_out])
-  for (int idx = t; idx < RPC * BLK; idx += RPC) {
-    int rr = idx / BLK, c = idx % BLK;
-    int64_t row = row0 + rr;
-    if (row >= a.d_out || c >= bw) continue;
-    a.W_hat[row * a.ldwh + i0 + c] = Ws[rr * WS_LD + c];
-    a.codes[row * a.ldq + i0 + c] = Qs[rr * BLK + c];
-  }
-  for (int idx = t; idx < RPC * BLK; idx += RPC) {
-    int c = idx / RPC, rr = idx % RPC;
-    int64_t row = row0 + rr;
-    if (row >= a.d_out || c >= bw) continue;
-    a.ET[(int64_t)c * a.d_out + row] = Es[rr * WS_LD + c];
+    if (a.Eb) {
+      float b[4], sm4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float ee = (c + e < bw) ? ev[4 * m + e] : 0.f;
+        uint32_t bits;
+        asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(bits) : "f"(ee));
+        b[e] = __uint_as_float(bits);
+        sm4[e] = ee - b[e];
+      }
+      *reinterpret_cast<float4*>(a.Eb + row * BLK + c) = make_float4(b[0], b[1], b[2], b[3]);
+      *reinterpret_cast<float4*>(a.Es + row * BLK + c) = make_float4(sm4[0], sm4[1], sm4[2], sm4[3]);
+    } else {
+      for (int e = 0; e < 4; ++e)
+        if (c + e < bw) a.ET[(int64_t)(c + e) * a.d_out + row] = ev[4 * m + e];
+    }
   }
 }
 
@@ -279,11 +350,38 @@ __global__ void __launch_bounds__(256) trailing_fp32_kernel(const float* __restr
 
 }  // namespace
 
+namespace {
+
+// Workspace: the block's errors (E^T for the fp32 path, or E split in two
+// for 3xTF32), then Uc^T split in two (3xTF32 only: the tensor-core product
+// reads its B operand transposed).
+struct QuantWs {
+  float *ET, *Eb, *Es, *Ub, *Us;
+  int64_t ldu;
+};
+
+size_t quant_layout(int64_t d_out, int64_t d_in, QuantWs* w, void* base) {
+  const int64_t ldu = (d_in + 3) / 4 * 4;
+  const size_t se = kq::align_up((size_t)d_out * BLK * sizeof(float), 256);
+  const size_t su = kq::align_up((size_t)d_in * ldu * sizeof(float), 256);
+  if (w && base) {
+    char* b = static_cast<char*>(base);
+    w->ET = reinterpret_cast<float*>(b);
+    w->Eb = reinterpret_cast<float*>(b);
+    w->Es = reinterpret_cast<float*>(b + se);
+    w->Ub = reinterpret_cast<float*>(b + 2 * se);
+    w->Us = reinterpret_cast<float*>(b + 2 * se + su);
+    w->ldu = ldu;
+  }
+  return 2 * se + 2 * su;
+}
+
+}  // namespace
+
 extern "C" size_t kq_quantize_layer_workspace_size(int64_t d_out, int64_t d_in, int block) {
-  (void)d_in;
   (void)block;
-  if (d_out < 1) return 0;
-  return kq::align_up((size_t)d_out * BLK * sizeof(float), 256);  // E^T [128][d_out]
+  if (d_out < 1 || d_in < 1) return 0;
+  return quant_layout(d_out, d_in, nullptr, nullptr);
 }
 
 extern "C" kq_status kq_quantize_layer(const float* W, int64_t d_out, int64_t d_in, int64_t ldw, const float* Uc,
@@ -299,17 +397,21 @@ extern "C" kq_status kq_quantize_layer(const float* W, int64_t d_out, int64_t d_
     return kq::fail(KQ_ERR_INVALID_ARG, "kq_quantize_layer: leading dimension too small");
   if (bits < 2 || bits > 8) return kq::fail(KQ_ERR_INVALID_ARG, "kq_quantize_layer: bits outside 2..8");
   if (block != BLK) return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_quantize_layer: only block = 128 is built");
-  if (group < 0 || (group && (group % SUB || BLK % group)))
+  if (group < 0 || (group && (group % 32 || BLK % group)))
     return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_quantize_layer: group must be 0 or a multiple of 32 dividing 128");
-  if (gemm_mode != KQ_GEMM_FP32)
-    return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_quantize_layer: only KQ_GEMM_FP32 is built");
+  if (gemm_mode != KQ_GEMM_FP32 && gemm_mode != KQ_GEMM_3XTF32)
+    return kq::fail(KQ_ERR_INVALID_ARG, "kq_quantize_layer: gemm_mode must be KQ_GEMM_FP32 or KQ_GEMM_3XTF32");
   if (W == W_hat) return kq::fail(KQ_ERR_INVALID_ARG, "kq_quantize_layer: W and W_hat must not alias");
   if (!kq::aligned(W, 16) || !kq::aligned(W_hat, 16) || !kq::aligned(Uc, 16) || (ldw & 3) || (ldwh & 3) || (lduc & 3))
     return kq::fail(KQ_ERR_ALIGNMENT, "kq_quantize_layer: W, W_hat, Uc need 16-byte alignment and ld % 4 == 0");
   if (!ws || !kq::aligned(ws, 256) || ws_bytes < kq_quantize_layer_workspace_size(d_out, d_in, block))
     return kq::fail(KQ_ERR_WORKSPACE, "kq_quantize_layer: workspace too small or not 256-byte aligned");
   cudaStream_t st = (cudaStream_t)stream;
-  float* ET = static_cast<float*>(ws);
+  QuantWs w;
+  quant_layout(d_out, d_in, &w, ws);
+  const bool tc = (gemm_mode == KQ_GEMM_3XTF32);
+  if (tc) KQ_TRY(kq::split_tf32(Uc, lduc, nullptr, 0, d_in, d_in, w.Ub, w.Us, w.ldu, true, st));
+
   const float nl = (float)((1 << bits) - 1);
   const int64_t n_groups = group ? kq::cdiv(d_in, group) : 1;
 
@@ -318,8 +420,7 @@ extern "C" kq_status kq_quantize_layer(const float* W, int64_t d_out, int64_t d_
                                                                    info);
     KQ_TRY(kq::launch_check("kq_quantize_layer grid"));
   }
-  const size_t smem = (size_t)BLK * UT_LD * sizeof(float) + 2 * (size_t)RPC * WS_LD * sizeof(float) + RPC * BLK;
-  KQ_TRY(kq::cuda_check(cudaFuncSetAttribute(inblock_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
+  KQ_TRY(kq::cuda_check(cudaFuncSetAttribute(inblock_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, IB_SMEM),
                         "kq_quantize_layer: smem attribute"));
   for (int64_t i0 = 0; i0 < d_in; i0 += BLK) {
     const int bw = (int)std::min<int64_t>(BLK, d_in - i0);
@@ -343,16 +444,39 @@ extern "C" kq_status kq_quantize_layer(const float* W, int64_t d_out, int64_t d_
     a.n_groups = n_groups;
     a.codes = codes;
     a.ldq = ldq;
-    a.ET = ET;
+    a.ET = w.ET;
+    a.Eb = tc ? w.Eb : nullptr;
+    a.Es = tc ? w.Es : nullptr;
     a.info = info;
-    inblock_kernel<<<(unsigned)kq::cdiv(d_out, RPC), RPC, smem, st>>>(a);
+    inblock_kernel<<<(unsigned)kq::cdiv(d_out, IB_ROWS), IB_THREADS, IB_SMEM, st>>>(a);
     KQ_TRY(kq::launch_check("kq_quantize_layer inblock"));
     const int64_t cstart = i0 + bw;
-    if (cstart < d_in) {
+    if (cstart < d_in && !tc) {
       dim3 grid((unsigned)kq::cdiv(d_in - cstart, TN), (unsigned)kq::cdiv(d_out, TM));
-      trailing_fp32_kernel<<<grid, 256, 0, st>>>(first ? W : W_hat, first ? ldw : ldwh, W_hat, ldwh, ET, Uc, lduc,
+      trailing_fp32_kernel<<<grid, 256, 0, st>>>(first ? W : W_hat, first ? ldw : ldwh, W_hat, ldwh, w.ET, Uc, lduc,
                                                 first ? dead_mask : nullptr, d_out, d_in, i0, bw, cstart);
       KQ_TRY(kq::launch_check("kq_quantize_layer trailing"));
+    } else if (cstart < d_in) {
+      kq::Gemm3xTF32 g;   // W_hat[:, cstart:] = src[:, cstart:] - E Uc[i0:i0+bw, cstart:]
+      g.M = d_out;
+      g.N = d_in - cstart;
+      g.K = bw;
+      g.a_big = w.Eb;
+      g.a_small = w.Es;
+      g.lda = BLK;
+      g.bt_big = w.Ub;         // Uc^T: (k, n) of Uc[i0:, cstart:] at Ut[cstart + n][i0 + k]
+      g.bt_small = w.Us;
+      g.ldbt = w.ldu;
+      g.bt_row0 = cstart;
+      g.bt_col0 = i0;
+      g.epilogue = kq::kEpiSubtract;
+      g.C = W_hat + cstart;
+      g.ldc = ldwh;
+      g.src = (first ? W : W_hat) + cstart;
+      g.ld_src = first ? ldw : ldwh;
+      g.dead = first && dead_mask ? dead_mask + cstart : nullptr;
+      g.info = info;
+      KQ_TRY(kq::gemm_3xtf32(g, st));
     }
   }
   kq::clear_error();

@@ -30,9 +30,8 @@
 
 #include <algorithm>
 #include <cmath>
-#include <mutex>
 
-#include "kq_internal.cuh"
+#include "kq_tc.cuh"
 
 namespace {
 
@@ -45,11 +44,9 @@ constexpr int STAGE_BYTES = 2 * OPER_BYTES;
 constexpr int THREADS = 192;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 constexpr int ASSUMED_SMS = 148;          // the B200's SM count, used to size splits
-constexpr unsigned long long kTimeoutNs = 4000000000ull;
 
 // Instruction descriptor, kind::f16: D fp32, A/B bf16, both MN-major, M=128, N=256.
-constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) | ((256u >> 3) << 17) |
-                           ((128u >> 4) << 24);
+constexpr uint32_t IDESC = kq::tc::idesc(kq::tc::kFmtBF16, 1, 1, 128, 256);
 
 struct Params {
   int64_t n, d;
@@ -67,117 +64,13 @@ struct Params {
   int32_t* info;
 };
 
-// ------------------------------------------------------------------ PTX
+using namespace kq::tc;
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ unsigned long long globaltimer() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait for the phase with the given parity.  Returns false (and sets
-// the CTA's abort flag, recording a timeout once) when the limit expires or
-// another role already aborted.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int32_t* info,
-                                          int where) {
-  unsigned long long t0 = 0;
-  for (uint32_t it = 0;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0) {
-      if (*abort_flag) return false;
-      unsigned long long now = globaltimer();
-      if (it == 0) {
-        t0 = now;
-      } else if (now - t0 > kTimeoutNs) {
-        *abort_flag = 1;
-        kq::report(info, KQ_ERR_TIMEOUT, where);
-        return false;
-      }
-    }
-  }
-}
-
-// Wait used only while draining after an abort: bounded, never reports.
-__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
-  unsigned long long t0 = globaltimer();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer() - t0 > kTimeoutNs) return;
-  }
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-          dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// Shared-memory matrix descriptor: MN-major operand, 128-byte swizzle.
-// start address >> 4 in bits 0..13; leading byte offset (between 64-element
-// MN atoms) >> 4 in bits 16..29; stride byte offset (between 8-row K groups)
-// >> 4 in bits 32..45; descriptor version 1 in bits 46..47; layout 2
-// (SWIZZLE_128B) in bits 61..63.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
-  const uint64_t lbo = BOX_BYTES >> 4;  // next 64 channels: next TMA box
-  const uint64_t sbo = 1024 >> 4;       // next 8 tokens: 8 rows of 128 bytes
-  return (uint64_t)((addr >> 4) & 0x3FFF) | (lbo << 16) | (sbo << 32) | (1ull << 46) | (2ull << 61);
-}
-
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(IDESC), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+// Shared-memory descriptor of an MN-major 128-byte-swizzled operand: the
+// leading offset steps to the next 64-channel TMA box, the stride offset to
+// the next 8 tokens (8 rows of 128 bytes).
+__device__ __forceinline__ uint64_t operand_desc(uint32_t addr) {
+  return smem_desc(addr, BOX_BYTES, 1024, kSwizzle128);
 }
 
 __device__ __forceinline__ void tri_index(int64_t l, int* ti, int* tj) {
@@ -217,17 +110,13 @@ __global__ void __launch_bounds__(THREADS, 1) syrk_tc_kernel(const __grid_consta
     mbar_init(accempty, 128);
     mbar_init(drained, 1);
     *abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap)) : "memory");
+    mbar_init_fence();
+    prefetch_map(&tmap);
   }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(tmem_slot))
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-  tc_fence_before();
+  if (warp == 1) tmem_alloc<512>(smem_u32(tmem_slot));
+  fence_before();
   __syncthreads();
-  tc_fence_after();
+  fence_after();
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
@@ -290,21 +179,21 @@ __global__ void __launch_bounds__(THREADS, 1) syrk_tc_kernel(const __grid_consta
           ok = false;
           break;
         }
-        tc_fence_after();
+        fence_after();
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, p.info, 3)) {
             ok = false;
             break;
           }
-          tc_fence_after();
+          fence_after();
           const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
           const uint32_t sb = diag ? sa : sa + OPER_BYTES;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             const uint32_t acc = (kb > kb0 || k > 0) ? 1u : 0u;
-            const uint64_t db = smem_desc(sb + k * 2048);
-            mma_bf16(tmem, smem_desc(sa + k * 2048), db, acc);                    // rows 0..127
-            mma_bf16(tmem + 256, smem_desc(sa + 2 * BOX_BYTES + k * 2048), db, acc);  // rows 128..255
+            const uint64_t db = operand_desc(sb + k * 2048);
+            mma_f16<IDESC>(tmem, operand_desc(sa + k * 2048), db, acc);                    // rows 0..127
+            mma_f16<IDESC>(tmem + 256, operand_desc(sa + 2 * BOX_BYTES + k * 2048), db, acc);  // rows 128..255
           }
           any = true;
           mma_commit(empty0 + 8 * stage);   // stage is free once these MMAs have read it
@@ -331,8 +220,12 @@ __global__ void __launch_bounds__(THREADS, 1) syrk_tc_kernel(const __grid_consta
     for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
       int ti, tj, sp;
       unit_coords(p, u, &ti, &tj, &sp);
-      if (!mbar_wait(accfull, acc_phase, abort_flag, p.info, 4)) break;
-      tc_fence_after();
+      // one lane waits, the warp follows: every lane leaves together on abort
+      bool ready = true;
+      if (lane == 0) ready = mbar_wait(accfull, acc_phase, abort_flag, p.info, 4);
+      if (!__shfl_sync(0xffffffffu, ready ? 1 : 0, 0)) break;
+      __syncwarp();
+      fence_after();
       const int64_t i0 = (int64_t)ti * TILE, j0 = (int64_t)tj * TILE;
       const bool diag = (ti == tj);
 #pragma unroll 1
@@ -362,17 +255,17 @@ __global__ void __launch_bounds__(THREADS, 1) syrk_tc_kernel(const __grid_consta
           }
         }
       }
-      tc_fence_before();
+      fence_before();
       mbar_arrive(accempty);
       acc_phase ^= 1u;
     }
   }
 
-  tc_fence_before();
+  fence_before();
   __syncthreads();
   if (warp == 1) {
-    tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+    fence_after();
+    tmem_dealloc<512>(tmem);
   }
 }
 
@@ -462,26 +355,6 @@ Plan make_plan(int64_t n, int64_t d) {
   return pl;
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-kq_status get_encoder(EncodeTiledFn* fn) {
-  static std::mutex mu;
-  static EncodeTiledFn cached = nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!cached) {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q);
-    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !f)
-      return kq::fail(KQ_ERR_CUDA, "kq_accum_cov: cuTensorMapEncodeTiled unavailable");
-    cached = reinterpret_cast<EncodeTiledFn>(f);
-  }
-  *fn = cached;
-  return KQ_OK;
-}
-
 }  // namespace
 
 extern "C" size_t kq_accum_cov_workspace_size(int64_t n, int64_t d) {
@@ -513,17 +386,8 @@ extern "C" kq_status kq_accum_cov(const uint16_t* A, int64_t n, int64_t d, int64
   if (need && (!ws || !kq::aligned(ws, 256) || ws_bytes < need))
     return kq::fail(KQ_ERR_WORKSPACE, "kq_accum_cov: workspace of %zu bytes needed", need);
 
-  EncodeTiledFn encode;
-  KQ_TRY(get_encoder(&encode));
   CUtensorMap tmap;
-  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)n};
-  cuuint64_t strides[1] = {(cuuint64_t)lda * 2};
-  cuuint32_t box[2] = {64, 64};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult cr = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(A), dims, strides, box, estr,
-                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (cr != CUDA_SUCCESS) return kq::fail(KQ_ERR_CUDA, "kq_accum_cov: cuTensorMapEncodeTiled failed (%d)", (int)cr);
+  KQ_TRY(make_map_2d(&tmap, A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, n, lda, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B));
 
   Params p;
   p.n = n;

@@ -209,7 +209,7 @@ def test_chol_inv_dead_columns_and_errors(P):
 
 # ------------------------------------------------------------------ quantize
 
-def _quant_case(P, W, Uc, dead, bits, group):
+def _quant_case(P, W, Uc, dead, bits, group, gemm_mode=None):
     d_out, d_in = W.shape
     ng = 1 if not group else -(-d_in // group)
     codes = torch.empty((d_out, d_in), dtype=torch.uint8, device="cuda")
@@ -217,7 +217,8 @@ def _quant_case(P, W, Uc, dead, bits, group):
     zeros = torch.empty((d_out, ng), device="cuda")
     W_hat = torch.empty((d_out, d_in), device="cuda")
     info = _info()
-    P.kq_quantize_layer(W, Uc, dead, bits, group, codes, scales, zeros, W_hat, info=info)
+    mode = P.KQ_GEMM_FP32 if gemm_mode is None else gemm_mode
+    P.kq_quantize_layer(W, Uc, dead, bits, group, codes, scales, zeros, W_hat, gemm_mode=mode, info=info)
     torch.cuda.synchronize()
     assert _info_code(info)[0] == 0
     return codes.cpu().numpy(), scales.cpu().numpy(), zeros.cpu().numpy(), np64(W_hat)
@@ -265,9 +266,11 @@ def rotated_small(P):
 
 
 @pytest.mark.parametrize("bits,group", [(2, 0), (3, 0), (4, 0), (3, 128), (2, 128), (8, 0), (4, 32)])
-def test_quantize_parity(P, rotated_small, bits, group):
+@pytest.mark.parametrize("mode", ["fp32", "3xtf32"])
+def test_quantize_parity(P, rotated_small, bits, group, mode):
     lq, _ = rotated_small
-    got = _quant_case(P, lq.Wp, lq.Uc, lq.dead, bits, group)
+    gm = P.KQ_GEMM_FP32 if mode == "fp32" else P.KQ_GEMM_3XTF32
+    got = _quant_case(P, lq.Wp, lq.Uc, lq.dead, bits, group, gm)
     _check_quant(lq.Wp, lq.Uc, lq.dead, bits, group, got)
 
 
@@ -301,8 +304,9 @@ def test_quantize_dead_columns_degenerate_rows(P):
     P.kq_chol_inv(torch.from_numpy(H).cuda(), 0.01, Uc, dead, None, _info())
     Wg = torch.from_numpy(W).cuda()
     for group in (0, 128):
-        got = _quant_case(P, Wg, Uc, dead, 3, group)
-        _check_quant(Wg, Uc, dead, 3, group, got)
+        for gm in (P.KQ_GEMM_FP32, P.KQ_GEMM_3XTF32):
+            got = _quant_case(P, Wg, Uc, dead, 3, group, gm)
+            _check_quant(Wg, Uc, dead, 3, group, got)
 
 
 def test_quantize_constant_row_per_channel(P):
@@ -332,6 +336,23 @@ def test_quantize_nonfinite_reported(P):
 
 
 # ------------------------------------------------------------------ loss
+
+@pytest.mark.parametrize("d_out,d_in", [(352, 704), (200, 136), (40, 300), (513, 260)])
+@pytest.mark.parametrize("with_hg", [True, False])
+def test_kron_loss_shapes(P, d_out, d_in, with_hg):
+    """Ragged tile edges and K tails of the tensor-core products."""
+    rng = np.random.default_rng(d_out * 7 + d_in)
+    W = rng.normal(0, 0.02, (d_out, d_in)).astype(np.float32)
+    Wh = (W + rng.normal(0, 0.004, W.shape)).astype(np.float32)
+    HX = _spd(d_in, 1, 1.0)
+    HG = _spd(d_out, 2, 1.0)
+    loss = torch.zeros(1, dtype=torch.float64, device="cuda")
+    P.kq_kron_loss(torch.from_numpy(W).cuda(), torch.from_numpy(Wh).cuda(), torch.from_numpy(HX).cuda(),
+                   torch.from_numpy(HG).cuda() if with_hg else None, loss)
+    ref = O.kron_loss(W.astype(np.float64), Wh.astype(np.float64), HX.astype(np.float64),
+                      HG.astype(np.float64) if with_hg else None)
+    assert abs(loss.item() - ref) <= 1e-3 * abs(ref), (loss.item(), ref)
+
 
 @pytest.mark.parametrize("with_hg", [True, False])
 def test_kron_loss_parity(P, rotated_small, with_hg):
