@@ -13,11 +13,11 @@
 // final Uc is rounded to fp32.
 //
 // Blocked right-looking algorithms over nb = 64 tiles:
-//   Cholesky, per block column k: factor + invert the diagonal block (1 CTA),
-//   panel  X = A_panel L_kk^-T (GEMM with the inverted block),
-//   trailing lower-triangle update A -= P P^T.
-//   Inverse, per block row i (forward substitution on B = I):
-//   X_i = L_ii^-1 B_i, then B_below -= L_below,i X_i.
+//   per block column k: factor + invert the diagonal block (1 CTA); then one
+//   launch for the panel X = A_panel L_kk^-T (GEMM with the inverted block)
+//   and row block k of the inverse, X_k = L_kk^-1 B_k (forward substitution
+//   on B = I); then one launch for the trailing lower-triangle update
+//   A -= P P^T and the substitution update B_below -= L_below,k X_k.
 #include <math.h>
 
 #include <algorithm>
@@ -127,69 +127,74 @@ __global__ void damp_kernel(double* __restrict__ A, int64_t n, double damp, doub
   if (threadIdx.x == 0) *lam_out = lam;
 }
 
-// Factor the kb x kb diagonal block at (k0, k0) in place and write its
-// inverse (padded to 64x64 with the identity) to Dinv.
+// Factor the kb x kb diagonal block at (k0, k0) in place (lower Cholesky) and
+// write its lower-triangular inverse, padded to 64 x 64 with the identity, to
+// Dinv.  256 threads: four per row (Cholesky, left-looking by columns, the
+// dot products split four ways) or four per column (inverse, forward
+// substitution with split dot products).  Two block barriers per column.
 __global__ void __launch_bounds__(256) potrf_kernel(double* __restrict__ A, int64_t n, int64_t k0, int kb,
                                                     double* __restrict__ Dinv, int32_t* info) {
   extern __shared__ double psm[];
   double (*a)[kPad] = reinterpret_cast<double (*)[kPad]>(psm);
   double (*inv)[kPad] = reinterpret_cast<double (*)[kPad]>(psm + NB * kPad);
-  for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) {
+  __shared__ double rdiag[NB];
+  __shared__ double diag0[NB];   // the block's diagonal before factorisation (read-only below)
+  const int t = threadIdx.x, g = t >> 2, part = t & 3;
+  for (int idx = t; idx < NB * NB; idx += blockDim.x) {
     int i = idx / NB, j = idx % NB;
     double v;
     if (i < kb && j < kb) v = (j <= i) ? A[(k0 + i) * n + k0 + j] : 0.0;
     else v = (i == j) ? 1.0 : 0.0;
     a[i][j] = v;
+    if (i == j) diag0[i] = v;
   }
   __syncthreads();
+  // Column j: every 4-thread group forms its own row's dot product and the
+  // pivot row's (same operands, same order, so every group holds the same
+  // pivot), scales by 1/sqrt(pivot) and the column is final after one barrier.
   for (int j = 0; j < NB; ++j) {
-    if (threadIdx.x == 0) {
-      double d = a[j][j];
-      if (!(d > 0.0) || !isfinite(d)) {
-        kq::report(info, KQ_ERR_NOT_PD, n - 1 - (k0 + j));
-        d = 1.0;
-      }
-      a[j][j] = sqrt(d);
+    const int i = g;
+    double s = 0.0, sp = 0.0;
+    for (int l = part; l < j; l += 4) {
+      sp = fma(a[j][l], a[j][l], sp);
+      if (i > j) s = fma(a[i][l], a[j][l], s);
     }
-    __syncthreads();
-    const double piv = a[j][j];
-    for (int i = j + 1 + threadIdx.x; i < NB; i += blockDim.x) a[i][j] /= piv;
-    __syncthreads();
-    const int m = NB - 1 - j;  // trailing size
-    for (int idx = threadIdx.x; idx < m * m; idx += blockDim.x) {
-      int i = j + 1 + idx / m, l = j + 1 + idx % m;
-      if (l <= i) a[i][l] -= a[i][j] * a[l][j];
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    s += __shfl_xor_sync(0xffffffffu, s, 2);
+    sp += __shfl_xor_sync(0xffffffffu, sp, 1);
+    sp += __shfl_xor_sync(0xffffffffu, sp, 2);
+    double d = diag0[j] - sp;
+    if (!(d > 0.0) || !isfinite(d)) {
+      if (i == j && part == 0) kq::report(info, KQ_ERR_NOT_PD, n - 1 - (k0 + j));
+      d = 1.0;
+    }
+    const double rs = rsqrt(d);
+    if (part == 0) {
+      if (i == j) a[j][j] = d * rs;
+      else if (i > j) a[i][j] = (a[i][j] - s) * rs;
     }
     __syncthreads();
   }
-  // Lower triangular inverse, one column per thread (forward substitution).
-  if (threadIdx.x < NB) {
-    const int c = threadIdx.x;
-    for (int i = 0; i < c; ++i) inv[i][c] = 0.0;
-    inv[c][c] = 1.0 / a[c][c];
-    for (int i = c + 1; i < NB; ++i) {
+  if (t < NB) rdiag[t] = 1.0 / a[t][t];
+  __syncthreads();
+  {
+    const int c = g;
+    for (int i = 0; i < NB; ++i) {
       double s = 0.0;
-      for (int l = c; l < i; ++l) s = fma(a[i][l], inv[l][c], s);
-      inv[i][c] = -s / a[i][i];
+      if (i > c)
+        for (int l = c + part; l < i; l += 4) s = fma(a[i][l], inv[l][c], s);
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      if (part == 0) inv[i][c] = (i < c) ? 0.0 : (i == c ? rdiag[c] : -s * rdiag[i]);
+      __syncwarp();
     }
   }
   __syncthreads();
-  for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) {
+  for (int idx = t; idx < NB * NB; idx += blockDim.x) {
     int i = idx / NB, j = idx % NB;
     Dinv[idx] = inv[i][j];
     if (i < kb && j < kb && j <= i) A[(k0 + i) * n + k0 + j] = a[i][j];
   }
-}
-
-// Panel: rows r in [r0 + 64 b, ...) of block column k0: X = A_panel Dinv^T.
-__global__ void __launch_bounds__(kGemmThreads) panel_kernel(double* __restrict__ A, int64_t n, int64_t k0, int kb,
-                                                             const double* __restrict__ Dinv) {
-  extern __shared__ double smem[];
-  const int64_t r0 = k0 + kb + (int64_t)blockIdx.x * NB;
-  const int rv = (int)dmin64(NB, n - r0);
-  double* P = A + r0 * n + k0;
-  // A(r,k) = P[r*n + k];  B(k,c) = Dinv[c][k] = Dinv[c*64 + k]
-  gemm_tile(smem, P, n, 1, Dinv, NB, 1, kb, P, n, rv, kb, 1.0, 0.0);
 }
 
 __device__ __forceinline__ void tri_index(int64_t l, int64_t* ti, int64_t* tj) {
@@ -200,17 +205,54 @@ __device__ __forceinline__ void tri_index(int64_t l, int64_t* ti, int64_t* tj) {
   *tj = l - t * (t + 1) / 2;
 }
 
-// Trailing update of the lower tiles: A[ti][tj] -= P_ti P_tj^T.
-__global__ void __launch_bounds__(kGemmThreads) trailing_kernel(double* __restrict__ A, int64_t n, int64_t k0,
-                                                                int kb) {
+// One launch per block step k (after the diagonal factorisation):
+//   CTAs [0, tr):     panel rows below the block, X = A_panel Dinv_k^T;
+//   CTAs [tr, ...):   forward substitution, X_k = Dinv_k B_k for column
+//                     blocks 0..k of the inverse being formed in B.
+__global__ void __launch_bounds__(kGemmThreads) step_a_kernel(double* __restrict__ A, double* __restrict__ X,
+                                                             int64_t n, int64_t k0, int kb, int64_t tr,
+                                                             const double* __restrict__ Dinv) {
   extern __shared__ double smem[];
-  int64_t ti, tj;
-  tri_index(blockIdx.x, &ti, &tj);
+  if ((int64_t)blockIdx.x < tr) {
+    const int64_t r0 = k0 + kb + (int64_t)blockIdx.x * NB;
+    const int rv = (int)dmin64(NB, n - r0);
+    double* P = A + r0 * n + k0;
+    // A(r,k) = P[r*n + k];  B(k,c) = Dinv[c][k]
+    gemm_tile(smem, P, n, 1, Dinv, NB, 1, kb, P, n, rv, kb, 1.0, 0.0);
+  } else {
+    const int64_t c0 = ((int64_t)blockIdx.x - tr) * NB;
+    const int cv = (int)dmin64(NB, n - c0);
+    double* T = X + k0 * n + c0;
+    // A(r,k) = Dinv[r*64 + k];  B(k,c) = T[k*n + c]
+    gemm_tile(smem, Dinv, NB, 1, T, 1, n, kb, T, n, kb, cv, 1.0, 0.0);
+  }
+}
+
+// One launch per block step k (after step_a):
+//   CTAs [0, tr(tr+1)/2):  Cholesky trailing update of the lower tiles,
+//                          A[ti][tj] -= P_ti P_tj^T;
+//   CTAs after:            substitution update of the rows below,
+//                          B[r][c] -= L[r][k] X_k[c] for column blocks c <= k.
+__global__ void __launch_bounds__(kGemmThreads) step_b_kernel(double* __restrict__ A, double* __restrict__ X,
+                                                             int64_t n, int64_t k0, int kb, int64_t tr,
+                                                             int64_t kblocks) {
+  extern __shared__ double smem[];
+  const int64_t ntri = tr * (tr + 1) / 2;
   const int64_t base = k0 + kb;
-  const int64_t r0 = base + ti * NB, c0 = base + tj * NB;
-  const int rv = (int)dmin64(NB, n - r0), cv = (int)dmin64(NB, n - c0);
-  // A(r,k) = A[(r0+r)*n + k0 + k];  B(k,c) = A[(c0+c)*n + k0 + k]
-  gemm_tile(smem, A + r0 * n + k0, n, 1, A + c0 * n + k0, n, 1, kb, A + r0 * n + c0, n, rv, cv, -1.0, 1.0);
+  if ((int64_t)blockIdx.x < ntri) {
+    int64_t ti, tj;
+    tri_index(blockIdx.x, &ti, &tj);
+    const int64_t r0 = base + ti * NB, c0 = base + tj * NB;
+    const int rv = (int)dmin64(NB, n - r0), cv = (int)dmin64(NB, n - c0);
+    gemm_tile(smem, A + r0 * n + k0, n, 1, A + c0 * n + k0, n, 1, kb, A + r0 * n + c0, n, rv, cv, -1.0, 1.0);
+  } else {
+    const int64_t idx = (int64_t)blockIdx.x - ntri;
+    const int64_t cb = idx % kblocks, rb = idx / kblocks;
+    const int64_t c0 = cb * NB, r0 = base + rb * NB;
+    const int cv = (int)dmin64(NB, n - c0), rv = (int)dmin64(NB, n - r0);
+    // A(r,k) = L[(r0+r)*n + k0 + k];  B(k,c) = X[(k0+k)*n + c0 + c]
+    gemm_tile(smem, A + r0 * n + k0, n, 1, X + k0 * n + c0, 1, n, kb, X + r0 * n + c0, n, rv, cv, -1.0, 1.0);
+  }
 }
 
 __global__ void identity_kernel(double* __restrict__ X, int64_t n) {
@@ -218,28 +260,6 @@ __global__ void identity_kernel(double* __restrict__ X, int64_t n) {
   for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += (int64_t)gridDim.x * blockDim.x)
     X[idx] = (idx / n == idx % n) ? 1.0 : 0.0;
-}
-
-// X[i-block, c-block] = Dinv_i X[i-block, c-block] for c-blocks 0..i.
-__global__ void __launch_bounds__(kGemmThreads) rowsolve_kernel(double* __restrict__ X, int64_t n, int64_t i0, int ib,
-                                                                const double* __restrict__ Dinv) {
-  extern __shared__ double smem[];
-  const int64_t c0 = (int64_t)blockIdx.x * NB;
-  const int cv = (int)dmin64(NB, n - c0);
-  double* T = X + i0 * n + c0;
-  // A(r,k) = Dinv[r*64 + k];  B(k,c) = T[k*n + c]
-  gemm_tile(smem, Dinv, NB, 1, T, 1, n, ib, T, n, ib, cv, 1.0, 0.0);
-}
-
-// B[r-block, c-block] -= L[r-block, i-block] X[i-block, c-block], r > i, c <= i.
-__global__ void __launch_bounds__(kGemmThreads) fsub_update_kernel(double* __restrict__ X, const double* __restrict__ L,
-                                                                   int64_t n, int64_t i0, int ib) {
-  extern __shared__ double smem[];
-  const int64_t c0 = (int64_t)blockIdx.x * NB;
-  const int64_t r0 = i0 + ib + (int64_t)blockIdx.y * NB;
-  const int cv = (int)dmin64(NB, n - c0), rv = (int)dmin64(NB, n - r0);
-  // A(r,k) = L[(r0+r)*n + i0 + k];  B(k,c) = X[(i0+k)*n + c0 + c]
-  gemm_tile(smem, L + r0 * n + i0, n, 1, X + i0 * n + c0, 1, n, ib, X + r0 * n + c0, n, rv, cv, -1.0, 1.0);
 }
 
 // Uc[i][j] = X[n-1-i][n-1-j] for j >= i, 0 below the diagonal.
@@ -299,44 +319,35 @@ extern "C" kq_status kq_chol_inv(const float* H, int64_t n, int64_t ldh, float d
   ws_layout(n, &w, ws);
   static_assert(kGemmSmem <= 227 * 1024, "smem");
   KQ_TRY(kq::cuda_check(cudaFuncSetAttribute(potrf_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem), "attr"));
-  KQ_TRY(kq::cuda_check(cudaFuncSetAttribute(panel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem), "attr"));
-  KQ_TRY(kq::cuda_check(cudaFuncSetAttribute(trailing_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem), "attr"));
-  KQ_TRY(kq::cuda_check(cudaFuncSetAttribute(rowsolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem), "attr"));
-  KQ_TRY(kq::cuda_check(cudaFuncSetAttribute(fsub_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem), "attr"));
+  KQ_TRY(kq::cuda_check(cudaFuncSetAttribute(step_a_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem), "attr"));
+  KQ_TRY(kq::cuda_check(cudaFuncSetAttribute(step_b_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem), "attr"));
 
   const unsigned nt = (unsigned)kq::cdiv(n, 32);
   prep_kernel<<<dim3(nt, nt), dim3(32, 8), 0, st>>>(H, ldh, n, w.A, dead_mask, info);
   KQ_TRY(kq::launch_check("kq_chol_inv prep"));
   damp_kernel<<<1, 1024, 0, st>>>(w.A, n, (double)damp_frac, w.lam);
   KQ_TRY(kq::launch_check("kq_chol_inv damp"));
+  identity_kernel<<<1024, 256, 0, st>>>(w.X, n);
+  KQ_TRY(kq::launch_check("kq_chol_inv identity"));
 
+  // Cholesky of the reversed matrix and the inverse of its factor, formed
+  // together: step k factors diagonal block k, then (a) its panel and the
+  // k-th block row of the inverse, then (b) the trailing Cholesky update and
+  // the substitution update of the inverse's rows below.
   const int64_t nblk = kq::cdiv(n, NB);
   for (int64_t b = 0; b < nblk; ++b) {
     const int64_t k0 = b * NB;
     const int kb = (int)std::min<int64_t>(NB, n - k0);
-    potrf_kernel<<<1, 256, kGemmSmem, st>>>(w.A, n, k0, kb, w.Dinv + b * NB * NB, info);
+    double* Dk = w.Dinv + b * NB * NB;
+    potrf_kernel<<<1, 256, kGemmSmem, st>>>(w.A, n, k0, kb, Dk, info);
     KQ_TRY(kq::launch_check("kq_chol_inv potrf"));
-    const int64_t rest = n - k0 - kb;
-    if (rest > 0) {
-      const int64_t tr = kq::cdiv(rest, NB);
-      panel_kernel<<<(unsigned)tr, kGemmThreads, kGemmSmem, st>>>(w.A, n, k0, kb, w.Dinv + b * NB * NB);
-      KQ_TRY(kq::launch_check("kq_chol_inv panel"));
-      trailing_kernel<<<(unsigned)(tr * (tr + 1) / 2), kGemmThreads, kGemmSmem, st>>>(w.A, n, k0, kb);
-      KQ_TRY(kq::launch_check("kq_chol_inv trailing"));
-    }
-  }
-  identity_kernel<<<1024, 256, 0, st>>>(w.X, n);
-  KQ_TRY(kq::launch_check("kq_chol_inv identity"));
-  for (int64_t b = 0; b < nblk; ++b) {
-    const int64_t i0 = b * NB;
-    const int ib = (int)std::min<int64_t>(NB, n - i0);
-    rowsolve_kernel<<<(unsigned)(b + 1), kGemmThreads, kGemmSmem, st>>>(w.X, n, i0, ib, w.Dinv + b * NB * NB);
-    KQ_TRY(kq::launch_check("kq_chol_inv rowsolve"));
-    const int64_t rest = n - i0 - ib;
-    if (rest > 0) {
-      fsub_update_kernel<<<dim3((unsigned)(b + 1), (unsigned)kq::cdiv(rest, NB)), kGemmThreads, kGemmSmem, st>>>(
-          w.X, w.A, n, i0, ib);
-      KQ_TRY(kq::launch_check("kq_chol_inv update"));
+    const int64_t tr = kq::cdiv(n - k0 - kb, NB);
+    step_a_kernel<<<(unsigned)(tr + b + 1), kGemmThreads, kGemmSmem, st>>>(w.A, w.X, n, k0, kb, tr, Dk);
+    KQ_TRY(kq::launch_check("kq_chol_inv step a"));
+    if (tr > 0) {
+      step_b_kernel<<<(unsigned)(tr * (tr + 1) / 2 + tr * (b + 1)), kGemmThreads, kGemmSmem, st>>>(w.A, w.X, n, k0,
+                                                                                                   kb, tr, b + 1);
+      KQ_TRY(kq::launch_check("kq_chol_inv step b"));
     }
   }
   output_kernel<<<(unsigned)n, 256, 0, st>>>(w.X, n, Uc, lduc);
