@@ -142,7 +142,8 @@ kq_status kq_sensitivity(const float* H_X, int64_t d_in, int64_t ldhx,
  *   axis == KQ_AXIS_COLS : M <- M . T^T  (T acts on the column index; T->n == cols)
  *   inverse != 0 applies T^T instead of T.
  * In place on fp32 M [rows, cols], ld >= cols, 16-byte aligned, ld % 4 == 0.
- * Limits: 1 <= m <= 64, 0 <= log2_p <= 15, n <= 65536; T->signs device
+ * Limits: 1 <= m <= 64, 0 <= log2_p <= 15, n <= 32768, and for
+ * KQ_AXIS_ROWS also m * max(1, p / 128) <= 256; T->signs device
  * fp32[n] of +-1; T->Qm device fp32[m*m] row-major orthogonal, may be NULL
  * only when m == 1.  BiIP of a layer is:
  *   W:   kq_rotate(W,  KQ_AXIS_COLS, U) then kq_rotate(W, KQ_AXIS_ROWS, V)

@@ -9,13 +9,13 @@
 // T = (Q_m kron H_p / sqrt(p)) diag(s), n = m p.  The transform is HBM bound
 // (8 bytes per element per pass), so the kernels stage a whole vector (row
 // transform) or a strided tile of vectors (column transform) in shared memory,
-// run the Walsh-Hadamard butterflies there, and touch HBM once per pass with
-// coalesced 128-byte rows.
+// run the Walsh-Hadamard butterflies there (radix-16 passes in registers),
+// and touch HBM once per pass with coalesced float4 accesses.
 //
 //  * KQ_AXIS_COLS (M <- M T^T, each row transformed): one CTA per row, the row
 //    lives in shared memory (n <= 32768 floats).
 //  * KQ_AXIS_ROWS (M <- T M, each column transformed): H_p = H_p1 kron H_p2 is
-//    split into two passes over 32-column strips.  Pass "inner" applies H_p2 to
+//    split into two passes over 128-column strips (512-byte row runs).  Pass "inner" applies H_p2 to
 //    groups of p2 consecutive rows (plus signs and the 1/sqrt(p) scale); pass
 //    "outer" applies H_p1 and Q_m to the m*p1 rows that share one inner index
 //    (stride p2).  Each pass reads and writes M once.
@@ -25,82 +25,144 @@ namespace {
 
 constexpr int kMaxM = 64;
 constexpr int kMaxRowN = 32768;
-constexpr int kStrip = 32;           // columns per tile in the column transform
-constexpr int kMaxP2Log = 9;         // p2 <= 512
-constexpr int kMaxOuterRows = 1024;  // m * p1 <= 1024
+constexpr int kStrip = 128;          // columns per tile in the column transform (512-byte row runs)
+constexpr int kMaxP2Log = 7;         // inner pass: p2 <= 128 rows
+constexpr int kMaxOuterRows = 256;   // outer pass: m * p1 <= 256 rows
 
-// In-smem butterflies over blocks of `len` contiguous elements (len = 2^k)
-// of a vector of `n` elements, all threads of the CTA cooperating.
-__device__ __forceinline__ void fwht_smem(float* x, int n, int len) {
-  for (int h = 1; h < len; h <<= 1) {
-    for (int idx = threadIdx.x; idx < n / 2; idx += blockDim.x) {
-      int i = (idx / h) * (2 * h) + (idx % h);
-      float a = x[i], b = x[i + h];
-      x[i] = a + b;
-      x[i + h] = a - b;
+// Shared-memory position of element i of a row: one spare float after every
+// 16, so a thread reading 16 consecutive elements, and a warp reading 32
+// such runs, meets no bank conflict.
+__device__ __forceinline__ int pad16(int i) { return i + (i >> 4); }
+
+// Butterflies over index bits [lo, lo + g) of 2^g register-held elements
+// (g <= 4; predicated for g < 4).
+__device__ __forceinline__ void fwht_regs(float (&r)[16], int g) {
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    if (s >= g) break;
+    const int h = 1 << s;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      if ((e & h) || e + h >= (1 << g)) continue;
+      const float a = r[e], b = r[e + h];
+      r[e] = a + b;
+      r[e + h] = a - b;
+    }
+  }
+}
+
+// y[a] = sum_c Q[a][c] x[c] (or Q^T) for one strand of m <= 64 values kept in
+// registers (fully unrolled over the 64 slots, predicated on m).
+template <typename Get, typename Put>
+__device__ __forceinline__ void qmix_strand(const float* Qs, int m, bool transpose, Get get, Put put) {
+  float x[kMaxM];
+#pragma unroll
+  for (int c = 0; c < kMaxM; ++c) x[c] = (c < m) ? get(c) : 0.f;
+  for (int a = 0; a < m; ++a) {
+    float acc = 0.f;
+#pragma unroll
+    for (int c = 0; c < kMaxM; ++c)
+      if (c < m) acc = fmaf(transpose ? Qs[c * m + a] : Qs[a * m + c], x[c], acc);
+    put(a, acc);
+  }
+}
+
+// Walsh-Hadamard butterflies over bits [0, k) of the element index of nvec
+// vectors held in shared memory, in passes over 4-bit groups of the index:
+// each thread gathers the 16 elements of one group into registers, runs the
+// butterflies there and scatters them back (index arithmetic by shifts and
+// masks only).
+//   ROW layout:  element i of vector v at pad16(v * 2^k + i)
+//   TILE layout: element i of vector v (v = column + 128 * block) at
+//                ((v >> 7) * 2^k + i) * 128 + (v & 127)
+template <bool ROW>
+__device__ void fwht_passes(float* x, int k, int nvec) {
+  for (int lo = 0; lo < k; lo += 4) {
+    const int g = min(4, k - lo);
+    const int rest_bits = k - g;
+    const int groups = nvec << rest_bits;
+    for (int grp = threadIdx.x; grp < groups; grp += blockDim.x) {
+      int v, rest;
+      if (ROW) {
+        v = grp >> rest_bits;
+        rest = grp & ((1 << rest_bits) - 1);
+      } else {
+        v = (grp & 127) | ((grp >> (7 + rest_bits)) << 7);
+        rest = (grp >> 7) & ((1 << rest_bits) - 1);
+      }
+      const int base = ((rest >> lo) << (lo + g)) | (rest & ((1 << lo) - 1));
+      float r[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        if (e >= (1 << g)) break;
+        const int i = base | (e << lo);
+        r[e] = ROW ? x[pad16((v << k) + i)] : x[(((v >> 7) << k) + i) * 128 + (v & 127)];
+      }
+      fwht_regs(r, g);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        if (e >= (1 << g)) break;
+        const int i = base | (e << lo);
+        if (ROW) x[pad16((v << k) + i)] = r[e];
+        else x[(((v >> 7) << k) + i) * 128 + (v & 127)] = r[e];
+      }
     }
     __syncthreads();
   }
 }
 
-// Mix the m blocks of p elements with Q (or Q^T): x[a*p+b] <- sum_a' Q[a][a'] x[a'*p+b].
-__device__ __forceinline__ void qmix_smem(float* x, int p, int m, const float* Qs, bool transpose) {
-  float tmp[kMaxM];
-  for (int b = threadIdx.x; b < p; b += blockDim.x) {
-    for (int a = 0; a < m; ++a) tmp[a] = x[a * p + b];
-    for (int a = 0; a < m; ++a) {
-      float acc = 0.f;
-      for (int c = 0; c < m; ++c) acc = fmaf(transpose ? Qs[c * m + a] : Qs[a * m + c], tmp[c], acc);
-      x[a * p + b] = acc;
-    }
-  }
-  __syncthreads();
-}
-
-// Row transform: M[r, :] <- T M[r, :] (or T^T).  One CTA per row.
-__global__ void __launch_bounds__(512) rotate_rows_kernel(float* __restrict__ M, int64_t ld, int n, int log2_p, int m,
+// Row transform: M[r, :] <- T M[r, :] (or T^T).  One CTA per row; the row
+// lives in shared memory in the padded layout.
+__global__ void __launch_bounds__(256) rotate_rows_kernel(float* __restrict__ M, int64_t ld, int n, int log2_p, int m,
                                                           const float* __restrict__ signs,
                                                           const float* __restrict__ Qm, int inverse, float scale) {
   extern __shared__ float sm[];
   float* x = sm;
-  float* Qs = sm + n;
+  float* Qs = sm + pad16(n) + 4;
   const int p = 1 << log2_p;
   float* row = M + (int64_t)blockIdx.x * ld;
   if (m > 1)
     for (int i = threadIdx.x; i < m * m; i += blockDim.x) Qs[i] = Qm[i];
   if ((n & 3) == 0) {
-    const float4* src = reinterpret_cast<const float4*>(row);
-    const float4* sg = reinterpret_cast<const float4*>(signs);
-    for (int i = threadIdx.x; i < n / 4; i += blockDim.x) {
-      float4 v = src[i];
+    for (int i4 = threadIdx.x; i4 < n / 4; i4 += blockDim.x) {
+      float4 v = reinterpret_cast<const float4*>(row)[i4];
       if (!inverse) {
-        float4 s = sg[i];
-        v.x *= s.x; v.y *= s.y; v.z *= s.z; v.w *= s.w;
+        const float4 sg = reinterpret_cast<const float4*>(signs)[i4];
+        v.x *= sg.x; v.y *= sg.y; v.z *= sg.z; v.w *= sg.w;
       }
-      reinterpret_cast<float4*>(x)[i] = v;
+      const int i = 4 * i4;
+      x[pad16(i)] = v.x;
+      x[pad16(i + 1)] = v.y;
+      x[pad16(i + 2)] = v.z;
+      x[pad16(i + 3)] = v.w;
     }
   } else {
-    for (int i = threadIdx.x; i < n; i += blockDim.x) x[i] = inverse ? row[i] : row[i] * signs[i];
+    for (int i = threadIdx.x; i < n; i += blockDim.x) x[pad16(i)] = inverse ? row[i] : row[i] * signs[i];
   }
   __syncthreads();
-  if (inverse && m > 1) qmix_smem(x, p, m, Qs, true);
-  fwht_smem(x, n, p);
-  if (!inverse && m > 1) qmix_smem(x, p, m, Qs, false);
+  auto qmix = [&](bool transpose) {
+    for (int b = threadIdx.x; b < p; b += blockDim.x)
+      qmix_strand(Qs, m, transpose, [&](int c) { return x[pad16(c * p + b)]; },
+                  [&](int a, float v) { x[pad16(a * p + b)] = v; });
+    __syncthreads();
+  };
+  if (inverse && m > 1) qmix(true);
+  fwht_passes<true>(x, log2_p, m);
+  if (!inverse && m > 1) qmix(false);
   if ((n & 3) == 0) {
-    float4* dst = reinterpret_cast<float4*>(row);
-    const float4* sg = reinterpret_cast<const float4*>(signs);
-    for (int i = threadIdx.x; i < n / 4; i += blockDim.x) {
-      float4 v = reinterpret_cast<float4*>(x)[i];
-      v.x *= scale; v.y *= scale; v.z *= scale; v.w *= scale;
+    for (int i4 = threadIdx.x; i4 < n / 4; i4 += blockDim.x) {
+      const int i = 4 * i4;
+      float4 v = make_float4(x[pad16(i)] * scale, x[pad16(i + 1)] * scale, x[pad16(i + 2)] * scale,
+                             x[pad16(i + 3)] * scale);
       if (inverse) {
-        float4 s = sg[i];
-        v.x *= s.x; v.y *= s.y; v.z *= s.z; v.w *= s.w;
+        const float4 sg = reinterpret_cast<const float4*>(signs)[i4];
+        v.x *= sg.x; v.y *= sg.y; v.z *= sg.z; v.w *= sg.w;
       }
-      dst[i] = v;
+      reinterpret_cast<float4*>(row)[i4] = v;
     }
   } else {
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      float v = x[i] * scale;
+      const float v = x[pad16(i)] * scale;
       row[i] = inverse ? v * signs[i] : v;
     }
   }
@@ -111,35 +173,45 @@ __global__ void __launch_bounds__(512) rotate_rows_kernel(float* __restrict__ M,
 // (forward: before), H_p2 along the rows, the 1/sqrt(p) scale, and (inverse:
 // after) the signs.
 __global__ void __launch_bounds__(256) rotate_cols_inner_kernel(float* __restrict__ M, int64_t ld, int64_t cols,
-                                                                int p2, const float* __restrict__ signs, int inverse,
-                                                                float scale) {
-  extern __shared__ float t[];  // [p2][kStrip]
+                                                                int log2_p2, const float* __restrict__ signs,
+                                                                int inverse, float scale) {
+  extern __shared__ float t[];  // [p2][128]
+  const int p2 = 1 << log2_p2;
   const int64_t r0 = (int64_t)blockIdx.y * p2;
   const int64_t c0 = (int64_t)blockIdx.x * kStrip;
-  const int c = threadIdx.x % kStrip;
-  const int rs = threadIdx.x / kStrip;
-  const int rstep = blockDim.x / kStrip;
-  const bool cok = c0 + c < cols;
+  const int c4 = 4 * (threadIdx.x % (kStrip / 4));   // this thread's 4 columns
+  const int rs = threadIdx.x / (kStrip / 4);
+  const int rstep = blockDim.x / (kStrip / 4);
+  const bool full = c0 + c4 + 3 < cols;
   for (int r = rs; r < p2; r += rstep) {
-    float v = cok ? M[(r0 + r) * ld + c0 + c] : 0.f;
-    if (!inverse) v *= signs[r0 + r];
-    t[r * kStrip + c] = v;
+    const float* src = M + (r0 + r) * ld + c0 + c4;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (full) {
+      v = *reinterpret_cast<const float4*>(src);
+    } else {
+      if (c0 + c4 + 0 < cols) v.x = src[0];
+      if (c0 + c4 + 1 < cols) v.y = src[1];
+      if (c0 + c4 + 2 < cols) v.z = src[2];
+    }
+    if (!inverse) {
+      const float sg = signs[r0 + r];
+      v.x *= sg; v.y *= sg; v.z *= sg; v.w *= sg;
+    }
+    *reinterpret_cast<float4*>(t + r * kStrip + c4) = v;
   }
   __syncthreads();
-  for (int h = 1; h < p2; h <<= 1) {
-    for (int idx = rs; idx < p2 / 2; idx += rstep) {
-      int i = (idx / h) * (2 * h) + (idx % h);
-      float a = t[i * kStrip + c], b = t[(i + h) * kStrip + c];
-      t[i * kStrip + c] = a + b;
-      t[(i + h) * kStrip + c] = a - b;
-    }
-    __syncthreads();
-  }
-  if (cok) {
-    for (int r = rs; r < p2; r += rstep) {
-      float v = t[r * kStrip + c] * scale;
-      if (inverse) v *= signs[r0 + r];
-      M[(r0 + r) * ld + c0 + c] = v;
+  fwht_passes<false>(t, log2_p2, kStrip);
+  for (int r = rs; r < p2; r += rstep) {
+    float4 v = *reinterpret_cast<const float4*>(t + r * kStrip + c4);
+    const float f = inverse ? scale * signs[r0 + r] : scale;
+    v.x *= f; v.y *= f; v.z *= f; v.w *= f;
+    float* dst = M + (r0 + r) * ld + c0 + c4;
+    if (full) {
+      *reinterpret_cast<float4*>(dst) = v;
+    } else {
+      if (c0 + c4 + 0 < cols) dst[0] = v.x;
+      if (c0 + c4 + 1 < cols) dst[1] = v.y;
+      if (c0 + c4 + 2 < cols) dst[2] = v.z;
     }
   }
 }
@@ -148,53 +220,56 @@ __global__ void __launch_bounds__(256) rotate_cols_inner_kernel(float* __restric
 // b2 = blockIdx.y, strip blockIdx.x.  Applies H_p1 over b1 and Q_m over a
 // (Q_m^T first when inverse; the two commute, they act on different factors).
 __global__ void __launch_bounds__(256) rotate_cols_outer_kernel(float* __restrict__ M, int64_t ld, int64_t cols,
-                                                                int p, int p1, int p2, int m,
+                                                                int p, int log2_p1, int p2, int m,
                                                                 const float* __restrict__ Qm, int inverse) {
   extern __shared__ float sm[];
   float* Qs = sm;                   // [m*m]
-  float* t = sm + kMaxM * kMaxM;    // [m*p1][kStrip]
+  float* t = sm + ((m * m + 3) & ~3);  // [m*p1][128]
+  const int p1 = 1 << log2_p1;
   const int R = m * p1;
   const int b2 = blockIdx.y;
   const int64_t c0 = (int64_t)blockIdx.x * kStrip;
-  const int c = threadIdx.x % kStrip;
-  const int rs = threadIdx.x / kStrip;
-  const int rstep = blockDim.x / kStrip;
-  const bool cok = c0 + c < cols;
+  const int c4 = 4 * (threadIdx.x % (kStrip / 4));
+  const int rs = threadIdx.x / (kStrip / 4);
+  const int rstep = blockDim.x / (kStrip / 4);
+  const bool full = c0 + c4 + 3 < cols;
   if (m > 1)
     for (int i = threadIdx.x; i < m * m; i += blockDim.x) Qs[i] = Qm[i];
   for (int r = rs; r < R; r += rstep) {
-    int a = r / p1, b1 = r % p1;
-    int64_t row = (int64_t)a * p + (int64_t)b1 * p2 + b2;
-    t[r * kStrip + c] = cok ? M[row * ld + c0 + c] : 0.f;
+    const int a = r >> log2_p1, b1 = r & (p1 - 1);
+    const float* src = M + ((int64_t)a * p + (int64_t)b1 * p2 + b2) * ld + c0 + c4;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (full) {
+      v = *reinterpret_cast<const float4*>(src);
+    } else {
+      if (c0 + c4 + 0 < cols) v.x = src[0];
+      if (c0 + c4 + 1 < cols) v.y = src[1];
+      if (c0 + c4 + 2 < cols) v.z = src[2];
+    }
+    *reinterpret_cast<float4*>(t + r * kStrip + c4) = v;
   }
   __syncthreads();
-  // H_p1 over b1 within each a-block (rows a*p1 .. a*p1 + p1 - 1 of the tile)
-  for (int h = 1; h < p1; h <<= 1) {
-    for (int idx = rs; idx < R / 2; idx += rstep) {
-      int i = (idx / h) * (2 * h) + (idx % h);
-      float a0 = t[i * kStrip + c], b0 = t[(i + h) * kStrip + c];
-      t[i * kStrip + c] = a0 + b0;
-      t[(i + h) * kStrip + c] = a0 - b0;
+  auto qmix = [&](bool transpose) {
+    for (int idx = threadIdx.x; idx < p1 * kStrip; idx += blockDim.x) {
+      const int b1 = idx / kStrip, c = idx % kStrip;
+      qmix_strand(Qs, m, transpose, [&](int q) { return t[(q * p1 + b1) * kStrip + c]; },
+                  [&](int a, float v) { t[(a * p1 + b1) * kStrip + c] = v; });
     }
     __syncthreads();
-  }
-  if (m > 1) {
-    float tmp[kMaxM];
-    for (int b1 = rs; b1 < p1; b1 += rstep) {
-      for (int a = 0; a < m; ++a) tmp[a] = t[(a * p1 + b1) * kStrip + c];
-      for (int a = 0; a < m; ++a) {
-        float acc = 0.f;
-        for (int q = 0; q < m; ++q) acc = fmaf(inverse ? Qs[q * m + a] : Qs[a * m + q], tmp[q], acc);
-        t[(a * p1 + b1) * kStrip + c] = acc;
-      }
-    }
-    __syncthreads();
-  }
-  if (cok) {
-    for (int r = rs; r < R; r += rstep) {
-      int a = r / p1, b1 = r % p1;
-      int64_t row = (int64_t)a * p + (int64_t)b1 * p2 + b2;
-      M[row * ld + c0 + c] = t[r * kStrip + c];
+  };
+  if (m > 1 && inverse) qmix(true);
+  fwht_passes<false>(t, log2_p1, kStrip * m);
+  if (m > 1 && !inverse) qmix(false);
+  for (int r = rs; r < R; r += rstep) {
+    const int a = r >> log2_p1, b1 = r & (p1 - 1);
+    const float4 v = *reinterpret_cast<const float4*>(t + r * kStrip + c4);
+    float* dst = M + ((int64_t)a * p + (int64_t)b1 * p2 + b2) * ld + c0 + c4;
+    if (full) {
+      *reinterpret_cast<float4*>(dst) = v;
+    } else {
+      if (c0 + c4 + 0 < cols) dst[0] = v.x;
+      if (c0 + c4 + 1 < cols) dst[1] = v.y;
+      if (c0 + c4 + 2 < cols) dst[2] = v.z;
     }
   }
 }
@@ -222,38 +297,38 @@ extern "C" kq_status kq_rotate(float* M, int64_t rows, int64_t cols, int64_t ld,
   if (axis == KQ_AXIS_COLS) {
     if (n > kMaxRowN) return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_rotate: row length above 32768");
     if (rows > 0x7fffffff) return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_rotate: too many rows");
-    size_t smem = (size_t)(n + (m > 1 ? m * m : 0)) * sizeof(float);
+    size_t smem = (size_t)(n + n / 16 + 4 + (m > 1 ? m * m : 0)) * sizeof(float);
     KQ_TRY(kq::cuda_check(cudaFuncSetAttribute(rotate_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                (int)smem), "kq_rotate: smem attribute"));
-    rotate_rows_kernel<<<(unsigned)rows, 512, smem, st>>>(M, ld, (int)n, lp, m, T->signs, T->Qm, inverse, scale);
+    rotate_rows_kernel<<<(unsigned)rows, 256, smem, st>>>(M, ld, (int)n, lp, m, T->signs, T->Qm, inverse, scale);
     KQ_TRY(kq::launch_check("kq_rotate rows"));
   } else {
     const int lp2 = lp < kMaxP2Log ? lp : kMaxP2Log;
     const int p2 = 1 << lp2, p1 = 1 << (lp - lp2);
     if ((int64_t)m * p1 > kMaxOuterRows)
-      return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_rotate: m * p / 512 above 1024");
+      return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_rotate: m * p / 128 above 256");
     const unsigned strips = (unsigned)kq::cdiv(cols, kStrip);
     const bool outer = (m > 1 || p1 > 1);
     size_t smem_in = (size_t)p2 * kStrip * sizeof(float);
-    size_t smem_out = (size_t)(kMaxM * kMaxM + m * p1 * kStrip) * sizeof(float);
+    size_t smem_out = (size_t)(((m * m + 3) & ~3) + m * p1 * kStrip) * sizeof(float);
     KQ_TRY(kq::cuda_check(cudaFuncSetAttribute(rotate_cols_inner_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                (int)smem_in), "kq_rotate: smem attribute"));
     KQ_TRY(kq::cuda_check(cudaFuncSetAttribute(rotate_cols_outer_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                (int)smem_out), "kq_rotate: smem attribute"));
     dim3 gin(strips, (unsigned)(n / p2)), gout(strips, (unsigned)p2);
     if (!inverse) {
-      rotate_cols_inner_kernel<<<gin, 256, smem_in, st>>>(M, ld, cols, p2, T->signs, 0, scale);
+      rotate_cols_inner_kernel<<<gin, 256, smem_in, st>>>(M, ld, cols, lp2, T->signs, 0, scale);
       KQ_TRY(kq::launch_check("kq_rotate cols inner"));
       if (outer) {
-        rotate_cols_outer_kernel<<<gout, 256, smem_out, st>>>(M, ld, cols, p, p1, p2, m, T->Qm, 0);
+        rotate_cols_outer_kernel<<<gout, 256, smem_out, st>>>(M, ld, cols, p, lp - lp2, p2, m, T->Qm, 0);
         KQ_TRY(kq::launch_check("kq_rotate cols outer"));
       }
     } else {
       if (outer) {
-        rotate_cols_outer_kernel<<<gout, 256, smem_out, st>>>(M, ld, cols, p, p1, p2, m, T->Qm, 1);
+        rotate_cols_outer_kernel<<<gout, 256, smem_out, st>>>(M, ld, cols, p, lp - lp2, p2, m, T->Qm, 1);
         KQ_TRY(kq::launch_check("kq_rotate cols outer"));
       }
-      rotate_cols_inner_kernel<<<gin, 256, smem_in, st>>>(M, ld, cols, p2, T->signs, 1, scale);
+      rotate_cols_inner_kernel<<<gin, 256, smem_in, st>>>(M, ld, cols, lp2, T->signs, 1, scale);
       KQ_TRY(kq::launch_check("kq_rotate cols inner"));
     }
   }
