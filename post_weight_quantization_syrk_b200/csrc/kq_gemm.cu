@@ -14,7 +14,7 @@
 // K-major, 64-byte swizzle; tcgen05 kind::tf32 produced no result with an
 // MN-major operand on B200 when measured, so callers pass B transposed), big
 // and small parts, through a 3-stage ring; one thread of warp 1 issues 12
-// tcgen05.mma kind::tf32 per stage; warps 2-5 run the epilogue from TMEM.
+// tcgen05.mma kind::tf32 per stage; warps 2-9 run the epilogue from TMEM.
 // Waits are time-bounded.
 #include <cuda.h>
 
@@ -33,7 +33,7 @@ constexpr int A_BYTES = BM * BKF * 4;               // 16 KB per part
 constexpr int B_BYTES = BN * BKF * 4;               // 16 KB per part
 constexpr int STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;
 constexpr int STAGES = 3;
-constexpr int THREADS = 192;
+constexpr int THREADS = 320;                        // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 
 struct Params {
@@ -80,7 +80,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       mbar_init(empty0 + 8 * s, 1);
     }
     mbar_init(accfull, 1);
-    mbar_init(accempty, 128);
+    mbar_init(accempty, 256);
     mbar_init(drained, 1);
     *abort_flag = 0;
     mbar_init_fence();
@@ -176,7 +176,13 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       }
     }
   } else {
+    // Epilogue: 8 warps; warp w reads TMEM lanes 32 (w % 4) .. (the rows it
+    // may access) for one 128-column half of each accumulator.  Source
+    // operands (src / other) for 64 columns are fetched before they are
+    // needed, so each thread keeps 16 float4 loads in flight.
+    const int e = warp - 2;
     const int wq = warp & 3;
+    const int cbase = (e >> 2) * 128;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
       const int64_t m0 = (int64_t)(t / p.tiles_n) * BM, n0 = (int64_t)(t % p.tiles_n) * BN;
@@ -192,50 +198,56 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
         const int64_t gi = m0 + h * 128 + 32 * wq + lane;
         const bool row_ok = gi < p.M;
 #pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 16) {
-          float v[16];
-          tmem_ld16(tmem + ((uint32_t)(32 * wq) << 16) + (uint32_t)(256 * h + c0), v);
-          const int64_t gj0 = n0 + c0;
-          if (!row_ok || gj0 >= p.N) continue;
-          const bool full16 = gj0 + 16 <= p.N;
-          if (p.epilogue == kEpiDot) {
-            const float* o = p.other + gi * p.ld_other + gj0;
-            if (full16) {
+        for (int g0 = 0; g0 < 128; g0 += 64) {
+          const int64_t gj0 = n0 + cbase + g0;
+          const bool any = row_ok && gj0 < p.N;
+          const bool fast = any && gj0 + 64 <= p.N && !(p.epilogue == kEpiSubtract && p.dead);
+          float pre[64];
+          if (fast && p.epilogue != kEpiStore) {
+            const float* sp = (p.epilogue == kEpiDot ? p.other + gi * p.ld_other : p.src + gi * p.ld_src) + gj0;
 #pragma unroll
-              for (int q = 0; q < 16; q += 4) {
-                const float4 w = *reinterpret_cast<const float4*>(o + q);
-                dot += (double)v[q] * w.x + (double)v[q + 1] * w.y + (double)v[q + 2] * w.z + (double)v[q + 3] * w.w;
-              }
-            } else {
-              for (int q = 0; gj0 + q < p.N && q < 16; ++q) dot += (double)v[q] * o[q];
+            for (int q = 0; q < 64; q += 4) {
+              const float4 w = *reinterpret_cast<const float4*>(sp + q);
+              pre[q] = w.x;
+              pre[q + 1] = w.y;
+              pre[q + 2] = w.z;
+              pre[q + 3] = w.w;
             }
-          } else {
-            float* c = p.C + gi * p.ldc + gj0;
-            if (p.epilogue == kEpiSubtract) {
-              const float* s = p.src + gi * p.ld_src + gj0;
-              if (full16 && !p.dead) {
+          }
+#pragma unroll
+          for (int cc = 0; cc < 64; cc += 16) {
+            float v[16];
+            tmem_ld16(tmem + ((uint32_t)(32 * wq) << 16) + (uint32_t)(256 * h + cbase + g0 + cc), v);
+            if (!any) continue;
+            const int64_t gj = gj0 + cc;
+            if (fast) {
+              if (p.epilogue == kEpiDot) {
+#pragma unroll
+                for (int q = 0; q < 16; ++q) dot += (double)v[q] * (double)pre[cc + q];
+              } else {
+                float* c = p.C + gi * p.ldc + gj;
 #pragma unroll
                 for (int q = 0; q < 16; q += 4) {
-                  float4 w = *reinterpret_cast<const float4*>(s + q);
-                  w.x -= v[q];
-                  w.y -= v[q + 1];
-                  w.z -= v[q + 2];
-                  w.w -= v[q + 3];
-                  *reinterpret_cast<float4*>(c + q) = w;
-                }
-              } else {
-                for (int q = 0; gj0 + q < p.N && q < 16; ++q) {
-                  const float sv = (p.dead && p.dead[gj0 + q]) ? 0.f : s[q];
-                  c[q] = sv - v[q];
+                  float4 o;
+                  if (p.epilogue == kEpiSubtract)
+                    o = make_float4(pre[cc + q] - v[q], pre[cc + q + 1] - v[q + 1], pre[cc + q + 2] - v[q + 2],
+                                    pre[cc + q + 3] - v[q + 3]);
+                  else
+                    o = make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
+                  *reinterpret_cast<float4*>(c + q) = o;
                 }
               }
             } else {
-              if (full16) {
-#pragma unroll
-                for (int q = 0; q < 16; q += 4)
-                  *reinterpret_cast<float4*>(c + q) = make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
-              } else {
-                for (int q = 0; gj0 + q < p.N && q < 16; ++q) c[q] = v[q];
+              for (int q = 0; q < 16 && gj + q < p.N; ++q) {
+                const int64_t j = gj + q;
+                if (p.epilogue == kEpiDot) {
+                  dot += (double)v[q] * (double)p.other[gi * p.ld_other + j];
+                } else if (p.epilogue == kEpiSubtract) {
+                  const float sv = (p.dead && p.dead[j]) ? 0.f : p.src[gi * p.ld_src + j];
+                  p.C[gi * p.ldc + j] = sv - v[q];
+                } else {
+                  p.C[gi * p.ldc + j] = v[q];
+                }
               }
             }
           }
@@ -245,9 +257,9 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       mbar_arrive(accempty);
       if (p.epilogue == kEpiDot) {
         // fixed-order reduction within the warp (xor butterfly); one partial
-        // per (tile, warp), summed later in index order: no CTA barrier here
+        // per (tile, epilogue warp), summed later in index order
         for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-        if (lane == 0) p.partial[4 * (int64_t)t + wq] = dot;
+        if (lane == 0) p.partial[8 * (int64_t)t + e] = dot;
       }
       acc_phase ^= 1u;
     }

@@ -33,11 +33,11 @@ struct Gemm3xTF32 {
   const uint8_t* dead = nullptr;   // subtract: src column n reads as 0 when dead[n]
   const float* other = nullptr;    // (m, n) at other[m * ld_other + n] (dot)
   int64_t ld_other = 0;
-  double* partial = nullptr;       // dot: 4 fp64 per output tile (one per epilogue warp)
+  double* partial = nullptr;       // dot: 8 fp64 per output tile (one per epilogue warp)
   int32_t* info = nullptr;
 };
 
-// Output tiles of an M x N product (`partial` holds 4 per tile for kEpiDot).
+// Output tiles of an M x N product (`partial` holds 8 per tile for kEpiDot).
 int64_t gemm_tiles(int64_t M, int64_t N);
 
 kq_status gemm_3xtf32(const Gemm3xTF32& g, cudaStream_t st);

@@ -97,8 +97,9 @@ struct InblockArgs {
   uint8_t* codes;
   int64_t ldq;
   float* ET;   // [128, d_out]: the block's errors, transposed (fp32 SIMT trailing update)
-  float* Eb;   // [d_out, 128]: tf32 part of the errors (3xTF32 trailing update), or NULL
-  float* Es;   // [d_out, 128]: remainder
+  float* Eb;   // tf32 part of the errors (3xTF32 trailing update), or NULL:
+  float* Es;   // row r, column c of the block at [r * ldE + e_col0 + c]; remainder
+  int64_t ldE, e_col0;
   int32_t* info;
 };
 
@@ -267,8 +268,8 @@ __global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
         b[e] = __uint_as_float(bits);
         sm4[e] = ee - b[e];
       }
-      *reinterpret_cast<float4*>(a.Eb + row * BLK + c) = make_float4(b[0], b[1], b[2], b[3]);
-      *reinterpret_cast<float4*>(a.Es + row * BLK + c) = make_float4(sm4[0], sm4[1], sm4[2], sm4[3]);
+      *reinterpret_cast<float4*>(a.Eb + row * a.ldE + a.e_col0 + c) = make_float4(b[0], b[1], b[2], b[3]);
+      *reinterpret_cast<float4*>(a.Es + row * a.ldE + a.e_col0 + c) = make_float4(sm4[0], sm4[1], sm4[2], sm4[3]);
     } else {
       for (int e = 0; e < 4; ++e)
         if (c + e < bw) a.ET[(int64_t)(c + e) * a.d_out + row] = ev[4 * m + e];
@@ -352,9 +353,14 @@ __global__ void __launch_bounds__(256) trailing_fp32_kernel(const float* __restr
 
 namespace {
 
-// Workspace: the block's errors (E^T for the fp32 path, or E split in two
-// for 3xTF32), then Uc^T split in two (3xTF32 only: the tensor-core product
-// reads its B operand transposed).
+// Outer block of the two-level lazy update (3xTF32 path): after each
+// 128-column block only the rest of its outer block is updated; after each
+// outer block one GEMM with K = OUTER updates all columns to its right.
+constexpr int OUTER = 1024;
+
+// Workspace: the errors (E^T of one block for the fp32 path, or E of one
+// outer block split in two for 3xTF32), then Uc^T split in two (3xTF32 only:
+// the tensor-core product reads its B operand transposed).
 struct QuantWs {
   float *ET, *Eb, *Es, *Ub, *Us;
   int64_t ldu;
@@ -362,7 +368,7 @@ struct QuantWs {
 
 size_t quant_layout(int64_t d_out, int64_t d_in, QuantWs* w, void* base) {
   const int64_t ldu = (d_in + 3) / 4 * 4;
-  const size_t se = kq::align_up((size_t)d_out * BLK * sizeof(float), 256);
+  const size_t se = kq::align_up((size_t)d_out * OUTER * sizeof(float), 256);
   const size_t su = kq::align_up((size_t)d_in * ldu * sizeof(float), 256);
   if (w && base) {
     char* b = static_cast<char*>(base);
@@ -422,7 +428,7 @@ extern "C" kq_status kq_quantize_layer(const float* W, int64_t d_out, int64_t d_
   }
   KQ_TRY(kq::cuda_check(cudaFuncSetAttribute(inblock_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, IB_SMEM),
                         "kq_quantize_layer: smem attribute"));
-  for (int64_t i0 = 0; i0 < d_in; i0 += BLK) {
+  auto inblock = [&](int64_t i0, int64_t o0) -> kq_status {
     const int bw = (int)std::min<int64_t>(BLK, d_in - i0);
     const bool first = (i0 == 0);
     InblockArgs a;
@@ -447,36 +453,59 @@ extern "C" kq_status kq_quantize_layer(const float* W, int64_t d_out, int64_t d_
     a.ET = w.ET;
     a.Eb = tc ? w.Eb : nullptr;
     a.Es = tc ? w.Es : nullptr;
+    a.ldE = OUTER;
+    a.e_col0 = i0 - o0;
     a.info = info;
     inblock_kernel<<<(unsigned)kq::cdiv(d_out, IB_ROWS), IB_THREADS, IB_SMEM, st>>>(a);
-    KQ_TRY(kq::launch_check("kq_quantize_layer inblock"));
-    const int64_t cstart = i0 + bw;
-    if (cstart < d_in && !tc) {
-      dim3 grid((unsigned)kq::cdiv(d_in - cstart, TN), (unsigned)kq::cdiv(d_out, TM));
-      trailing_fp32_kernel<<<grid, 256, 0, st>>>(first ? W : W_hat, first ? ldw : ldwh, W_hat, ldwh, w.ET, Uc, lduc,
-                                                first ? dead_mask : nullptr, d_out, d_in, i0, bw, cstart);
-      KQ_TRY(kq::launch_check("kq_quantize_layer trailing"));
-    } else if (cstart < d_in) {
-      kq::Gemm3xTF32 g;   // W_hat[:, cstart:] = src[:, cstart:] - E Uc[i0:i0+bw, cstart:]
-      g.M = d_out;
-      g.N = d_in - cstart;
-      g.K = bw;
-      g.a_big = w.Eb;
-      g.a_small = w.Es;
-      g.lda = BLK;
-      g.bt_big = w.Ub;         // Uc^T: (k, n) of Uc[i0:, cstart:] at Ut[cstart + n][i0 + k]
-      g.bt_small = w.Us;
-      g.ldbt = w.ldu;
-      g.bt_row0 = cstart;
-      g.bt_col0 = i0;
-      g.epilogue = kq::kEpiSubtract;
-      g.C = W_hat + cstart;
-      g.ldc = ldwh;
-      g.src = (first ? W : W_hat) + cstart;
-      g.ld_src = first ? ldw : ldwh;
-      g.dead = first && dead_mask ? dead_mask + cstart : nullptr;
-      g.info = info;
-      KQ_TRY(kq::gemm_3xtf32(g, st));
+    return kq::launch_check("kq_quantize_layer inblock");
+  };
+  // W_hat[:, c0:c0+N] = src[:, c0:c0+N] - E[:, e0:e0+K] Uc[k0:k0+K, c0:c0+N]; the
+  // source is W (dead columns as zeros) while those columns are still untouched.
+  auto update = [&](int64_t c0, int64_t N, int64_t e0, int64_t k0, int64_t K, bool from_w) -> kq_status {
+    kq::Gemm3xTF32 g;
+    g.M = d_out;
+    g.N = N;
+    g.K = K;
+    g.a_big = w.Eb;
+    g.a_small = w.Es;
+    g.lda = OUTER;
+    g.a_col0 = e0;
+    g.bt_big = w.Ub;         // Uc^T: (k, n) of Uc[k0:, c0:] at Ut[c0 + n][k0 + k]
+    g.bt_small = w.Us;
+    g.ldbt = w.ldu;
+    g.bt_row0 = c0;
+    g.bt_col0 = k0;
+    g.epilogue = kq::kEpiSubtract;
+    g.C = W_hat + c0;
+    g.ldc = ldwh;
+    g.src = (from_w ? W : W_hat) + c0;
+    g.ld_src = from_w ? ldw : ldwh;
+    g.dead = from_w && dead_mask ? dead_mask + c0 : nullptr;
+    g.info = info;
+    return kq::gemm_3xtf32(g, st);
+  };
+  if (!tc) {
+    for (int64_t i0 = 0; i0 < d_in; i0 += BLK) {
+      const int bw = (int)std::min<int64_t>(BLK, d_in - i0);
+      const bool first = (i0 == 0);
+      KQ_TRY(inblock(i0, i0));
+      const int64_t cstart = i0 + bw;
+      if (cstart < d_in) {
+        dim3 grid((unsigned)kq::cdiv(d_in - cstart, TN), (unsigned)kq::cdiv(d_out, TM));
+        trailing_fp32_kernel<<<grid, 256, 0, st>>>(first ? W : W_hat, first ? ldw : ldwh, W_hat, ldwh, w.ET, Uc,
+                                                  lduc, first ? dead_mask : nullptr, d_out, d_in, i0, bw, cstart);
+        KQ_TRY(kq::launch_check("kq_quantize_layer trailing"));
+      }
+    }
+  } else {
+    for (int64_t o0 = 0; o0 < d_in; o0 += OUTER) {
+      const int64_t o1 = std::min<int64_t>(o0 + OUTER, d_in);
+      for (int64_t i0 = o0; i0 < o1; i0 += BLK) {
+        const int64_t bw = std::min<int64_t>(BLK, d_in - i0);
+        KQ_TRY(inblock(i0, o0));
+        if (i0 + bw < o1) KQ_TRY(update(i0 + bw, o1 - (i0 + bw), i0 - o0, i0, bw, i0 == 0));
+      }
+      if (o1 < d_in) KQ_TRY(update(o1, d_in - o1, 0, o0, o1 - o0, o0 == 0));
     }
   }
   kq::clear_error();
