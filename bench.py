@@ -48,6 +48,8 @@ def parse():
                     help="precision mode of the solver's trailing update")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-model", action="store_true", help="skip the whole 7B-shaped model run")
+    ap.add_argument("--model-blocks", type=int, default=32)
     a = ap.parse_args()
     a.warmup = max(a.warmup, 3)
     return a
@@ -217,6 +219,19 @@ def run_kronq(a):
     if not a.no_e2e:
         e2e = run_e2e(a, lq, results, W, X, G, T_in, T_out, spec, settings, world, dev)
 
+    # ---- the whole 7B-shaped model (32 blocks x 7 linears), one GPU
+    model = None
+    if world == 1 and not a.no_model:
+        from post_weight_quantization_syrk_b200.model import synthetic_model
+        del X, G
+        torch.cuda.empty_cache()
+        r = synthetic_model(n_tokens=spec.n_tokens, n_blocks=a.model_blocks, device=dev, gemm_mode=gemm_mode).run()
+        model = {k: r[k] for k in ("blocks", "linears", "weights", "gpu_seconds", "weights_per_s", "phase_seconds",
+                                   "input_generation_seconds", "average_bits", "bits_histogram")}
+        model["tokens"] = spec.n_tokens
+        model["note"] = ("end-to-end GPU time of the whole path for all linears (statistics, sensitivity, bit "
+                         "allocation, BiIP, Cholesky, solver, loss); synthetic inputs generated per block, untimed")
+
     pk, src = peaks()
     flops = spec.n_tokens * spec.d_in * (spec.d_in + 1)    # one SYRK launch on X (d_out == d_in here)
     syrk_avg = statistics.mean(syrk_ms)
@@ -239,6 +254,7 @@ def run_kronq(a):
         "gpu_launches": launches,
         "clocks": clk,
         "e2e": e2e,
+        "model_7b": model,
     }
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         out["cpu_baseline"] = oracle_sample(spec, settings)

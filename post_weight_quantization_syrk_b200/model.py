@@ -1,0 +1,189 @@
+"""A whole Llama-2-7B-shaped model through the KronQ path (32 decoder blocks x
+7 linears), driven through the C ABI.
+
+Order (KronQ paper page, Abstract; KronQ review, Method and Comparison):
+  pass 1, per block: covariances of the four distinct linear inputs
+    (attention input shared by q/k/v, o-projection input, MLP input shared by
+    gate/up, down-projection input) and of the seven output gradients, kept
+    resident; the trace sensitivity tr(H_G) tr(H_X) of each linear;
+  allocation of {2,3,4} bits to an average of 3.0 over all 224 linears from
+    the scores (kq_allocate_bits);
+  pass 2, per block: BiIP of each input covariance once (q/k/v and gate/up
+    share U and H_X, hence one damped Cholesky factor), then per linear the
+    rotation of W and H_G, the blocked OBS solve at its allocated bit-width
+    and its Kronecker loss.
+GPU time is taken with CUDA events around each phase; generating the
+synthetic inputs is reported separately and is not part of the quantization
+time.
+"""
+from __future__ import annotations
+
+import dataclasses
+import time
+
+import torch
+
+from . import _lib as K
+
+D_MODEL = 4096
+D_FF = 11008
+N_BLOCKS = 32
+LINEARS = ("q", "k", "v", "o", "gate", "up", "down")
+# input group of each linear, its (d_out, d_in)
+INPUT_OF = {"q": "attn", "k": "attn", "v": "attn", "o": "oin", "gate": "mlp", "up": "mlp", "down": "dn"}
+SHAPE = {"q": (D_MODEL, D_MODEL), "k": (D_MODEL, D_MODEL), "v": (D_MODEL, D_MODEL), "o": (D_MODEL, D_MODEL),
+         "gate": (D_FF, D_MODEL), "up": (D_FF, D_MODEL), "down": (D_MODEL, D_FF)}
+INPUT_WIDTH = {"attn": D_MODEL, "oin": D_MODEL, "mlp": D_MODEL, "dn": D_FF}
+
+
+def synthetic_model(n_tokens, n_blocks=N_BLOCKS, device="cuda", **kw):
+    """A ModelQuantizer over the seeded synthetic 7B-shaped model."""
+    import synth
+
+    def make_inputs(b, stats_only):
+        return synth.model_block(b, n_tokens, stats_only, device)
+
+    def make_rht(b, name, n):
+        p = synth.model_rht(b, name, n)
+        return K.RHT(p.n, p.log2_p, p.m, p.signs.to(device), None if p.Qm is None else p.Qm.to(device))
+
+    return ModelQuantizer(make_inputs, make_rht, n_tokens, n_blocks, device, **kw)
+
+
+@dataclasses.dataclass
+class Phase:
+    ms: float = 0.0
+
+    def add(self, e0, e1):
+        self.ms += e0.elapsed_time(e1)
+
+
+class ModelQuantizer:
+    """Drives the 7B-shaped model; `make_inputs(block)` supplies the synthetic
+    tensors of one block (X per input group, G and W per linear)."""
+
+    def __init__(self, make_inputs, make_rht, n_tokens, n_blocks=N_BLOCKS, device="cuda",
+                 choices=(2, 3, 4), avg_bits=3.0, gemm_mode=K.KQ_GEMM_3XTF32, damp=0.01):
+        self.make_inputs, self.make_rht = make_inputs, make_rht
+        self.n_tokens, self.n_blocks, self.dev = n_tokens, n_blocks, torch.device(device)
+        self.choices, self.avg_bits, self.gemm_mode, self.damp = choices, avg_bits, gemm_mode, damp
+        self.info = K.new_info(self.dev)
+        self.ws = K.workspace(256, self.dev)
+        self.phases = {k: Phase() for k in ("statistics", "sensitivity", "rotate", "chol_inv", "quantize", "loss")}
+        self.gen_s = 0.0
+
+    def _ws(self, nbytes):
+        if nbytes > self.ws.numel():
+            self.ws = K.workspace(nbytes, self.dev)
+        return self.ws
+
+    def _timed(self, name, fn):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        self._events.append((name, e0, e1))
+
+    def run(self):
+        self._events = []
+        dev = self.dev
+        HX, HG, sens = {}, {}, {}
+        sens_dev = {}
+        # ---------------- pass 1: statistics and sensitivities
+        for b in range(self.n_blocks):
+            t0 = time.perf_counter()
+            inp = self.make_inputs(b, stats_only=True)
+            torch.cuda.synchronize()
+            self.gen_s += time.perf_counter() - t0
+            for g, X in inp["X"].items():
+                d = X.shape[1]
+                H = torch.empty((d, d), dtype=torch.float32, device=dev)
+                ws = self._ws(K.kq_accum_cov_workspace_size(X.shape[0], d))
+                self._timed("statistics", lambda: K.kq_accum_cov(X, H, 1.0 / X.shape[0], False, ws, self.info))
+                HX[(b, g)] = H
+            for lin, G in inp["G"].items():
+                d = G.shape[1]
+                H = torch.empty((d, d), dtype=torch.float32, device=dev)
+                ws = self._ws(K.kq_accum_cov_workspace_size(G.shape[0], d))
+                self._timed("statistics", lambda: K.kq_accum_cov(G, H, 1.0 / G.shape[0], False, ws, self.info))
+                HG[(b, lin)] = H
+            for lin in LINEARS:
+                out = torch.zeros(3, dtype=torch.float64, device=dev)
+                self._timed("sensitivity",
+                            lambda: K.kq_sensitivity(HX[(b, INPUT_OF[lin])], HG[(b, lin)], out))
+                sens_dev[(b, lin)] = out
+            del inp
+        torch.cuda.synchronize()
+        K.check_info(self.info, "model statistics")
+        keys = [(b, lin) for b in range(self.n_blocks) for lin in LINEARS]
+        for k in keys:
+            sens[k] = sens_dev[k].cpu().tolist()
+        n_params = [SHAPE[lin][0] * SHAPE[lin][1] for _, lin in keys]
+        bits = K.kq_allocate_bits([sens[k][2] for k in keys], n_params, self.choices, self.avg_bits)
+        alloc = dict(zip(keys, bits))
+
+        # ---------------- pass 2: BiIP, Cholesky, solver, loss
+        results = {}
+        for b in range(self.n_blocks):
+            t0 = time.perf_counter()
+            inp = self.make_inputs(b, stats_only=False)
+            torch.cuda.synchronize()
+            self.gen_s += time.perf_counter() - t0
+            U = {g: self.make_rht(b, "in:" + g, INPUT_WIDTH[g]) for g in INPUT_WIDTH}
+            Uc, dead = {}, {}
+            for g in INPUT_WIDTH:
+                H = HX.pop((b, g))
+                self._timed("rotate", lambda: (K.kq_rotate(H, K.KQ_AXIS_COLS, U[g]),
+                                               K.kq_rotate(H, K.KQ_AXIS_ROWS, U[g])))
+                n = H.shape[0]
+                Uc[g] = torch.empty_like(H)
+                dead[g] = torch.zeros(n, dtype=torch.uint8, device=dev)
+                ws = self._ws(K.kq_chol_inv_workspace_size(n))
+                self._timed("chol_inv", lambda: K.kq_chol_inv(H, self.damp, Uc[g], dead[g], ws, self.info))
+                HX[(b, g)] = H
+            for lin in LINEARS:
+                g = INPUT_OF[lin]
+                d_out, d_in = SHAPE[lin]
+                V = self.make_rht(b, "out:" + lin, d_out)
+                W = inp["W"][lin]
+                Hg = HG.pop((b, lin))
+                self._timed("rotate", lambda: (K.kq_rotate(W, K.KQ_AXIS_COLS, U[g]), K.kq_rotate(W, K.KQ_AXIS_ROWS, V),
+                                               K.kq_rotate(Hg, K.KQ_AXIS_COLS, V),
+                                               K.kq_rotate(Hg, K.KQ_AXIS_ROWS, V)))
+                nb = alloc[(b, lin)]
+                codes = torch.empty((d_out, d_in), dtype=torch.uint8, device=dev)
+                scales = torch.empty((d_out, 1), dtype=torch.float32, device=dev)
+                zeros = torch.empty((d_out, 1), dtype=torch.float32, device=dev)
+                W_hat = torch.empty((d_out, d_in), dtype=torch.float32, device=dev)
+                loss = torch.zeros(1, dtype=torch.float64, device=dev)
+                ws = self._ws(K.kq_quantize_layer_workspace_size(d_out, d_in))
+                self._timed("quantize", lambda: K.kq_quantize_layer(W, Uc[g], dead[g], nb, 0, codes, scales, zeros,
+                                                                     W_hat, gemm_mode=self.gemm_mode, ws=ws,
+                                                                     info=self.info))
+                ws = self._ws(K.kq_kron_loss_workspace_size(d_out, d_in))
+                self._timed("loss", lambda: K.kq_kron_loss(W, W_hat, HX[(b, g)], Hg, loss, ws))
+                results[(b, lin)] = {"bits": nb, "loss": loss, "codes_bytes": codes.numel()}
+                del Hg, codes, W_hat
+            for g in INPUT_WIDTH:
+                del HX[(b, g)]
+            del inp, Uc, dead
+        torch.cuda.synchronize()
+        K.check_info(self.info, "model quantization")
+        for name, e0, e1 in self._events:
+            self.phases[name].add(e0, e1)
+        total_ms = sum(p.ms for p in self.phases.values())
+        n_weights = sum(SHAPE[lin][0] * SHAPE[lin][1] for _, lin in keys)
+        avg = sum(alloc[k] * SHAPE[k[1]][0] * SHAPE[k[1]][1] for k in keys) / n_weights
+        return {
+            "blocks": self.n_blocks, "linears": len(keys), "weights": n_weights,
+            "gpu_seconds": total_ms / 1e3,
+            "weights_per_s": n_weights / (total_ms / 1e3),
+            "phase_seconds": {k: v.ms / 1e3 for k, v in self.phases.items()},
+            "input_generation_seconds": self.gen_s,
+            "average_bits": avg,
+            "bits_histogram": {str(c): sum(1 for k in keys if alloc[k] == c) for c in self.choices},
+            "loss_sum": float(sum(r["loss"].item() for r in results.values())),
+            "per_linear": [{"block": b, "linear": lin, "score": sens[(b, lin)][2], "tr_X": sens[(b, lin)][0],
+                            "tr_G": sens[(b, lin)][1], "bits": alloc[(b, lin)],
+                            "loss": results[(b, lin)]["loss"].item()} for b, lin in keys],
+        }

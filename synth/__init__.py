@@ -200,3 +200,48 @@ def layer(spec: LayerSpec, seed: int, device="cpu"):
     T_in = rht_params(spec.d_in, seed * 2 + 11)
     T_out = rht_params(spec.d_out, seed * 2 + 12)
     return W, X, G, T_in, T_out
+
+
+# ---------------------------------------------------------------------------
+# Whole 7B-shaped model (32 blocks x 7 linears): per-block synthetic inputs.
+# 4096-wide inputs follow the attention-projection recipe (log-normal(0, 1.5)
+# channel scales, 8 massive channels), the 11008-wide down-projection input is
+# the SiLU-gated product; gradients get LogUniform[1e-4, 1] output scales.
+# ---------------------------------------------------------------------------
+MODEL_LINEARS = ("q", "k", "v", "o", "gate", "up", "down")
+MODEL_INPUT_OF = {"q": "attn", "k": "attn", "v": "attn", "o": "oin", "gate": "mlp", "up": "mlp", "down": "dn"}
+MODEL_SHAPE = {"q": (4096, 4096), "k": (4096, 4096), "v": (4096, 4096), "o": (4096, 4096),
+               "gate": (11008, 4096), "up": (11008, 4096), "down": (4096, 11008)}
+
+
+def model_block(block: int, n_tokens: int, stats_only: bool, device="cuda"):
+    """{"X": {group: X}, "G": {linear: G}} (stats_only) or {"W": {linear: W}}."""
+    base = WORKLOADS["attn4096"]
+    out = {}
+    if stats_only:
+        X = {}
+        for gi, g in enumerate(("attn", "oin", "mlp", "dn")):
+            seed = layer_seed(5, 100 * block + gi)
+            spec = (scaled(WORKLOADS["mlp_down11008"], d_in=11008, n_tokens=n_tokens) if g == "dn"
+                    else scaled(base, d_in=4096, n_tokens=n_tokens))
+            X[g] = activations(spec, seed, device)
+        G = {}
+        for li, lin in enumerate(MODEL_LINEARS):
+            d_out, d_in = MODEL_SHAPE[lin]
+            spec = scaled(base, d_out=d_out, d_in=d_in, n_tokens=n_tokens)
+            G[lin] = gradients(spec, layer_seed(5, 100 * block + 10 + li), device)
+        out["X"], out["G"] = X, G
+    else:
+        W = {}
+        for li, lin in enumerate(MODEL_LINEARS):
+            d_out, d_in = MODEL_SHAPE[lin]
+            spec = scaled(base, d_out=d_out, d_in=d_in)
+            W[lin] = weights(spec, layer_seed(5, 100 * block + 20 + li), device)
+        out["W"] = W
+    return out
+
+
+def model_rht(block: int, name: str, n: int) -> RHTParams:
+    """Rotation parameters of input group / output of one linear of a block."""
+    tag = sum((i + 1) * ord(c) for i, c in enumerate(name))
+    return rht_params(n, layer_seed(5, 100 * block + 50) * 7 + tag)

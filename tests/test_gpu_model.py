@@ -1,0 +1,35 @@
+"""The whole-model driver (statistics of every linear, trace-sensitivity bit
+allocation, then BiIP + solver + loss per linear) on one 7B-shaped block with
+few tokens, checked against the oracle where the oracle can follow it: the
+allocation of bits from the same scores, and scores that separate q/k/v
+(same inputs, different gradients)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+
+pytestmark = pytest.mark.gpu
+
+
+def test_one_block_model():
+    if not torch.cuda.is_available():
+        pytest.fail("needs a CUDA GPU")
+    from post_weight_quantization_syrk_b200.model import SHAPE, synthetic_model
+    r = synthetic_model(n_tokens=2048, n_blocks=1).run()
+    pl = r["per_linear"]
+    assert len(pl) == 7 and r["weights"] == sum(SHAPE[x["linear"]][0] * SHAPE[x["linear"]][1] for x in pl)
+    scores = [x["score"] for x in pl]
+    n = [SHAPE[x["linear"]][0] * SHAPE[x["linear"]][1] for x in pl]
+    assert [x["bits"] for x in pl] == list(O.allocate_bits(scores, n, (2, 3, 4), 3.0))
+    assert r["average_bits"] <= 3.0 + 1e-12
+    # q, k, v share H_X but not H_G: the joint score tells them apart
+    trX = {x["linear"]: x["tr_X"] for x in pl}
+    assert trX["q"] == trX["k"] == trX["v"]
+    assert len({x["score"] for x in pl if x["linear"] in "qkv"}) == 3
+    for x in pl:
+        assert math.isfinite(x["loss"]) and x["loss"] > 0
+        assert abs(x["score"] - x["tr_X"] * x["tr_G"]) <= 1e-12 * abs(x["score"])
+    assert r["gpu_seconds"] > 0
