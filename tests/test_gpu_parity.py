@@ -166,7 +166,7 @@ def _uc_ok(got, ref):
     return np.max(np.abs(got - ref) - tol)
 
 
-@pytest.mark.parametrize("n,seed", [(1, 0), (63, 1), (64, 2), (200, 3), (704, 4), (1000, 5)])
+@pytest.mark.parametrize("n,seed", [(1, 0), (63, 1), (64, 2), (200, 3), (704, 4), (1000, 5), (1537, 6)])
 def test_chol_inv_parity(P, n, seed):
     H = _spd(n, seed)
     Hg = torch.from_numpy(H).cuda()
