@@ -9,8 +9,12 @@
 // up to ~60x to cancellation, which rules out plain TF32 or bf16 there.
 //
 // Structure (same as the covariance SYRK): persistent CTAs, one per SM, walk
-// 256 x 256 output tiles; each tile is two M=128 x N=256 accumulators (all
-// 512 TMEM columns).  Warp 0 streams 16-deep K slices of A and B (both
+// the output tiles in one of two shapes chosen per launch: wide tiles of
+// 256 x 256 (two M=128 x N=256 accumulators, all 512 TMEM columns), or
+// narrow tiles of 128 x 256 with two accumulators used in turn, so that the
+// epilogue of one tile overlaps the MMAs of the next (for products with few
+// tiles or a short K, where the wide tile's un-overlapped epilogue and the
+// last partial wave dominate).  Warp 0 streams 16-deep K slices of A and B (both
 // K-major, 64-byte swizzle; tcgen05 kind::tf32 produced no result with an
 // MN-major operand on B200 when measured, so callers pass B transposed), big
 // and small parts, through a 3-stage ring; one thread of warp 1 issues 12
@@ -35,9 +39,11 @@ constexpr int STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;
 constexpr int STAGES = 3;
 constexpr int THREADS = 320;                        // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr int kMaxSms = 148;   // SMs of a B200
 
 struct Params {
   int64_t M, N, K;
+  int wide;   // 1: 256 x 256 tiles, 0: 128 x 256 tiles
   int tiles_m, tiles_n, num_tiles, kblocks;
   int a_x0, a_y0, b_x0, b_y0;   // tensor-map coordinates of A(0,0) and B(0,0)
   int epilogue;
@@ -67,11 +73,12 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 3);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES);
-  const uint32_t accfull = smem_u32(bars + 2 * STAGES), accempty = smem_u32(bars + 2 * STAGES + 1);
-  const uint32_t drained = smem_u32(bars + 2 * STAGES + 2);
+  const uint32_t accfull0 = smem_u32(bars + 2 * STAGES), accempty0 = smem_u32(bars + 2 * STAGES + 2);
+  const uint32_t drained = smem_u32(bars + 2 * STAGES + 4);
+  const int bm = p.wide ? 256 : 128;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
   if (threadIdx.x == 0) {
@@ -79,8 +86,10 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
-    mbar_init(accfull, 1);
-    mbar_init(accempty, 256);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accfull0 + 8 * b, 1);
+      mbar_init(accempty0 + 8 * b, 256);
+    }
     mbar_init(drained, 1);
     *abort_flag = 0;
     mbar_init_fence();
@@ -103,18 +112,21 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       bool issued[STAGES] = {false, false, false};
       bool ok = true;
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
-        const int m0 = (t / p.tiles_n) * BM, n0 = (t % p.tiles_n) * BN;
+        const int m0 = (t / p.tiles_n) * bm, n0 = (t % p.tiles_n) * BN;
         for (int kb = 0; kb < p.kblocks; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.info, 11)) {
             ok = false;
             break;
           }
           const uint32_t fb = full0 + 8 * stage;
-          mbar_arrive_expect_tx(fb, STAGE_BYTES);
+          mbar_arrive_expect_tx(fb, p.wide ? STAGE_BYTES : STAGE_BYTES - A_BYTES);
           const uint32_t s0 = smem_u32(smem + stage * STAGE_BYTES);
           const int k0 = kb * BKF;
-          tma_load_2d(s0, &maps.ab, p.a_x0 + k0, p.a_y0 + m0, fb);
-          tma_load_2d(s0 + A_BYTES, &maps.as, p.a_x0 + k0, p.a_y0 + m0, fb);
+          // A boxes are 128 rows; a wide tile takes two per part
+          for (int h = 0; h <= p.wide; ++h) {
+            tma_load_2d(s0 + h * (A_BYTES / 2), &maps.ab, p.a_x0 + k0, p.a_y0 + m0 + 128 * h, fb);
+            tma_load_2d(s0 + A_BYTES + h * (A_BYTES / 2), &maps.as, p.a_x0 + k0, p.a_y0 + m0 + 128 * h, fb);
+          }
           tma_load_2d(s0 + 2 * A_BYTES, &maps.bb, p.b_x0 + k0, p.b_y0 + n0, fb);
           tma_load_2d(s0 + 2 * A_BYTES + B_BYTES, &maps.bs, p.b_x0 + k0, p.b_y0 + n0, fb);
           issued[stage] = true;
@@ -132,10 +144,12 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
   } else if (warp == 1) {
     if (lane == 0) {
       int stage = 0;
-      uint32_t phase = 0, acc_phase = 0;
+      uint32_t phase = 0, acc_bits = 0;   // bit b: phase of accumulator b
       bool ok = true, any = false;
-      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
-        if (!mbar_wait(accempty, acc_phase ^ 1u, abort_flag, p.info, 12)) break;
+      int local = 0;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++local) {
+        const int buf = p.wide ? 0 : (local & 1);
+        if (!mbar_wait(accempty0 + 8 * buf, ((acc_bits >> buf) & 1u) ^ 1u, abort_flag, p.info, 12)) break;
         fence_after();
         for (int kb = 0; kb < p.kblocks; ++kb) {
           if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, p.info, 13)) {
@@ -148,9 +162,8 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
 #pragma unroll
           for (int ks = 0; ks < BKF / 8; ++ks) {
             const uint64_t dbb = desc_op(bb + ks * 32), dbs = desc_op(bs + ks * 32);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const uint32_t d = tmem + 256 * h;
+            for (int h = 0; h <= p.wide; ++h) {
+              const uint32_t d = tmem + 256 * (h + buf);
               const uint32_t first = (kb == 0 && ks == 0) ? 0u : 1u;
               const uint64_t dab = desc_op(ab + h * (A_BYTES / 2) + ks * 32);
               const uint64_t das = desc_op(as + h * (A_BYTES / 2) + ks * 32);
@@ -167,8 +180,8 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
           }
         }
         if (!ok) break;
-        mma_commit(accfull);
-        acc_phase ^= 1u;
+        mma_commit(accfull0 + 8 * buf);
+        acc_bits ^= 1u << buf;
       }
       if (any) {
         mma_commit(drained);
@@ -183,18 +196,20 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
     const int e = warp - 2;
     const int wq = warp & 3;
     const int cbase = (e >> 2) * 128;
-    uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
-      const int64_t m0 = (int64_t)(t / p.tiles_n) * BM, n0 = (int64_t)(t % p.tiles_n) * BN;
+    uint32_t acc_bits = 0;   // bit b: phase of accumulator b
+    int local = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++local) {
+      const int buf = p.wide ? 0 : (local & 1);
+      const int64_t m0 = (int64_t)(t / p.tiles_n) * bm, n0 = (int64_t)(t % p.tiles_n) * BN;
       // one lane waits, the warp follows: every lane leaves together on abort
       bool ready = true;
-      if (lane == 0) ready = mbar_wait(accfull, acc_phase, abort_flag, p.info, 14);
+      if (lane == 0) ready = mbar_wait(accfull0 + 8 * buf, (acc_bits >> buf) & 1u, abort_flag, p.info, 14);
       if (!__shfl_sync(0xffffffffu, ready ? 1 : 0, 0)) break;
       __syncwarp();
       fence_after();
       double dot = 0.0;
 #pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
+      for (int h = 0; h <= p.wide; ++h) {
         const int64_t gi = m0 + h * 128 + 32 * wq + lane;
         const bool row_ok = gi < p.M;
 #pragma unroll 1
@@ -217,7 +232,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
 #pragma unroll
           for (int cc = 0; cc < 64; cc += 16) {
             float v[16];
-            tmem_ld16(tmem + ((uint32_t)(32 * wq) << 16) + (uint32_t)(256 * h + cbase + g0 + cc), v);
+            tmem_ld16(tmem + ((uint32_t)(32 * wq) << 16) + (uint32_t)(256 * (h + buf) + cbase + g0 + cc), v);
             if (!any) continue;
             const int64_t gj = gj0 + cc;
             if (fast) {
@@ -254,14 +269,14 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
         }
       }
       fence_before();
-      mbar_arrive(accempty);
+      mbar_arrive(accempty0 + 8 * buf);
       if (p.epilogue == kEpiDot) {
         // fixed-order reduction within the warp (xor butterfly); one partial
         // per (tile, epilogue warp), summed later in index order
         for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
         if (lane == 0) p.partial[8 * (int64_t)t + e] = dot;
       }
-      acc_phase ^= 1u;
+      acc_bits ^= 1u << buf;
     }
   }
 
@@ -320,7 +335,19 @@ __global__ void __launch_bounds__(256) split_kernel(const float* __restrict__ x,
 
 }  // namespace
 
-int64_t gemm_tiles(int64_t M, int64_t N) { return cdiv(M, BM) * cdiv(N, BN); }
+// Wide tiles when they fill two waves, or when K is long enough that the
+// un-overlapped epilogue is a small share of a tile (measured on B200: the
+// 4096^3 products of the loss run 15 % faster wide, the solver's K <= 1024
+// updates 20 % faster narrow).
+bool gemm_wide(int64_t M, int64_t N, int64_t K) {
+  return cdiv(M, BM) * cdiv(N, BN) >= 2 * kMaxSms || K >= 2048;
+}
+
+int64_t gemm_tiles(int64_t M, int64_t N, int64_t K) {
+  return cdiv(M, gemm_wide(M, N, K) ? BM : BM / 2) * cdiv(N, BN);
+}
+
+int64_t gemm_tiles_max(int64_t M, int64_t N) { return cdiv(M, BM / 2) * cdiv(N, BN); }
 
 kq_status split_tf32(const float* x, int64_t ldx, const float* y, int64_t ldy, int64_t rows, int64_t cols, float* big,
                      float* small, int64_t ldo, bool transpose, cudaStream_t st) {
@@ -344,20 +371,21 @@ kq_status gemm_3xtf32(const Gemm3xTF32& g, cudaStream_t st) {
   // Tensor maps end exactly at the used region, so every read past M, N or K
   // (ragged tiles, a K tail) is filled with zeros by the TMA unit.
   Maps maps;
-  auto map_op = [&](CUtensorMap* m, const float* base, int64_t ld, int64_t row0, int64_t col0, int64_t rows)
-      -> kq_status {
-    return tc::make_map_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, col0 + g.K, row0 + rows, ld, BKF, BM,
+  auto map_op = [&](CUtensorMap* m, const float* base, int64_t ld, int64_t row0, int64_t col0, int64_t rows,
+                    int box_rows) -> kq_status {
+    return tc::make_map_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, col0 + g.K, row0 + rows, ld, BKF, box_rows,
                            CU_TENSOR_MAP_SWIZZLE_64B);
   };
-  KQ_TRY(map_op(&maps.ab, g.a_big, g.lda, g.a_row0, g.a_col0, g.M));
-  KQ_TRY(map_op(&maps.as, g.a_small, g.lda, g.a_row0, g.a_col0, g.M));
-  KQ_TRY(map_op(&maps.bb, g.bt_big, g.ldbt, g.bt_row0, g.bt_col0, g.N));
-  KQ_TRY(map_op(&maps.bs, g.bt_small, g.ldbt, g.bt_row0, g.bt_col0, g.N));
+  KQ_TRY(map_op(&maps.ab, g.a_big, g.lda, g.a_row0, g.a_col0, g.M, 128));
+  KQ_TRY(map_op(&maps.as, g.a_small, g.lda, g.a_row0, g.a_col0, g.M, 128));
+  KQ_TRY(map_op(&maps.bb, g.bt_big, g.ldbt, g.bt_row0, g.bt_col0, g.N, BN));
+  KQ_TRY(map_op(&maps.bs, g.bt_small, g.ldbt, g.bt_row0, g.bt_col0, g.N, BN));
   Params p;
   p.M = g.M;
   p.N = g.N;
   p.K = g.K;
-  p.tiles_m = (int)cdiv(g.M, BM);
+  p.wide = gemm_wide(g.M, g.N, g.K) ? 1 : 0;
+  p.tiles_m = (int)cdiv(g.M, p.wide ? BM : BM / 2);
   p.tiles_n = (int)cdiv(g.N, BN);
   p.num_tiles = p.tiles_m * p.tiles_n;
   p.kblocks = (int)cdiv(g.K, BKF);

@@ -37,8 +37,10 @@ struct Gemm3xTF32 {
   int32_t* info = nullptr;
 };
 
-// Output tiles of an M x N product (`partial` holds 8 per tile for kEpiDot).
-int64_t gemm_tiles(int64_t M, int64_t N);
+// Output tiles of an M x N x K product as launched (`partial` holds 8 per
+// tile for kEpiDot), and the most tiles any M x N product can use.
+int64_t gemm_tiles(int64_t M, int64_t N, int64_t K);
+int64_t gemm_tiles_max(int64_t M, int64_t N);
 
 kq_status gemm_3xtf32(const Gemm3xTF32& g, cudaStream_t st);
 

@@ -157,7 +157,7 @@ size_t loss_layout(int64_t d_out, int64_t d_in, LossWs* w, void* base) {
                sg = (size_t)d_out * ldg * 4;
   size_t oDb = take(sd), oDs = take(sd), oTb = take(st_), oTs = take(st_), oXb = take(sx), oXs = take(sx),
          oGb = take(sg), oGs = take(sg), oA = take(sd);
-  const int64_t np = std::max<int64_t>(8 * kq::gemm_tiles(d_out, d_in), kDotBlocks);
+  const int64_t np = std::max<int64_t>(8 * kq::gemm_tiles_max(d_out, d_in), kDotBlocks);
   size_t oP = take((size_t)np * 8);
   if (w && base) {
     char* b = static_cast<char*>(base);
@@ -234,7 +234,7 @@ extern "C" kq_status kq_kron_loss(const float* W, int64_t ldw, const float* W_ha
     g2.ld_other = w.ldd;
     g2.partial = w.partial;
     KQ_TRY(kq::gemm_3xtf32(g2, st));
-    np = 8 * kq::gemm_tiles(d_out, d_in);
+    np = 8 * kq::gemm_tiles(d_out, d_in, d_out);
   } else {
     dot_rows_kernel<<<kDotBlocks, 256, 0, st>>>(w.A1, w.Db, w.Ds, w.ldd, d_out, d_in, w.partial);
     KQ_TRY(kq::launch_check("kq_kron_loss dot"));

@@ -51,19 +51,49 @@ __device__ __forceinline__ void fwht_regs(float (&r)[16], int g) {
   }
 }
 
-// y[a] = sum_c Q[a][c] x[c] (or Q^T) for one strand of m <= 64 values kept in
-// registers (fully unrolled over the 64 slots, predicated on m).
-template <typename Get, typename Put>
-__device__ __forceinline__ void qmix_strand(const float* Qs, int m, bool transpose, Get get, Put put) {
-  float x[kMaxM];
+// In-place Q_m mix of S strands of m <= 64 values in shared memory:
+// element q of strand s at buf[addr(q, s)] becomes sum_c Q[q][c] x_s[c]
+// (Q^T when transposing).  A register-tiled small product: thread t owns the
+// output rows of group t / 64 (ceil(m / 4) rows) for the four strands
+// t % 64 + 64 j of each 256-strand chunk, so every Q value it reads from
+// shared memory (a warp-wide broadcast) feeds four FMAs and every strand
+// value feeds up to 16.  Must be called by all 256 threads; ends with a
+// barrier.
+template <typename Addr>
+__device__ void qmix_tile(float* buf, const float* Qs, int m, int S, bool transpose, Addr addr) {
+  const int t = threadIdx.x, bb = t & 63, ag = t >> 6;
+  const int am = (m + 3) >> 2, a0 = ag * am;
+  for (int chunk = 0; chunk < S; chunk += 256) {
+    float acc[16][4];
 #pragma unroll
-  for (int c = 0; c < kMaxM; ++c) x[c] = (c < m) ? get(c) : 0.f;
-  for (int a = 0; a < m; ++a) {
-    float acc = 0.f;
+    for (int i = 0; i < 16; ++i)
 #pragma unroll
-    for (int c = 0; c < kMaxM; ++c)
-      if (c < m) acc = fmaf(transpose ? Qs[c * m + a] : Qs[a * m + c], x[c], acc);
-    put(a, acc);
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    for (int c = 0; c < m; ++c) {
+      float xv[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int sj = chunk + bb + 64 * j;
+        xv[j] = (sj < S) ? buf[addr(c, sj)] : 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        if (i < am && a0 + i < m) {
+          const float q = transpose ? Qs[c * m + a0 + i] : Qs[(a0 + i) * m + c];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(q, xv[j], acc[i][j]);
+        }
+      }
+    }
+    __syncthreads();   // every read of this chunk is done
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int sj = chunk + bb + 64 * j;
+        if (i < am && a0 + i < m && sj < S) buf[addr(a0 + i, sj)] = acc[i][j];
+      }
+    __syncthreads();
   }
 }
 
@@ -124,27 +154,36 @@ __global__ void __launch_bounds__(256) rotate_rows_kernel(float* __restrict__ M,
   if (m > 1)
     for (int i = threadIdx.x; i < m * m; i += blockDim.x) Qs[i] = Qm[i];
   if ((n & 3) == 0) {
-    for (int i4 = threadIdx.x; i4 < n / 4; i4 += blockDim.x) {
-      float4 v = reinterpret_cast<const float4*>(row)[i4];
-      if (!inverse) {
-        const float4 sg = reinterpret_cast<const float4*>(signs)[i4];
-        v.x *= sg.x; v.y *= sg.y; v.z *= sg.z; v.w *= sg.w;
+    // eight float4 loads of the row (and of the signs) in flight per thread
+    const int n4 = n / 4;
+    for (int b4 = 0; b4 < n4; b4 += 8 * 256) {
+      float4 v[8], sg[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i4 = b4 + threadIdx.x + 256 * u;
+        if (i4 < n4) {
+          v[u] = reinterpret_cast<const float4*>(row)[i4];
+          sg[u] = inverse ? make_float4(1.f, 1.f, 1.f, 1.f) : reinterpret_cast<const float4*>(signs)[i4];
+        }
       }
-      const int i = 4 * i4;
-      x[pad16(i)] = v.x;
-      x[pad16(i + 1)] = v.y;
-      x[pad16(i + 2)] = v.z;
-      x[pad16(i + 3)] = v.w;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i4 = b4 + threadIdx.x + 256 * u;
+        if (i4 < n4) {
+          const int i = 4 * i4;
+          x[pad16(i)] = v[u].x * sg[u].x;
+          x[pad16(i + 1)] = v[u].y * sg[u].y;
+          x[pad16(i + 2)] = v[u].z * sg[u].z;
+          x[pad16(i + 3)] = v[u].w * sg[u].w;
+        }
+      }
     }
   } else {
     for (int i = threadIdx.x; i < n; i += blockDim.x) x[pad16(i)] = inverse ? row[i] : row[i] * signs[i];
   }
   __syncthreads();
   auto qmix = [&](bool transpose) {
-    for (int b = threadIdx.x; b < p; b += blockDim.x)
-      qmix_strand(Qs, m, transpose, [&](int c) { return x[pad16(c * p + b)]; },
-                  [&](int a, float v) { x[pad16(a * p + b)] = v; });
-    __syncthreads();
+    qmix_tile(x, Qs, m, p, transpose, [&](int q, int b) { return pad16(q * p + b); });
   };
   if (inverse && m > 1) qmix(true);
   fwht_passes<true>(x, log2_p, m);
@@ -183,21 +222,32 @@ __global__ void __launch_bounds__(256) rotate_cols_inner_kernel(float* __restric
   const int rs = threadIdx.x / (kStrip / 4);
   const int rstep = blockDim.x / (kStrip / 4);
   const bool full = c0 + c4 + 3 < cols;
-  for (int r = rs; r < p2; r += rstep) {
-    const float* src = M + (r0 + r) * ld + c0 + c4;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (full) {
-      v = *reinterpret_cast<const float4*>(src);
-    } else {
-      if (c0 + c4 + 0 < cols) v.x = src[0];
-      if (c0 + c4 + 1 < cols) v.y = src[1];
-      if (c0 + c4 + 2 < cols) v.z = src[2];
+  for (int rb = rs; rb < p2; rb += 8 * rstep) {   // eight row loads in flight per thread
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int r = rb + u * rstep;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < p2) {
+        const float* src = M + (r0 + r) * ld + c0 + c4;
+        if (full) {
+          v[u] = *reinterpret_cast<const float4*>(src);
+        } else {
+          if (c0 + c4 + 0 < cols) v[u].x = src[0];
+          if (c0 + c4 + 1 < cols) v[u].y = src[1];
+          if (c0 + c4 + 2 < cols) v[u].z = src[2];
+        }
+      }
     }
-    if (!inverse) {
-      const float sg = signs[r0 + r];
-      v.x *= sg; v.y *= sg; v.z *= sg; v.w *= sg;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int r = rb + u * rstep;
+      if (r < p2) {
+        const float sg = inverse ? 1.f : signs[r0 + r];
+        *reinterpret_cast<float4*>(t + r * kStrip + c4) =
+            make_float4(v[u].x * sg, v[u].y * sg, v[u].z * sg, v[u].w * sg);
+      }
     }
-    *reinterpret_cast<float4*>(t + r * kStrip + c4) = v;
   }
   __syncthreads();
   fwht_passes<false>(t, log2_p2, kStrip);
@@ -235,27 +285,34 @@ __global__ void __launch_bounds__(256) rotate_cols_outer_kernel(float* __restric
   const bool full = c0 + c4 + 3 < cols;
   if (m > 1)
     for (int i = threadIdx.x; i < m * m; i += blockDim.x) Qs[i] = Qm[i];
-  for (int r = rs; r < R; r += rstep) {
-    const int a = r >> log2_p1, b1 = r & (p1 - 1);
-    const float* src = M + ((int64_t)a * p + (int64_t)b1 * p2 + b2) * ld + c0 + c4;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (full) {
-      v = *reinterpret_cast<const float4*>(src);
-    } else {
-      if (c0 + c4 + 0 < cols) v.x = src[0];
-      if (c0 + c4 + 1 < cols) v.y = src[1];
-      if (c0 + c4 + 2 < cols) v.z = src[2];
+  for (int rb = rs; rb < R; rb += 8 * rstep) {   // eight row loads in flight per thread
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int r = rb + u * rstep;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < R) {
+        const int a = r >> log2_p1, b1 = r & (p1 - 1);
+        const float* src = M + ((int64_t)a * p + (int64_t)b1 * p2 + b2) * ld + c0 + c4;
+        if (full) {
+          v[u] = *reinterpret_cast<const float4*>(src);
+        } else {
+          if (c0 + c4 + 0 < cols) v[u].x = src[0];
+          if (c0 + c4 + 1 < cols) v[u].y = src[1];
+          if (c0 + c4 + 2 < cols) v[u].z = src[2];
+        }
+      }
     }
-    *reinterpret_cast<float4*>(t + r * kStrip + c4) = v;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int r = rb + u * rstep;
+      if (r < R) *reinterpret_cast<float4*>(t + r * kStrip + c4) = v[u];
+    }
   }
   __syncthreads();
   auto qmix = [&](bool transpose) {
-    for (int idx = threadIdx.x; idx < p1 * kStrip; idx += blockDim.x) {
-      const int b1 = idx / kStrip, c = idx % kStrip;
-      qmix_strand(Qs, m, transpose, [&](int q) { return t[(q * p1 + b1) * kStrip + c]; },
-                  [&](int a, float v) { t[(a * p1 + b1) * kStrip + c] = v; });
-    }
-    __syncthreads();
+    // strand s = (b1, c) with b1 = s / 128, c = s % 128
+    qmix_tile(t, Qs, m, p1 * kStrip, transpose, [&](int q, int s) { return (q * p1 + (s >> 7)) * kStrip + (s & 127); });
   };
   if (m > 1 && inverse) qmix(true);
   fwht_passes<false>(t, log2_p1, kStrip * m);
