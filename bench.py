@@ -234,6 +234,7 @@ def run_kronq(a):
 
     pk, src = peaks()
     flops = spec.n_tokens * spec.d_in * (spec.d_in + 1)    # one SYRK launch on X (d_out == d_in here)
+    traffic = syrk_traffic(a.workload)
     syrk_avg = statistics.mean(syrk_ms)
     achieved = flops / (syrk_avg / 1e3) / 1e12
     peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
@@ -247,7 +248,7 @@ def run_kronq(a):
                    "trailing_update": a.gemm,
                    "l2": "inputs larger than L2 (X, G 2 GiB each); no flush"},
         "roofline": {"kernel": "kq_accum_cov (SYRK)", "bound": "tensor", "achieved": achieved, "peak": peak,
-                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{src} bf16 sustained", "algorithmic_flops_per_launch": flops,
                      "avg_launch_ms": syrk_avg},
         "stages_ms": stages_ms,
@@ -265,38 +266,47 @@ def run_kronq(a):
         print(json.dumps(out), flush=True)
 
 
+# DRAM bytes (read + write) of one kq_accum_cov call at 262144 x 4096, from the
+# ncu capture summarised in profiles/syrk_tc_kernel_attn4096_traffic.md; valid
+# only for the kernel sources it was taken on.
+SYRK_TRAFFIC = {"attn4096": 5.27e9}
+SYRK_SOURCE_SHA = {"kq_syrk.cu": "a119b81f79593294", "kq_tc.cuh": "f59b54090d782541"}
+
+
+def syrk_traffic(workload):
+    import hashlib
+    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "post_weight_quantization_syrk_b200", "csrc")
+    for name, want in SYRK_SOURCE_SHA.items():
+        with open(os.path.join(csrc, name), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest()[:16] != want:
+                return None
+    return SYRK_TRAFFIC.get(workload)
+
+
 def run_e2e(a, lq, results, W, X, G, T_in, T_out, spec, settings, world, dev):
-    """Same step through the public API from pinned host buffers: inputs are
-    copied host->device and the results (codes, grids, losses) device->host
-    inside the timed region."""
+    """Same step through the public API from pinned host buffers: every step
+    copies its inputs host->device and its results (codes, grids, losses)
+    device->host inside the timed region.  pipeline.quantize_from_host
+    overlaps step i+1's input copies with step i's compute."""
     import torch
+    from post_weight_quantization_syrk_b200.pipeline import quantize_from_host
     Wh, Xh, Gh = W.cpu().pin_memory(), X.cpu().pin_memory(), G.cpu().pin_memory()
-    Wd, Xd, Gd = torch.empty_like(W), torch.empty_like(X), torch.empty_like(G)
-    outs = [(torch.empty(r.codes.shape, dtype=torch.uint8, pin_memory=True),
-             torch.empty(r.scales.shape, pin_memory=True), torch.empty(r.zeros.shape, pin_memory=True),
-             torch.empty(1, dtype=torch.float64, pin_memory=True)) for r in results]
+    n = max(3, min(a.steps, 5))
+
+    def outputs():
+        return [(torch.empty(r.codes.shape, dtype=torch.uint8, pin_memory=True),
+                 torch.empty(r.scales.shape, pin_memory=True), torch.empty(r.zeros.shape, pin_memory=True),
+                 torch.empty(1, dtype=torch.float64, pin_memory=True)) for r in results]
+
+    outs = [outputs() for _ in range(n)]
     h2d = Wh.numel() * 4 + Xh.numel() * 2 + Gh.numel() * 2
-    d2h = sum(o[0].numel() + o[1].numel() * 4 + o[2].numel() * 4 + 8 for o in outs)
+    d2h = sum(o[0].numel() + o[1].numel() * 4 + o[2].numel() * 4 + 8 for o in outs[0])
     stream = torch.cuda.current_stream()
-    n = min(a.steps, 3)
-
-    def one():
-        Wd.copy_(Wh, non_blocking=True)
-        Xd.copy_(Xh, non_blocking=True)
-        Gd.copy_(Gh, non_blocking=True)
-        lq.run(Wd, Xd, Gd, T_in, T_out, settings, results=results)
-        for r, o in zip(results, outs):
-            o[0].copy_(r.codes, non_blocking=True)
-            o[1].copy_(r.scales, non_blocking=True)
-            o[2].copy_(r.zeros, non_blocking=True)
-            o[3].copy_(r.loss, non_blocking=True)
-
-    one()
+    quantize_from_host(lq, [(Wh, Xh, Gh)], T_in, T_out, settings, results, outs[:1])   # warm
     torch.cuda.synchronize()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     s.record(stream)
-    for _ in range(n):
-        one()
+    quantize_from_host(lq, [(Wh, Xh, Gh)] * n, T_in, T_out, settings, results, outs)
     e.record(stream)
     torch.cuda.synchronize()
     ms = s.elapsed_time(e)
@@ -306,7 +316,8 @@ def run_e2e(a, lq, results, W, X, G, T_in, T_out, spec, settings, world, dev):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms = float(t.item())
     return {"value": spec.d_out * spec.d_in * len(settings) * n * world / (ms / 1e3), "unit": UNIT,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms / n, "steps": n}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms / n, "steps": n,
+            "overlap": "step i+1's host->device copies run on a second stream during step i's compute"}
 
 
 # ----------------------------------------------------------------- CPU oracle

@@ -115,3 +115,58 @@ class LayerQuantizer:
 
     def check(self, where="kronq"):
         K.check_info(self.info, where)
+
+
+def quantize_from_host(lq: LayerQuantizer, host_layers, T_in, T_out, settings, results, host_outputs,
+                       damp_frac=0.01):
+    """Run the whole path over a sequence of layers of one shape whose inputs
+    live in pinned host memory, overlapping transfers with compute.
+
+    host_layers[i] = (W, X, G) pinned CPU tensors; host_outputs[i][k] =
+    (codes, scales, zeros, loss) pinned CPU tensors for settings[k].  Layer
+    i+1's inputs are copied host->device on a separate stream into the other
+    of two device buffer sets while layer i is quantized on the current
+    stream; layer i's results are copied back on the current stream right
+    after it (device->host, the other PCIe direction).  A buffer set is
+    refilled only after the layer that used it has finished.  Asynchronous:
+    the caller synchronises the current stream before reading host_outputs.
+    """
+    dev = lq.device
+    comp = torch.cuda.current_stream(dev)
+    copy = torch.cuda.Stream(device=dev)
+    first = host_layers[0]
+    bufs = [tuple(torch.empty(t.shape, dtype=t.dtype, device=dev) for t in first) for _ in range(2)]
+    copied = [torch.cuda.Event() for _ in range(2)]
+    freed = [torch.cuda.Event() for _ in range(2)]
+    start = torch.cuda.Event()
+    start.record(comp)
+    copy.wait_event(start)
+
+    def issue_copy(i):
+        slot = i % 2
+        with torch.cuda.stream(copy):
+            if i >= 2:
+                copy.wait_event(freed[slot])
+            for d, h in zip(bufs[slot], host_layers[i]):
+                d.copy_(h, non_blocking=True)
+            copied[slot].record(copy)
+
+    issue_copy(0)
+    for i in range(len(host_layers)):
+        if i + 1 < len(host_layers):
+            issue_copy(i + 1)
+        slot = i % 2
+        comp.wait_event(copied[slot])
+        W, X, G = bufs[slot]
+        lq.run(W, X, G, T_in, T_out, settings, damp_frac=damp_frac, results=results)
+        freed[slot].record(comp)
+        for r, o in zip(results, host_outputs[i]):
+            o[0].copy_(r.codes, non_blocking=True)
+            o[1].copy_(r.scales, non_blocking=True)
+            o[2].copy_(r.zeros, non_blocking=True)
+            o[3].copy_(r.loss, non_blocking=True)
+    # the device buffers were last used on `comp`; keep them alive until then
+    for b in bufs:
+        for t in b:
+            t.record_stream(comp)
+    return results
