@@ -127,21 +127,18 @@ __global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
   const int bw = a.bw;
   const int64_t i0 = a.i0;
 
-  for (int idx = t; idx < BLK * (BLK / 4); idx += IB_THREADS) {
+  // the block of Uc: 16 asynchronous 16-byte copies per thread, all in
+  // flight while the row is loaded (bytes past the block are zero-filled)
+#pragma unroll
+  for (int u = 0; u < BLK * (BLK / 4) / IB_THREADS; ++u) {
+    const int idx = t + IB_THREADS * u;
     const int j = idx / (BLK / 4), k = 4 * (idx % (BLK / 4));
-    float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (j < bw) {
-      const float* g = a.Uc + (i0 + j) * a.lduc + i0 + k;
-      if (k + 3 < bw) {
-        u = *reinterpret_cast<const float4*>(g);
-      } else {
-        if (k + 0 < bw) u.x = g[0];
-        if (k + 1 < bw) u.y = g[1];
-        if (k + 2 < bw) u.z = g[2];
-      }
-    }
-    *reinterpret_cast<float4*>(Us + j * BLK + k) = u;
+    const int nbytes = (j < bw) ? 4 * max(0, min(4, bw - k)) : 0;
+    const float* g = nbytes ? a.Uc + (i0 + j) * a.lduc + i0 + k : a.Uc + i0 * a.lduc + i0;
+    const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(Us + j * BLK + k));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(g), "r"(nbytes) : "memory");
   }
+  asm volatile("cp.async.commit_group;" ::: "memory");
 
   // this lane's 16 columns of the row
   float w[16];
@@ -163,6 +160,7 @@ __global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) w[4 * m + e] = v[e];
   }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
   if (t < BLK) inv_d[t] = (t < bw) ? 1.f / Us[t * BLK + t] : 0.f;
   __syncthreads();

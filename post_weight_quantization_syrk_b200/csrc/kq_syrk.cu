@@ -325,8 +325,17 @@ struct Plan {
   int T, num_tiles, kblocks, splits, kb_per_split, num_units;
 };
 
+// At most this many 64-token blocks accumulate in one TMEM accumulator.
+// The tensor core's fp32 accumulation loses a small systematic amount per
+// MMA (measured on B200 for bf16 inputs: the diagonal of a covariance comes
+// out low by about 4e-9 x the tokens in one accumulation chain: 4.8e-5 at
+// 12288 tokens, 1.1e-4 at 24576), so long token ranges are split and the
+// splits summed in fp32 in a fixed order.
+constexpr int kMaxKbPerSplit = 192;   // 12288 tokens
+
 // Token splits per tile: minimise (waves / splits) x full-tile MMA time plus
-// the partial-tile round trip through HBM, with waves counted on 148 SMs.
+// the partial-tile round trip through HBM, with waves counted on 148 SMs,
+// subject to the chain-length cap above.
 Plan make_plan(int64_t n, int64_t d) {
   Plan pl;
   pl.T = (int)kq::cdiv(d, TILE);
@@ -335,8 +344,9 @@ Plan make_plan(int64_t n, int64_t d) {
   const double tile_s = 2.0 * TILE * TILE * (double)n / (1.4e15 / ASSUMED_SMS);
   double best = 1e300;
   int best_s = 1;
-  const int smax = std::min(16, std::max(1, pl.kblocks));
-  for (int s = 1; s <= smax; ++s) {
+  const int smin = std::max(1, (int)kq::cdiv(pl.kblocks, kMaxKbPerSplit));
+  const int smax = std::max(smin, std::min(16, std::max(1, pl.kblocks)));
+  for (int s = smin; s <= smax; ++s) {
     const int per = (int)kq::cdiv(pl.kblocks, s);
     const int s_eff = (int)kq::cdiv(pl.kblocks, per);
     if (s_eff != s) continue;
