@@ -133,7 +133,9 @@ __global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
   for (int u = 0; u < BLK * (BLK / 4) / IB_THREADS; ++u) {
     const int idx = t + IB_THREADS * u;
     const int j = idx / (BLK / 4), k = 4 * (idx % (BLK / 4));
-    const int nbytes = (j < bw) ? 4 * max(0, min(4, bw - k)) : 0;
+    // chunks wholly below the diagonal (k + 3 < j) are zero-filled: only the
+    // upper triangle of Uc is the factor
+    const int nbytes = (j < bw && k + 3 >= j) ? 4 * max(0, min(4, bw - k)) : 0;
     const float* g = nbytes ? a.Uc + (i0 + j) * a.lduc + i0 + k : a.Uc + i0 * a.lduc + i0;
     const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(Us + j * BLK + k));
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(g), "r"(nbytes) : "memory");
@@ -161,6 +163,12 @@ __global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
     for (int e = 0; e < 4; ++e) w[4 * m + e] = v[e];
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
+  // ... and in the chunk holding the diagonal, the entries left of it are
+  // cleared, so that the column updates below can run unpredicated
+  if (t < BLK) {
+    for (int k = t & ~3; k < t; ++k) Us[t * BLK + k] = 0.f;
+  }
   __syncthreads();
   if (t < BLK) inv_d[t] = (t < bw) ? 1.f / Us[t * BLK + t] : 0.f;
   __syncthreads();
@@ -217,22 +225,23 @@ __global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
         const float q = fminf(fmaxf(rintf(v), 0.f), a.nl);
         const float wh = scale * (q - zero);
         const float e_own = (x - wh) * inv_d[j];
+        const float e = __shfl_sync(0xffffffffu, e_own, gbase + Lo);
+        // columns left of j see Uc[j][c] = 0 (cleared above), so the update
+        // runs over all of this lane's columns; column j itself is then set
+        // to its final dequantized value by its owner
+        // register blocks m2 < m hold columns left of 32 m <= j: final, skipped
+        const float4* urow = reinterpret_cast<const float4*>(Us + j * BLK);
+#pragma unroll
+        for (int m2 = m; m2 < 4; ++m2) {
+          const float4 u = urow[8 * m2 + L];
+          const float uu[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int t2 = 0; t2 < 4; ++t2) w[4 * m2 + t2] = fmaf(-e, uu[t2], w[4 * m2 + t2]);
+        }
         if (L == Lo) {
           qv[r] = q;
           w[r] = wh;   // the column is final: keep its dequantized value
           ev[r] = e_own;
-        }
-        const float e = __shfl_sync(0xffffffffu, e_own, gbase + Lo);
-        const float4* urow = reinterpret_cast<const float4*>(Us + j * BLK);
-#pragma unroll
-        for (int m2 = 0; m2 < 4; ++m2) {
-          const float4 u = urow[8 * m2 + L];
-          const float uu[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-          for (int t2 = 0; t2 < 4; ++t2) {
-            const int r2 = 4 * m2 + t2;
-            if (col_of(L, r2) > j) w[r2] = fmaf(-e, uu[t2], w[r2]);
-          }
         }
       }
     }
