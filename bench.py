@@ -269,8 +269,8 @@ def run_kronq(a):
 # DRAM bytes (read + write) of one kq_accum_cov call at 262144 x 4096, from the
 # ncu capture summarised in profiles/syrk_tc_kernel_attn4096_traffic.md; valid
 # only for the kernel sources it was taken on.
-SYRK_TRAFFIC = {"attn4096": 5.27e9}
-SYRK_SOURCE_SHA = {"kq_syrk.cu": "a119b81f79593294", "kq_tc.cuh": "f59b54090d782541"}
+SYRK_TRAFFIC = {"attn4096": 5.00e9}
+SYRK_SOURCE_SHA = {"kq_syrk.cu": "fae4d540a18d7937", "kq_tc.cuh": "f59b54090d782541"}
 
 
 def syrk_traffic(workload):
