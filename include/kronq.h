@@ -197,7 +197,11 @@ kq_status kq_chol_inv(const float* H, int64_t n, int64_t ldh, float damp_frac,
  * scale 1, zero rint(-min)); per output channel (group == 0, fitted on the
  * initial rows) or per `group` columns (fitted on the current values when the
  * group's first column is reached).  Dead columns (dead_mask[j] != 0) are
- * zeroed first.  All arithmetic is IEEE fp32 (true division, rint half-even).
+ * zeroed first.  Arithmetic is fp32: v = fma(w_j, 1/scale, zero) with the
+ * reciprocal rounded once per grid, q = clamp(rint(v)) (rint half-to-even),
+ * w_hat = scale (q - zero), e = (w_j - w_hat) * (1 / Uc[j][j]).  A code can
+ * therefore differ from one computed with true division only where v lies
+ * within about 1e-6 grid steps of a rounding boundary.
  *
  *   W        fp32 [d_out, d_in] rotated weights, ldw >= d_in (read only).
  *   Uc       fp32 [d_in, d_in] from kq_chol_inv, lduc >= d_in.
