@@ -219,18 +219,22 @@ def run_kronq(a):
     if not a.no_e2e:
         e2e = run_e2e(a, lq, results, W, X, G, T_in, T_out, spec, settings, world, dev)
 
-    # ---- the whole 7B-shaped model (32 blocks x 7 linears), one GPU
+    # ---- the whole 7B-shaped model (32 blocks x 7 linears); on N ranks each
+    # takes every N-th block and the sensitivity table is merged for the
+    # allocation (the model's total work is fixed: strong scaling)
     model = None
-    if world == 1 and not a.no_model:
+    if not a.no_model:
         from post_weight_quantization_syrk_b200.model import synthetic_model
         del X, G
         torch.cuda.empty_cache()
-        r = synthetic_model(n_tokens=spec.n_tokens, n_blocks=a.model_blocks, device=dev, gemm_mode=gemm_mode).run()
-        model = {k: r[k] for k in ("blocks", "linears", "weights", "gpu_seconds", "weights_per_s", "phase_seconds",
-                                   "input_generation_seconds", "average_bits", "bits_histogram")}
+        r = synthetic_model(n_tokens=spec.n_tokens, n_blocks=a.model_blocks, device=dev, gemm_mode=gemm_mode,
+                            rank=rank, world=world).run()
+        model = {k: r[k] for k in ("blocks", "linears", "weights", "ranks", "gpu_seconds", "weights_per_s",
+                                   "phase_seconds", "input_generation_seconds", "average_bits", "bits_histogram")}
         model["tokens"] = spec.n_tokens
         model["note"] = ("end-to-end GPU time of the whole path for all linears (statistics, sensitivity, bit "
-                         "allocation, BiIP, Cholesky, solver, loss); synthetic inputs generated per block, untimed")
+                         "allocation, BiIP, Cholesky, solver, loss), the slowest rank's when sharded; phase "
+                         "seconds are rank 0's; synthetic inputs generated per block, untimed")
 
     pk, src = peaks()
     flops = spec.n_tokens * spec.d_in * (spec.d_in + 1)    # one SYRK launch on X (d_out == d_in here)

@@ -14,7 +14,8 @@ Order (KronQ paper page, Abstract; KronQ review, Method and Comparison):
     and its Kronecker loss.
 GPU time is taken with CUDA events around each phase; generating the
 synthetic inputs is reported separately and is not part of the quantization
-time.
+time.  On several ranks each takes the blocks of dist.shard and the score
+table is merged across ranks before the (identical) allocation.
 """
 from __future__ import annotations
 
@@ -24,6 +25,7 @@ import time
 import torch
 
 from . import _lib as K
+from . import dist as D
 
 D_MODEL = 4096
 D_FF = 11008
@@ -63,7 +65,7 @@ class ModelQuantizer:
     tensors of one block (X per input group, G and W per linear)."""
 
     def __init__(self, make_inputs, make_rht, n_tokens, n_blocks=N_BLOCKS, device="cuda",
-                 choices=(2, 3, 4), avg_bits=3.0, gemm_mode=K.KQ_GEMM_3XTF32, damp=0.01):
+                 choices=(2, 3, 4), avg_bits=3.0, gemm_mode=K.KQ_GEMM_3XTF32, damp=0.01, rank=0, world=1):
         self.make_inputs, self.make_rht = make_inputs, make_rht
         self.n_tokens, self.n_blocks, self.dev = n_tokens, n_blocks, torch.device(device)
         self.choices, self.avg_bits, self.gemm_mode, self.damp = choices, avg_bits, gemm_mode, damp
@@ -71,6 +73,8 @@ class ModelQuantizer:
         self.ws = K.workspace(256, self.dev)
         self.phases = {k: Phase() for k in ("statistics", "sensitivity", "rotate", "chol_inv", "quantize", "loss")}
         self.gen_s = 0.0
+        self.rank, self.world = rank, world
+        self.blocks = D.shard(n_blocks, rank, world)
 
     def _ws(self, nbytes):
         if nbytes > self.ws.numel():
@@ -84,13 +88,29 @@ class ModelQuantizer:
         e1.record()
         self._events.append((name, e0, e1))
 
+    def allocate(self, sens):
+        """Bits for every linear of the model from this rank's scores: sens
+        maps (block, linear) -> (tr_X, tr_G, score) for the blocks of this
+        rank; the table is merged across ranks, then every rank runs the
+        same allocation.  Returns (alloc, full table)."""
+        table = torch.zeros((self.n_blocks, len(LINEARS), 3), dtype=torch.float64,
+                            device=self.dev if self.world > 1 and self.dev.type == "cuda" else "cpu")
+        for (b, lin), v in sens.items():
+            table[b, LINEARS.index(lin)] = torch.tensor(v, dtype=torch.float64)
+        table = D.merge_table(table).cpu()
+        keys = [(b, lin) for b in range(self.n_blocks) for lin in LINEARS]
+        full = {k: table[k[0], LINEARS.index(k[1])].tolist() for k in keys}
+        n_params = [SHAPE[lin][0] * SHAPE[lin][1] for _, lin in keys]
+        bits = K.kq_allocate_bits([full[k][2] for k in keys], n_params, self.choices, self.avg_bits)
+        return dict(zip(keys, bits)), full
+
     def run(self):
         self._events = []
         dev = self.dev
         HX, HG, sens = {}, {}, {}
         sens_dev = {}
-        # ---------------- pass 1: statistics and sensitivities
-        for b in range(self.n_blocks):
+        # ---------------- pass 1: statistics and sensitivities (this rank's blocks)
+        for b in self.blocks:
             t0 = time.perf_counter()
             inp = self.make_inputs(b, stats_only=True)
             torch.cuda.synchronize()
@@ -115,16 +135,15 @@ class ModelQuantizer:
             del inp
         torch.cuda.synchronize()
         K.check_info(self.info, "model statistics")
+        for k, v in sens_dev.items():
+            sens[k] = v.cpu().tolist()
+        alloc, sens = self.allocate(sens)
         keys = [(b, lin) for b in range(self.n_blocks) for lin in LINEARS]
-        for k in keys:
-            sens[k] = sens_dev[k].cpu().tolist()
-        n_params = [SHAPE[lin][0] * SHAPE[lin][1] for _, lin in keys]
-        bits = K.kq_allocate_bits([sens[k][2] for k in keys], n_params, self.choices, self.avg_bits)
-        alloc = dict(zip(keys, bits))
+        mine = [(b, lin) for b in self.blocks for lin in LINEARS]
 
-        # ---------------- pass 2: BiIP, Cholesky, solver, loss
+        # ---------------- pass 2: BiIP, Cholesky, solver, loss (this rank's blocks)
         results = {}
-        for b in range(self.n_blocks):
+        for b in self.blocks:
             t0 = time.perf_counter()
             inp = self.make_inputs(b, stats_only=False)
             torch.cuda.synchronize()
@@ -172,18 +191,20 @@ class ModelQuantizer:
         for name, e0, e1 in self._events:
             self.phases[name].add(e0, e1)
         total_ms = sum(p.ms for p in self.phases.values())
+        # the job's GPU time is the slowest rank's
+        total_s = D.all_max(total_ms / 1e3, self.dev)
         n_weights = sum(SHAPE[lin][0] * SHAPE[lin][1] for _, lin in keys)
         avg = sum(alloc[k] * SHAPE[k[1]][0] * SHAPE[k[1]][1] for k in keys) / n_weights
         return {
-            "blocks": self.n_blocks, "linears": len(keys), "weights": n_weights,
-            "gpu_seconds": total_ms / 1e3,
-            "weights_per_s": n_weights / (total_ms / 1e3),
+            "blocks": self.n_blocks, "linears": len(keys), "weights": n_weights, "ranks": self.world,
+            "gpu_seconds": total_s,
+            "weights_per_s": n_weights / total_s,
             "phase_seconds": {k: v.ms / 1e3 for k, v in self.phases.items()},
             "input_generation_seconds": self.gen_s,
             "average_bits": avg,
             "bits_histogram": {str(c): sum(1 for k in keys if alloc[k] == c) for c in self.choices},
-            "loss_sum": float(sum(r["loss"].item() for r in results.values())),
+            "loss_sum_this_rank": float(sum(r["loss"].item() for r in results.values())),
             "per_linear": [{"block": b, "linear": lin, "score": sens[(b, lin)][2], "tr_X": sens[(b, lin)][0],
                             "tr_G": sens[(b, lin)][1], "bits": alloc[(b, lin)],
-                            "loss": results[(b, lin)]["loss"].item()} for b, lin in keys],
+                            "loss": results[(b, lin)]["loss"].item()} for b, lin in mine],
         }
