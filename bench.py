@@ -170,11 +170,11 @@ def run_kronq(a):
         mark("rotate")
         lq.factor(0.01)
         mark("chol_inv")
-        for r in results:
-            lq.quantize(r)
-            mark(f"quantize_w{r.bits}")
-            lq.loss(r)
-            mark(f"loss_w{r.bits}")
+        tag = "".join(f"w{r.bits}" for r in results)
+        lq.quantize_all(results)   # every bit-width, one operand split of Uc
+        mark(f"quantize_{tag}")
+        lq.loss_all(results)       # every bit-width, one split of H_X and H_G
+        mark(f"loss_{tag}")
         if timed:
             stage_events.append(marks)
 

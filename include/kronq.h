@@ -226,6 +226,21 @@ kq_status kq_quantize_layer(const float* W, int64_t d_out, int64_t d_in, int64_t
                             float* W_hat, int64_t ldwh,
                             void* ws, size_t ws_bytes, int32_t* info, kq_stream_t stream);
 
+/* kq_quantize_layer_multi - kq_quantize_layer for `count` settings of one
+ * layer (the same W, Uc and dead mask; bit-width bits[i] and group group[i]
+ * into codes[i], scales[i], zeros[i], W_hat[i]), run one after the other on
+ * `stream`.  The 3xTF32 operand split of Uc is formed once for all settings
+ * (KronQ paper page, authors' reply: one set of statistics serves every
+ * bit-width).  The pointer arrays are HOST arrays of device pointers, read
+ * during the call.  Workspace: kq_quantize_layer_workspace_size (the same as
+ * for one setting).  Errors as kq_quantize_layer; count >= 1. */
+kq_status kq_quantize_layer_multi(const float* W, int64_t d_out, int64_t d_in, int64_t ldw,
+                                  const float* Uc, int64_t lduc, const uint8_t* dead_mask,
+                                  int count, const int* bits, const int* group, int block, int gemm_mode,
+                                  uint8_t* const* codes, int64_t ldq, float* const* scales,
+                                  float* const* zeros, float* const* W_hat, int64_t ldwh,
+                                  void* ws, size_t ws_bytes, int32_t* info, kq_stream_t stream);
+
 /* --------------------------------------------------------------------------
  * kq_kron_loss - Kronecker loss (a10).
  *
@@ -244,6 +259,16 @@ kq_status kq_kron_loss(const float* W, int64_t ldw, const float* W_hat, int64_t 
                        int64_t d_out, int64_t d_in,
                        const float* H_X, int64_t ldhx, const float* H_G, int64_t ldhg,
                        double* loss, void* ws, size_t ws_bytes, kq_stream_t stream);
+
+/* kq_kron_loss_multi - kq_kron_loss of `count` dequantized layers W_hat[i]
+ * against one W, H_X and H_G (loss[i], device fp64), run one after the other
+ * on `stream`; the 3xTF32 operand splits of H_X and H_G are formed once.  The
+ * pointer arrays are HOST arrays of device pointers, read during the call.
+ * Workspace: kq_kron_loss_workspace_size.  Errors as kq_kron_loss; count >= 1. */
+kq_status kq_kron_loss_multi(const float* W, int64_t ldw, int count, const float* const* W_hat,
+                             int64_t ldwh, int64_t d_out, int64_t d_in,
+                             const float* H_X, int64_t ldhx, const float* H_G, int64_t ldhg,
+                             double* const* loss, void* ws, size_t ws_bytes, kq_stream_t stream);
 
 /* --------------------------------------------------------------------------
  * kq_kron_loss_noalloc - kq_kron_loss without a caller workspace.

@@ -32,8 +32,8 @@ EXPORTS = (
     "kq_sensitivity",
     "kq_rotate",
     "kq_chol_inv_workspace_size", "kq_chol_inv",
-    "kq_quantize_layer_workspace_size", "kq_quantize_layer",
-    "kq_kron_loss_workspace_size", "kq_kron_loss", "kq_kron_loss_noalloc",
+    "kq_quantize_layer_workspace_size", "kq_quantize_layer", "kq_quantize_layer_multi",
+    "kq_kron_loss_workspace_size", "kq_kron_loss", "kq_kron_loss_multi", "kq_kron_loss_noalloc",
     "kq_allocate_bits",
 )
 
@@ -67,7 +67,13 @@ _SIGS = {
     "kq_quantize_layer_workspace_size": (_sz, [_i64, _i64, _i32]),
     "kq_quantize_layer": (_i32, [_vp, _i64, _i64, _i64, _vp, _i64, _vp, _i32, _i32, _i32, _i32,
                                  _vp, _i64, _vp, _vp, _vp, _i64, _vp, _sz, _vp, _vp]),
+    "kq_quantize_layer_multi": (_i32, [_vp, _i64, _i64, _i64, _vp, _i64, _vp, _i32, ctypes.POINTER(ctypes.c_int),
+                                       ctypes.POINTER(ctypes.c_int), _i32, _i32, ctypes.POINTER(_vp), _i64,
+                                       ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i64, _vp, _sz,
+                                       _vp, _vp]),
     "kq_kron_loss_workspace_size": (_sz, [_i64, _i64]),
+    "kq_kron_loss_multi": (_i32, [_vp, _i64, _i32, ctypes.POINTER(_vp), _i64, _i64, _i64, _vp, _i64, _vp, _i64,
+                                  ctypes.POINTER(_vp), _vp, _sz, _vp]),
     "kq_kron_loss": (_i32, [_vp, _i64, _vp, _i64, _i64, _i64, _vp, _i64, _vp, _i64, _vp, _vp, _sz, _vp]),
     "kq_kron_loss_noalloc": (_i32, [_vp, _i64, _vp, _i64, _i64, _i64, _vp, _i64, _vp, _i64, _vp, _vp]),
     "kq_allocate_bits": (_i32, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), _i32,
@@ -244,6 +250,40 @@ def kq_quantize_layer(W, Uc, dead_mask, bits, group, codes, scales, zeros, W_hat
                                     _ptr(W_hat), ldh, wp, wb, _ptr(info), _stream(stream)), "kq_quantize_layer")
 
 
+def _ptrs(ts):
+    return (_vp * len(ts))(*[t.data_ptr() for t in ts])
+
+
+def kq_quantize_layer_multi(W, Uc, dead_mask, settings, codes, scales, zeros, W_hat, block=128,
+                            gemm_mode=KQ_GEMM_FP32, ws=None, info=None, stream=None):
+    """kq_quantize_layer for several (bits, group) settings of one layer; the
+    output lists hold one tensor per setting (same shapes as for one)."""
+    k = len(settings)
+    if not (k and len(codes) == len(scales) == len(zeros) == len(W_hat) == k):
+        raise ValueError("one codes/scales/zeros/W_hat tensor per setting")
+    ldw = _mat(W, torch.float32, "W")
+    ldu = _mat(Uc, torch.float32, "Uc")
+    ldq = _mat(codes[0], torch.uint8, "codes")
+    ldh = _mat(W_hat[0], torch.float32, "W_hat")
+    d_out, d_in = W.shape
+    for (b, g), c, s_, z, wh in zip(settings, codes, scales, zeros, W_hat):
+        ng = 1 if not g else -(-d_in // g)
+        if _mat(c, torch.uint8, "codes") != ldq or _mat(wh, torch.float32, "W_hat") != ldh:
+            raise ValueError("every codes / W_hat tensor needs the same leading dimension")
+        for t, nm in ((s_, "scales"), (z, "zeros")):
+            if t.dtype != torch.float32 or not t.is_contiguous() or t.numel() < d_out * ng:
+                raise TypeError(f"{nm} must be contiguous float32 [d_out, n_groups]")
+    if ws is None:
+        ws = workspace(kq_quantize_layer_workspace_size(d_out, d_in, block), W.device)
+    wp, wb = _buf(ws)
+    bits = (ctypes.c_int * k)(*[int(b) for b, _ in settings])
+    groups = (ctypes.c_int * k)(*[int(g) for _, g in settings])
+    _check(load().kq_quantize_layer_multi(_ptr(W), d_out, d_in, ldw, _ptr(Uc), ldu, _ptr(dead_mask), k, bits, groups,
+                                          int(block), int(gemm_mode), _ptrs(codes), ldq, _ptrs(scales), _ptrs(zeros),
+                                          _ptrs(W_hat), ldh, wp, wb, _ptr(info), _stream(stream)),
+           "kq_quantize_layer_multi")
+
+
 def kq_kron_loss_workspace_size(d_out: int, d_in: int) -> int:
     return int(load().kq_kron_loss_workspace_size(int(d_out), int(d_in)))
 
@@ -261,6 +301,28 @@ def kq_kron_loss(W, W_hat, H_X, H_G, loss, ws=None, stream=None):
     wp, wb = _buf(ws)
     _check(load().kq_kron_loss(_ptr(W), ldw, _ptr(W_hat), ldh, d_out, d_in, _ptr(H_X), ldx, _ptr(H_G), ldg,
                                _ptr(loss), wp, wb, _stream(stream)), "kq_kron_loss")
+
+
+def kq_kron_loss_multi(W, W_hats, H_X, H_G, losses, ws=None, stream=None):
+    """kq_kron_loss of several dequantized layers against one W, H_X, H_G."""
+    k = len(W_hats)
+    if not (k and len(losses) == k):
+        raise ValueError("one loss tensor per W_hat")
+    ldw = _mat(W, torch.float32, "W")
+    ldh = _mat(W_hats[0], torch.float32, "W_hat")
+    for wh, l in zip(W_hats, losses):
+        if _mat(wh, torch.float32, "W_hat") != ldh:
+            raise ValueError("every W_hat needs the same leading dimension")
+        if l.dtype != torch.float64 or not l.is_cuda:
+            raise TypeError("loss must be a CUDA float64 tensor")
+    ldx = _mat(H_X, torch.float32, "H_X")
+    ldg = 0 if H_G is None else _mat(H_G, torch.float32, "H_G")
+    d_out, d_in = W.shape
+    if ws is None:
+        ws = workspace(kq_kron_loss_workspace_size(d_out, d_in), W.device)
+    wp, wb = _buf(ws)
+    _check(load().kq_kron_loss_multi(_ptr(W), ldw, k, _ptrs(W_hats), ldh, d_out, d_in, _ptr(H_X), ldx, _ptr(H_G), ldg,
+                                     _ptrs(losses), wp, wb, _stream(stream)), "kq_kron_loss_multi")
 
 
 def kq_kron_loss_noalloc(W, W_hat, H_X, H_G, loss, stream=None):

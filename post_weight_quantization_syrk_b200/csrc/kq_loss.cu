@@ -186,9 +186,13 @@ extern "C" size_t kq_kron_loss_workspace_size(int64_t d_out, int64_t d_in) {
   return loss_layout(d_out, d_in, nullptr, nullptr);
 }
 
-extern "C" kq_status kq_kron_loss(const float* W, int64_t ldw, const float* W_hat, int64_t ldwh, int64_t d_out,
-                                  int64_t d_in, const float* H_X, int64_t ldhx, const float* H_G, int64_t ldhg,
-                                  double* loss, void* ws, size_t ws_bytes, kq_stream_t stream) {
+namespace {
+
+// One loss; the tf32 splits of H_X and H_G are formed here unless `split_h`
+// is false (then they are already in the workspace from an earlier call).
+kq_status kron_loss_impl(const float* W, int64_t ldw, const float* W_hat, int64_t ldwh, int64_t d_out, int64_t d_in,
+                         const float* H_X, int64_t ldhx, const float* H_G, int64_t ldhg, double* loss, void* ws,
+                         size_t ws_bytes, kq_stream_t stream, bool split_h) {
   if (!W || !W_hat || !H_X || !loss) return kq::fail(KQ_ERR_INVALID_ARG, "kq_kron_loss: NULL pointer");
   if (d_out < 1 || d_in < 1) return kq::fail(KQ_ERR_INVALID_ARG, "kq_kron_loss: sizes must be >= 1");
   if (d_out > 65536 || d_in > 65536) return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_kron_loss: sizes above 65536");
@@ -200,7 +204,7 @@ extern "C" kq_status kq_kron_loss(const float* W, int64_t ldw, const float* W_ha
   LossWs w;
   loss_layout(d_out, d_in, &w, ws);
   KQ_TRY(kq::split_tf32(W, ldw, W_hat, ldwh, d_out, d_in, w.Db, w.Ds, w.ldd, false, st));
-  KQ_TRY(kq::split_tf32(H_X, ldhx, nullptr, 0, d_in, d_in, w.Xb, w.Xs, w.ldx, true, st));
+  if (split_h) KQ_TRY(kq::split_tf32(H_X, ldhx, nullptr, 0, d_in, d_in, w.Xb, w.Xs, w.ldx, true, st));
   kq::Gemm3xTF32 g1;                 // A1 = dW H_X   (B^T = H_X^T)
   g1.M = d_out;
   g1.N = d_in;
@@ -218,7 +222,7 @@ extern "C" kq_status kq_kron_loss(const float* W, int64_t ldw, const float* W_ha
   int64_t np;
   if (H_G) {
     KQ_TRY(kq::split_tf32(W, ldw, W_hat, ldwh, d_out, d_in, w.Dtb, w.Dts, w.ldt, true, st));
-    KQ_TRY(kq::split_tf32(H_G, ldhg, nullptr, 0, d_out, d_out, w.Gb, w.Gs, w.ldg, false, st));
+    if (split_h) KQ_TRY(kq::split_tf32(H_G, ldhg, nullptr, 0, d_out, d_out, w.Gb, w.Gs, w.ldg, false, st));
     kq::Gemm3xTF32 g2;               // sum (H_G dW) .* A1   (B^T = dW^T)
     g2.M = d_out;
     g2.N = d_in;
@@ -243,6 +247,27 @@ extern "C" kq_status kq_kron_loss(const float* W, int64_t ldw, const float* W_ha
   sum_kernel<<<1, 1024, 0, st>>>(w.partial, np, loss);
   KQ_TRY(kq::launch_check("kq_kron_loss sum"));
   kq::clear_error();
+  return KQ_OK;
+}
+
+}  // namespace
+
+extern "C" kq_status kq_kron_loss(const float* W, int64_t ldw, const float* W_hat, int64_t ldwh, int64_t d_out,
+                                  int64_t d_in, const float* H_X, int64_t ldhx, const float* H_G, int64_t ldhg,
+                                  double* loss, void* ws, size_t ws_bytes, kq_stream_t stream) {
+  return kron_loss_impl(W, ldw, W_hat, ldwh, d_out, d_in, H_X, ldhx, H_G, ldhg, loss, ws, ws_bytes, stream, true);
+}
+
+extern "C" kq_status kq_kron_loss_multi(const float* W, int64_t ldw, int count, const float* const* W_hat,
+                                        int64_t ldwh, int64_t d_out, int64_t d_in, const float* H_X, int64_t ldhx,
+                                        const float* H_G, int64_t ldhg, double* const* loss, void* ws,
+                                        size_t ws_bytes, kq_stream_t stream) {
+  if (count < 1 || !W_hat || !loss) return kq::fail(KQ_ERR_INVALID_ARG, "kq_kron_loss_multi: count < 1 or NULL array");
+  for (int i = 0; i < count; ++i)
+    if (!W_hat[i] || !loss[i]) return kq::fail(KQ_ERR_INVALID_ARG, "kq_kron_loss_multi: NULL W_hat or loss entry");
+  for (int i = 0; i < count; ++i)
+    KQ_TRY(kron_loss_impl(W, ldw, W_hat[i], ldwh, d_out, d_in, H_X, ldhx, H_G, ldhg, loss[i], ws, ws_bytes, stream,
+                          i == 0));
   return KQ_OK;
 }
 

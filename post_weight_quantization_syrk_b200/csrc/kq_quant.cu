@@ -397,11 +397,15 @@ extern "C" size_t kq_quantize_layer_workspace_size(int64_t d_out, int64_t d_in, 
   return quant_layout(d_out, d_in, nullptr, nullptr);
 }
 
-extern "C" kq_status kq_quantize_layer(const float* W, int64_t d_out, int64_t d_in, int64_t ldw, const float* Uc,
-                                       int64_t lduc, const uint8_t* dead_mask, int bits, int group, int block,
-                                       int gemm_mode, uint8_t* codes, int64_t ldq, float* scales, float* zeros,
-                                       float* W_hat, int64_t ldwh, void* ws, size_t ws_bytes, int32_t* info,
-                                       kq_stream_t stream) {
+namespace {
+
+// One setting; the tf32 split of Uc^T (3xTF32 mode) is formed here unless
+// `split_uc` is false (then it is already in the workspace from an earlier
+// call with the same Uc).
+kq_status quantize_impl(const float* W, int64_t d_out, int64_t d_in, int64_t ldw, const float* Uc, int64_t lduc,
+                        const uint8_t* dead_mask, int bits, int group, int block, int gemm_mode, uint8_t* codes,
+                        int64_t ldq, float* scales, float* zeros, float* W_hat, int64_t ldwh, void* ws,
+                        size_t ws_bytes, int32_t* info, kq_stream_t stream, bool split_uc) {
   if (!W || !Uc || !codes || !scales || !zeros || !W_hat || !info)
     return kq::fail(KQ_ERR_INVALID_ARG, "kq_quantize_layer: NULL pointer");
   if (d_out < 1 || d_in < 1 || d_in > 65536) return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_quantize_layer: sizes");
@@ -423,7 +427,7 @@ extern "C" kq_status kq_quantize_layer(const float* W, int64_t d_out, int64_t d_
   QuantWs w;
   quant_layout(d_out, d_in, &w, ws);
   const bool tc = (gemm_mode == KQ_GEMM_3XTF32);
-  if (tc) KQ_TRY(kq::split_tf32(Uc, lduc, nullptr, 0, d_in, d_in, w.Ub, w.Us, w.ldu, true, st));
+  if (tc && split_uc) KQ_TRY(kq::split_tf32(Uc, lduc, nullptr, 0, d_in, d_in, w.Ub, w.Us, w.ldu, true, st));
 
   const float nl = (float)((1 << bits) - 1);
   const int64_t n_groups = group ? kq::cdiv(d_in, group) : 1;
@@ -516,5 +520,30 @@ extern "C" kq_status kq_quantize_layer(const float* W, int64_t d_out, int64_t d_
     }
   }
   kq::clear_error();
+  return KQ_OK;
+}
+
+}  // namespace
+
+extern "C" kq_status kq_quantize_layer(const float* W, int64_t d_out, int64_t d_in, int64_t ldw, const float* Uc,
+                                       int64_t lduc, const uint8_t* dead_mask, int bits, int group, int block,
+                                       int gemm_mode, uint8_t* codes, int64_t ldq, float* scales, float* zeros,
+                                       float* W_hat, int64_t ldwh, void* ws, size_t ws_bytes, int32_t* info,
+                                       kq_stream_t stream) {
+  return quantize_impl(W, d_out, d_in, ldw, Uc, lduc, dead_mask, bits, group, block, gemm_mode, codes, ldq, scales,
+                       zeros, W_hat, ldwh, ws, ws_bytes, info, stream, true);
+}
+
+extern "C" kq_status kq_quantize_layer_multi(const float* W, int64_t d_out, int64_t d_in, int64_t ldw,
+                                             const float* Uc, int64_t lduc, const uint8_t* dead_mask, int count,
+                                             const int* bits, const int* group, int block, int gemm_mode,
+                                             uint8_t* const* codes, int64_t ldq, float* const* scales,
+                                             float* const* zeros, float* const* W_hat, int64_t ldwh, void* ws,
+                                             size_t ws_bytes, int32_t* info, kq_stream_t stream) {
+  if (count < 1 || !bits || !group || !codes || !scales || !zeros || !W_hat)
+    return kq::fail(KQ_ERR_INVALID_ARG, "kq_quantize_layer_multi: count < 1 or NULL array");
+  for (int i = 0; i < count; ++i)
+    KQ_TRY(quantize_impl(W, d_out, d_in, ldw, Uc, lduc, dead_mask, bits[i], group[i], block, gemm_mode, codes[i], ldq,
+                         scales[i], zeros[i], W_hat[i], ldwh, ws, ws_bytes, info, stream, i == 0));
   return KQ_OK;
 }

@@ -100,6 +100,20 @@ class LayerQuantizer:
         ws = self.workspace(K.kq_kron_loss_workspace_size(self.d_out, self.d_in))
         K.kq_kron_loss(self.Wp, res.W_hat, self.H_X, self.H_G, res.loss, ws, stream)
 
+    def quantize_all(self, results, stream=None):
+        """Every setting of `results` in one call (the factor's operand split is shared)."""
+        ws = self.workspace(K.kq_quantize_layer_workspace_size(self.d_out, self.d_in, self.block))
+        K.kq_quantize_layer_multi(self.Wp, self.Uc, self.dead, [(r.bits, r.group) for r in results],
+                                  [r.codes for r in results], [r.scales for r in results],
+                                  [r.zeros for r in results], [r.W_hat for r in results], self.block,
+                                  self.gemm_mode, ws, self.info, stream)
+
+    def loss_all(self, results, stream=None):
+        """Every result's Kronecker loss in one call (the H_X, H_G splits are shared)."""
+        ws = self.workspace(K.kq_kron_loss_workspace_size(self.d_out, self.d_in))
+        K.kq_kron_loss_multi(self.Wp, [r.W_hat for r in results], self.H_X, self.H_G, [r.loss for r in results], ws,
+                             stream)
+
     def run(self, W, X, G, T_in, T_out, settings, damp_frac=0.01, results=None, stream=None):
         """The whole path; settings = [(bits, group), ...].  Asynchronous."""
         self.statistics(X, G, stream=stream)
@@ -108,9 +122,8 @@ class LayerQuantizer:
         self.factor(damp_frac, stream)
         if results is None:
             results = [self.alloc_result(b, g) for b, g in settings]
-        for r in results:
-            self.quantize(r, stream)
-            self.loss(r, stream)
+        self.quantize_all(results, stream)
+        self.loss_all(results, stream)
         return results
 
     def check(self, where="kronq"):

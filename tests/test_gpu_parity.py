@@ -398,3 +398,36 @@ def test_layer512_whole_path_stagewise(P):
     # loss agrees to the statistical level the fp32 covariances allow
     full = O.quantize_linear(W.double().numpy(), Xn, Gn, Tin, Tout, 3)
     assert abs(r.loss.item() - full["loss"]) <= 0.05 * full["loss"]
+
+
+# ------------------------------------------------------------------ multi-setting entry points
+
+def test_multi_entry_points_match_single_calls(P, rotated_small):
+    """kq_quantize_layer_multi / kq_kron_loss_multi share the operand splits
+    across settings and must return exactly what the single calls return."""
+    lq = rotated_small[0]
+    settings = [(4, 0), (3, 128), (2, 0)]
+    d_out, d_in = lq.Wp.shape
+
+    def outputs():
+        res = []
+        for b, g in settings:
+            ng = 1 if not g else -(-d_in // g)
+            res.append((torch.empty((d_out, d_in), dtype=torch.uint8, device="cuda"),
+                        torch.empty((d_out, ng), device="cuda"), torch.empty((d_out, ng), device="cuda"),
+                        torch.empty((d_out, d_in), device="cuda"), torch.zeros(1, dtype=torch.float64, device="cuda")))
+        return res
+
+    one, many = outputs(), outputs()
+    info = _info()
+    for (b, g), (c, s, z, wh, l) in zip(settings, one):
+        P.kq_quantize_layer(lq.Wp, lq.Uc, lq.dead, b, g, c, s, z, wh, gemm_mode=P.KQ_GEMM_3XTF32, info=info)
+        P.kq_kron_loss(lq.Wp, wh, lq.H_X, lq.H_G, l)
+    P.kq_quantize_layer_multi(lq.Wp, lq.Uc, lq.dead, settings, [o[0] for o in many], [o[1] for o in many],
+                              [o[2] for o in many], [o[3] for o in many], gemm_mode=P.KQ_GEMM_3XTF32, info=info)
+    P.kq_kron_loss_multi(lq.Wp, [o[3] for o in many], lq.H_X, lq.H_G, [o[4] for o in many])
+    torch.cuda.synchronize()
+    assert _info_code(info)[0] == 0
+    for a, b in zip(one, many):
+        for x, y in zip(a, b):
+            assert torch.equal(x, y)
