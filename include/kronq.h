@@ -233,7 +233,8 @@ kq_status kq_quantize_layer(const float* W, int64_t d_out, int64_t d_in, int64_t
  * (KronQ paper page, authors' reply: one set of statistics serves every
  * bit-width).  The pointer arrays are HOST arrays of device pointers, read
  * during the call.  Workspace: kq_quantize_layer_workspace_size (the same as
- * for one setting).  Errors as kq_quantize_layer; count >= 1. */
+ * for one setting).  Errors as kq_quantize_layer; count >= 1; every setting
+ * is validated before any work is enqueued. */
 kq_status kq_quantize_layer_multi(const float* W, int64_t d_out, int64_t d_in, int64_t ldw,
                                   const float* Uc, int64_t lduc, const uint8_t* dead_mask,
                                   int count, const int* bits, const int* group, int block, int gemm_mode,

@@ -542,6 +542,16 @@ extern "C" kq_status kq_quantize_layer_multi(const float* W, int64_t d_out, int6
                                              size_t ws_bytes, int32_t* info, kq_stream_t stream) {
   if (count < 1 || !bits || !group || !codes || !scales || !zeros || !W_hat)
     return kq::fail(KQ_ERR_INVALID_ARG, "kq_quantize_layer_multi: count < 1 or NULL array");
+  // every setting is checked before any work is enqueued
+  for (int i = 0; i < count; ++i) {
+    if (!codes[i] || !scales[i] || !zeros[i] || !W_hat[i])
+      return kq::fail(KQ_ERR_INVALID_ARG, "kq_quantize_layer_multi: NULL output of setting %d", i);
+    if (bits[i] < 2 || bits[i] > 8) return kq::fail(KQ_ERR_INVALID_ARG, "kq_quantize_layer_multi: bits outside 2..8");
+    if (group[i] < 0 || (group[i] && (group[i] % 32 || BLK % group[i])))
+      return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE,
+                      "kq_quantize_layer_multi: group must be 0 or a multiple of 32 dividing 128");
+    if (W == W_hat[i]) return kq::fail(KQ_ERR_INVALID_ARG, "kq_quantize_layer_multi: W and W_hat must not alias");
+  }
   for (int i = 0; i < count; ++i)
     KQ_TRY(quantize_impl(W, d_out, d_in, ldw, Uc, lduc, dead_mask, bits[i], group[i], block, gemm_mode, codes[i], ldq,
                          scales[i], zeros[i], W_hat[i], ldwh, ws, ws_bytes, info, stream, i == 0));

@@ -138,3 +138,19 @@ def test_workspace_sizes():
     assert P.kq_quantize_layer_workspace_size(4096, 4096) >= 4096 * 128 * 4
     assert P.kq_kron_loss_workspace_size(4096, 4096) >= 64 * 64 * 8
     assert P.kq_chol_inv_workspace_size(0) == 0
+
+
+def test_multi_entry_points_validate_before_enqueue():
+    """Host-side rejections of the multi-setting calls (no device work)."""
+    import ctypes
+    lib = P.load()
+    vp = ctypes.c_void_p
+    dummy = vp(16)  # never dereferenced: validation fails first
+    arr = (vp * 2)(dummy, dummy)
+    bits = (ctypes.c_int * 2)(3, 9)          # second setting invalid
+    groups = (ctypes.c_int * 2)(0, 0)
+    st = lib.kq_quantize_layer_multi(dummy, 4, 128, 128, dummy, 128, None, 2, bits, groups, 128, 0, arr, 128, arr,
+                                     arr, arr, 128, dummy, 1 << 30, dummy, None)
+    assert st == 1 and b"bits" in lib.kq_last_error()   # KQ_ERR_INVALID_ARG
+    st = lib.kq_kron_loss_multi(dummy, 128, 0, arr, 128, 4, 128, dummy, 128, dummy, 4, arr, dummy, 1 << 30, None)
+    assert st == 1   # KQ_ERR_INVALID_ARG
