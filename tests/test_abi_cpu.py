@@ -146,7 +146,7 @@ def test_multi_entry_points_validate_before_enqueue():
     lib = P.load()
     vp = ctypes.c_void_p
     dummy = vp(16)  # never dereferenced: validation fails first
-    arr = (vp * 2)(dummy, dummy)
+    arr = (vp * 2)(vp(32), vp(48))
     bits = (ctypes.c_int * 2)(3, 9)          # second setting invalid
     groups = (ctypes.c_int * 2)(0, 0)
     st = lib.kq_quantize_layer_multi(dummy, 4, 128, 128, dummy, 128, None, 2, bits, groups, 128, 0, arr, 128, arr,
