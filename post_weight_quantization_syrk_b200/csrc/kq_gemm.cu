@@ -17,7 +17,8 @@
 // last partial wave dominate).  Warp 0 streams 16-deep K slices of A and B (both
 // K-major, 64-byte swizzle; tcgen05 kind::tf32 produced no result with an
 // MN-major operand on B200 when measured, so callers pass B transposed), big
-// and small parts, through a 3-stage ring; one thread of warp 1 issues 12
+// and small parts, through a ring of 3 stages (wide tiles, 64 KB each) or 4
+// stages (narrow tiles, 48 KB each); one thread of warp 1 issues 12
 // tcgen05.mma kind::tf32 per stage; warps 2-9 run the epilogue from TMEM.
 // Waits are time-bounded.
 #include <cuda.h>
@@ -35,8 +36,12 @@ using namespace kq::tc;
 constexpr int BM = 256, BN = 256, BKF = 16;         // tile rows, cols, K per stage (fp32)
 constexpr int A_BYTES = BM * BKF * 4;               // 16 KB per part
 constexpr int B_BYTES = BN * BKF * 4;               // 16 KB per part
-constexpr int STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;
+constexpr int STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;   // wide tiles: 3 stages of 64 KB
 constexpr int STAGES = 3;
+constexpr int NARROW_STAGE_BYTES = A_BYTES + 2 * B_BYTES; // narrow tiles: 4 stages of 48 KB
+constexpr int NARROW_STAGES = 4;
+constexpr int MAX_STAGES = 4;
+static_assert(NARROW_STAGES * NARROW_STAGE_BYTES <= STAGES * STAGE_BYTES, "ring size");
 constexpr int THREADS = 320;                        // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 constexpr int kMaxSms = 148;   // SMs of a B200
@@ -72,17 +77,21 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
   constexpr uint32_t IDESC = idesc(kFmtTF32, /*A K-major*/ 0, /*B K-major*/ 0, 128, 256);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // ring: wide tiles 3 stages of 64 KB, narrow tiles 4 stages of 48 KB
+  const int nstages = p.wide ? STAGES : NARROW_STAGES;
+  const int sbytes = p.wide ? STAGE_BYTES : NARROW_STAGE_BYTES;
+  const int apart = p.wide ? A_BYTES : A_BYTES / 2;   // bytes of one A part in a stage
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * MAX_STAGES + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES);
-  const uint32_t accfull0 = smem_u32(bars + 2 * STAGES), accempty0 = smem_u32(bars + 2 * STAGES + 2);
-  const uint32_t drained = smem_u32(bars + 2 * STAGES + 4);
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + MAX_STAGES);
+  const uint32_t accfull0 = smem_u32(bars + 2 * MAX_STAGES), accempty0 = smem_u32(bars + 2 * MAX_STAGES + 2);
+  const uint32_t drained = smem_u32(bars + 2 * MAX_STAGES + 4);
   const int bm = p.wide ? 256 : 128;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < MAX_STAGES; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
@@ -108,8 +117,8 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t issued_phase[STAGES];
-      bool issued[STAGES] = {false, false, false};
+      uint32_t issued_phase[MAX_STAGES];
+      bool issued[MAX_STAGES] = {false, false, false, false};
       bool ok = true;
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
         const int m0 = (t / p.tiles_n) * bm, n0 = (t % p.tiles_n) * BN;
@@ -119,26 +128,26 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
             break;
           }
           const uint32_t fb = full0 + 8 * stage;
-          mbar_arrive_expect_tx(fb, p.wide ? STAGE_BYTES : STAGE_BYTES - A_BYTES);
-          const uint32_t s0 = smem_u32(smem + stage * STAGE_BYTES);
+          mbar_arrive_expect_tx(fb, sbytes);
+          const uint32_t s0 = smem_u32(smem + stage * sbytes);
           const int k0 = kb * BKF;
           // A boxes are 128 rows; a wide tile takes two per part
           for (int h = 0; h <= p.wide; ++h) {
             tma_load_2d(s0 + h * (A_BYTES / 2), &maps.ab, p.a_x0 + k0, p.a_y0 + m0 + 128 * h, fb);
-            tma_load_2d(s0 + A_BYTES + h * (A_BYTES / 2), &maps.as, p.a_x0 + k0, p.a_y0 + m0 + 128 * h, fb);
+            tma_load_2d(s0 + apart + h * (A_BYTES / 2), &maps.as, p.a_x0 + k0, p.a_y0 + m0 + 128 * h, fb);
           }
-          tma_load_2d(s0 + 2 * A_BYTES, &maps.bb, p.b_x0 + k0, p.b_y0 + n0, fb);
-          tma_load_2d(s0 + 2 * A_BYTES + B_BYTES, &maps.bs, p.b_x0 + k0, p.b_y0 + n0, fb);
+          tma_load_2d(s0 + 2 * apart, &maps.bb, p.b_x0 + k0, p.b_y0 + n0, fb);
+          tma_load_2d(s0 + 2 * apart + B_BYTES, &maps.bs, p.b_x0 + k0, p.b_y0 + n0, fb);
           issued[stage] = true;
           issued_phase[stage] = phase;
-          if (++stage == STAGES) {
+          if (++stage == nstages) {
             stage = 0;
             phase ^= 1u;
           }
         }
       }
       if (!ok)
-        for (int s = 0; s < STAGES; ++s)
+        for (int s = 0; s < nstages; ++s)
           if (issued[s]) mbar_drain(full0 + 8 * s, issued_phase[s]);
     }
   } else if (warp == 1) {
@@ -157,8 +166,8 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
             break;
           }
           fence_after();
-          const uint32_t s0 = smem_u32(smem + stage * STAGE_BYTES);
-          const uint32_t ab = s0, as = s0 + A_BYTES, bb = s0 + 2 * A_BYTES, bs = bb + B_BYTES;
+          const uint32_t s0 = smem_u32(smem + stage * sbytes);
+          const uint32_t ab = s0, as = s0 + apart, bb = s0 + 2 * apart, bs = bb + B_BYTES;
 #pragma unroll
           for (int ks = 0; ks < BKF / 8; ++ks) {
             const uint64_t dbb = desc_op(bb + ks * 32), dbs = desc_op(bs + ks * 32);
@@ -174,7 +183,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
           }
           any = true;
           mma_commit(empty0 + 8 * stage);
-          if (++stage == STAGES) {
+          if (++stage == nstages) {
             stage = 0;
             phase ^= 1u;
           }
