@@ -248,10 +248,17 @@ kq_status kq_quantize_layer_multi(const float* W, int64_t d_out, int64_t d_in, i
  * loss = tr(dW H_X dW^T H_G), dW = W - W_hat (KronQ review, Background: the
  * layer Hessian H ~ H_X kron H_G; Unified Hessian-Guided PTQ, Appendix A.1:
  * the Kronecker-weighted norm as a trace).  H_G == NULL means the identity
- * (the H_X-only GPTQ objective).  Products on the tensor cores in 3xTF32
- * (fp32-level accuracy), elementwise products and sums in fp64.
+ * (the H_X-only GPTQ objective).  Evaluated as the Frobenius product of the
+ * larger Hessian H2 with P = D H1^T D^T, H1 the smaller Hessian and D = dW or
+ * dW^T (P = dW^T dW when H_G == NULL), P formed only in its upper block
+ * triangle: d_out d_in (min + max/2) multiply-adds.  Products on the tensor
+ * cores in 3xTF32 (fp32-level accuracy), elementwise products and sums in
+ * fp64.
  *
  *   W, W_hat fp32 [d_out, d_in];  H_X fp32 [d_in, d_in];  H_G fp32 [d_out, d_out].
+ *   H_X, H_G symmetric (as covariances are): of the larger one only the
+ *            256 x 256 blocks on and above the block diagonal are read, and
+ *            the result is the loss of the symmetric matrix they define.
  *   loss     device fp64[1].
  *   ws       kq_kron_loss_workspace_size(d_out, d_in) bytes.
  * ------------------------------------------------------------------------ */
@@ -263,7 +270,7 @@ kq_status kq_kron_loss(const float* W, int64_t ldw, const float* W_hat, int64_t 
 
 /* kq_kron_loss_multi - kq_kron_loss of `count` dequantized layers W_hat[i]
  * against one W, H_X and H_G (loss[i], device fp64), run one after the other
- * on `stream`; the 3xTF32 operand splits of H_X and H_G are formed once.  The
+ * on `stream`; the 3xTF32 operand split of the smaller Hessian is formed once.  The
  * pointer arrays are HOST arrays of device pointers, read during the call.
  * Workspace: kq_kron_loss_workspace_size.  Errors as kq_kron_loss; count >= 1. */
 kq_status kq_kron_loss_multi(const float* W, int64_t ldw, int count, const float* const* W_hat,
@@ -278,9 +285,10 @@ kq_status kq_kron_loss_multi(const float* W, int64_t ldw, int count, const float
  * that cannot allocate device memory: code embedded in a host application
  * that owns every device allocation through its own pool, or a latency-bound
  * loop where the implicit synchronisation of cudaMalloc/cudaFree is not
- * acceptable.  It computes the same loss with the same kernels as
- * kq_kron_loss, but keeps the per-tile partial sums in a fixed array inside
- * the library (static device memory: KQ_KRON_LOSS_NOALLOC_MAX_TILES fp64
+ * acceptable.  It computes the same loss (all of H_X and H_G read, no
+ * symmetry assumed) with an fp32 CUDA-core kernel that forms one 64 x 64 tile
+ * of dW H_X and of H_G dW per CTA, and keeps the per-tile partial sums in a
+ * fixed array inside the library (static device memory: KQ_KRON_LOSS_NOALLOC_MAX_TILES fp64
  * values, 512 KiB, held by every GPU that loads the library until the
  * process exits).  It calls no cudaMalloc, cudaFree or allocating routine.
  *

@@ -49,16 +49,19 @@ constexpr int kMaxSms = 148;   // SMs of a B200
 struct Params {
   int64_t M, N, K;
   int wide;   // 1: 256 x 256 tiles, 0: 128 x 256 tiles
+  int upper;  // 1: upper block triangle only (M == N), off-diagonal partials doubled
   int tiles_m, tiles_n, num_tiles, kblocks;
   int a_x0, a_y0, b_x0, b_y0;   // tensor-map coordinates of A(0,0) and B(0,0)
   int epilogue;
   float* C;
+  float* C_small;
   int64_t ldc;
   const float* src;
   int64_t ld_src;
   const uint8_t* dead;
   const float* other;
   int64_t ld_other;
+  int other_vec;   // `other` rows can be read as float4 (16-byte aligned rows)
   double* partial;
   int32_t* info;
 };
@@ -72,6 +75,34 @@ __device__ __forceinline__ uint64_t desc_op(uint32_t addr) { return smem_desc(ad
 struct Maps {
   CUtensorMap ab, as, bb, bs;
 };
+
+// Tile t -> (row tile, column tile).  Row tile tm holds tiles_n - rb(tm)
+// tiles, rb(tm) = 0, or in the upper block triangle the 256-column block of
+// its first row; tiles are numbered row by row.  A role visits its tiles in
+// increasing t, so the walk resumes where the last call stopped.
+struct TileWalk {
+  int tm = 0, base = 0;
+  __device__ __forceinline__ void at(const Params& p, int bm, int t, int& tm_out, int& tn_out, int& rb_out) {
+    for (;;) {
+      const int rb = p.upper ? (tm * bm) / BN : 0;
+      const int cnt = p.tiles_n - rb;
+      if (t < base + cnt || tm + 1 >= p.tiles_m) {
+        tm_out = tm;
+        tn_out = rb + (t - base);
+        rb_out = rb;
+        return;
+      }
+      base += cnt;
+      ++tm;
+    }
+  }
+};
+
+__device__ __forceinline__ float tf32_round(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
 
 __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant__ Maps maps, Params p) {
   constexpr uint32_t IDESC = idesc(kFmtTF32, /*A K-major*/ 0, /*B K-major*/ 0, 128, 256);
@@ -120,8 +151,11 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       uint32_t issued_phase[MAX_STAGES];
       bool issued[MAX_STAGES] = {false, false, false, false};
       bool ok = true;
+      TileWalk walk;
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
-        const int m0 = (t / p.tiles_n) * bm, n0 = (t % p.tiles_n) * BN;
+        int tm, tn, rb;
+        walk.at(p, bm, t, tm, tn, rb);
+        const int m0 = tm * bm, n0 = tn * BN;
         for (int kb = 0; kb < p.kblocks; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.info, 11)) {
             ok = false;
@@ -207,9 +241,12 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
     const int cbase = (e >> 2) * 128;
     uint32_t acc_bits = 0;   // bit b: phase of accumulator b
     int local = 0;
+    TileWalk walk;
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++local) {
       const int buf = p.wide ? 0 : (local & 1);
-      const int64_t m0 = (int64_t)(t / p.tiles_n) * bm, n0 = (int64_t)(t % p.tiles_n) * BN;
+      int tm, tn, rb;
+      walk.at(p, bm, t, tm, tn, rb);
+      const int64_t m0 = (int64_t)tm * bm, n0 = (int64_t)tn * BN;
       // one lane waits, the warp follows: every lane leaves together on abort
       bool ready = true;
       if (lane == 0) ready = mbar_wait(accfull0 + 8 * buf, (acc_bits >> buf) & 1u, abort_flag, p.info, 14);
@@ -225,9 +262,10 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
         for (int g0 = 0; g0 < 128; g0 += 64) {
           const int64_t gj0 = n0 + cbase + g0;
           const bool any = row_ok && gj0 < p.N;
-          const bool fast = any && gj0 + 64 <= p.N && !(p.epilogue == kEpiSubtract && p.dead);
+          const bool fast = any && gj0 + 64 <= p.N && !(p.epilogue == kEpiSubtract && p.dead) &&
+                            !(p.epilogue == kEpiDot && !p.other_vec);
           float pre[64];
-          if (fast && p.epilogue != kEpiStore) {
+          if (fast && (p.epilogue == kEpiDot || p.epilogue == kEpiSubtract)) {
             const float* sp = (p.epilogue == kEpiDot ? p.other + gi * p.ld_other : p.src + gi * p.ld_src) + gj0;
 #pragma unroll
             for (int q = 0; q < 64; q += 4) {
@@ -248,6 +286,20 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
               if (p.epilogue == kEpiDot) {
 #pragma unroll
                 for (int q = 0; q < 16; ++q) dot += (double)v[q] * (double)pre[cc + q];
+              } else if (p.epilogue == kEpiStoreSplit) {
+                float* c = p.C + gi * p.ldc + gj;
+                float* cs = p.C_small + gi * p.ldc + gj;
+#pragma unroll
+                for (int q = 0; q < 16; q += 4) {
+                  float b[4], r[4];
+#pragma unroll
+                  for (int u = 0; u < 4; ++u) {
+                    b[u] = tf32_round(v[q + u]);
+                    r[u] = v[q + u] - b[u];
+                  }
+                  *reinterpret_cast<float4*>(c + q) = make_float4(b[0], b[1], b[2], b[3]);
+                  *reinterpret_cast<float4*>(cs + q) = make_float4(r[0], r[1], r[2], r[3]);
+                }
               } else {
                 float* c = p.C + gi * p.ldc + gj;
 #pragma unroll
@@ -269,6 +321,10 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
                 } else if (p.epilogue == kEpiSubtract) {
                   const float sv = (p.dead && p.dead[j]) ? 0.f : p.src[gi * p.ld_src + j];
                   p.C[gi * p.ldc + j] = sv - v[q];
+                } else if (p.epilogue == kEpiStoreSplit) {
+                  const float b = tf32_round(v[q]);
+                  p.C[gi * p.ldc + j] = b;
+                  p.C_small[gi * p.ldc + j] = v[q] - b;
                 } else {
                   p.C[gi * p.ldc + j] = v[q];
                 }
@@ -283,6 +339,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
         // fixed-order reduction within the warp (xor butterfly); one partial
         // per (tile, epilogue warp), summed later in index order
         for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        if (p.upper && tn > rb) dot *= 2.0;   // stands for the mirror tile below the diagonal
         if (lane == 0) p.partial[8 * (int64_t)t + e] = dot;
       }
       acc_bits ^= 1u << buf;
@@ -295,12 +352,6 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
     fence_after();
     tmem_dealloc<512>(tmem);
   }
-}
-
-__device__ __forceinline__ float tf32_round(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return __uint_as_float(r);
 }
 
 // big = tf32(x - y), small = (x - y) - big at (r, c), or at (c, r) when
@@ -348,15 +399,28 @@ __global__ void __launch_bounds__(256) split_kernel(const float* __restrict__ x,
 // un-overlapped epilogue is a small share of a tile (measured on B200: the
 // 4096^3 products of the loss run 15 % faster wide, the solver's K <= 1024
 // updates 20 % faster narrow).
-bool gemm_wide(int64_t M, int64_t N, int64_t K) {
-  return cdiv(M, BM) * cdiv(N, BN) >= 2 * kMaxSms || K >= 2048;
+namespace {
+
+// Tiles of an M x N product with bm-row tiles; the same count as TileWalk.
+int64_t tile_count(int64_t M, int64_t N, int bm, bool upper) {
+  const int64_t tm = cdiv(M, bm), tn = cdiv(N, BN);
+  if (!upper) return tm * tn;
+  int64_t c = 0;
+  for (int64_t r = 0; r < tm; ++r) c += tn - (r * bm) / BN;
+  return c;
 }
 
-int64_t gemm_tiles(int64_t M, int64_t N, int64_t K) {
-  return cdiv(M, gemm_wide(M, N, K) ? BM : BM / 2) * cdiv(N, BN);
+bool gemm_wide(int64_t M, int64_t N, int64_t K, bool upper) {
+  return tile_count(M, N, BM, upper) >= 2 * kMaxSms || K >= 2048;
 }
 
-int64_t gemm_tiles_max(int64_t M, int64_t N) { return cdiv(M, BM / 2) * cdiv(N, BN); }
+}  // namespace
+
+int64_t gemm_tiles(int64_t M, int64_t N, int64_t K, bool upper) {
+  return tile_count(M, N, gemm_wide(M, N, K, upper) ? BM : BM / 2, upper);
+}
+
+int64_t gemm_tiles_max(int64_t M, int64_t N, bool upper) { return tile_count(M, N, BM / 2, upper); }
 
 kq_status split_tf32(const float* x, int64_t ldx, const float* y, int64_t ldy, int64_t rows, int64_t cols, float* big,
                      float* small, int64_t ldo, bool transpose, cudaStream_t st) {
@@ -393,10 +457,13 @@ kq_status gemm_3xtf32(const Gemm3xTF32& g, cudaStream_t st) {
   p.M = g.M;
   p.N = g.N;
   p.K = g.K;
-  p.wide = gemm_wide(g.M, g.N, g.K) ? 1 : 0;
+  p.wide = gemm_wide(g.M, g.N, g.K, g.upper) ? 1 : 0;
+  p.upper = g.upper ? 1 : 0;
   p.tiles_m = (int)cdiv(g.M, p.wide ? BM : BM / 2);
   p.tiles_n = (int)cdiv(g.N, BN);
-  p.num_tiles = p.tiles_m * p.tiles_n;
+  const int64_t tiles = tile_count(g.M, g.N, p.wide ? BM : BM / 2, g.upper);
+  if (tiles > 0x7fffffff) return fail(KQ_ERR_UNSUPPORTED_SHAPE, "gemm: too many tiles");
+  p.num_tiles = (int)tiles;
   p.kblocks = (int)cdiv(g.K, BKF);
   p.a_x0 = (int)g.a_col0;
   p.a_y0 = (int)g.a_row0;
@@ -404,19 +471,24 @@ kq_status gemm_3xtf32(const Gemm3xTF32& g, cudaStream_t st) {
   p.b_y0 = (int)g.bt_row0;
   p.epilogue = g.epilogue;
   p.C = g.C;
+  p.C_small = g.C_small;
   p.ldc = g.ldc;
   p.src = g.src;
   p.ld_src = g.ld_src;
   p.dead = g.dead;
   p.other = g.other;
   p.ld_other = g.ld_other;
+  p.other_vec = (g.other && aligned(g.other, 16) && !(g.ld_other & 3)) ? 1 : 0;
   p.partial = g.partial;
   p.info = g.info;
+  if (g.upper && (g.M != g.N || g.epilogue != kEpiDot))
+    return fail(KQ_ERR_INVALID_ARG, "gemm: the upper block triangle needs M == N and the dot epilogue");
   if (g.epilogue == kEpiDot) {
-    if (!g.other || !g.partial || !aligned(g.other, 16) || (g.ld_other & 3))
-      return fail(KQ_ERR_ALIGNMENT, "gemm: dot epilogue needs an aligned `other` and `partial`");
+    if (!g.other || !g.partial) return fail(KQ_ERR_INVALID_ARG, "gemm: dot epilogue needs `other` and `partial`");
   } else {
     if (!g.C || !aligned(g.C, 16) || (g.ldc & 3)) return fail(KQ_ERR_ALIGNMENT, "gemm: C must be 16-byte aligned");
+    if (g.epilogue == kEpiStoreSplit && (!g.C_small || !aligned(g.C_small, 16)))
+      return fail(KQ_ERR_ALIGNMENT, "gemm: C_small must be 16-byte aligned");
     if (g.epilogue == kEpiSubtract && (!g.src || !aligned(g.src, 16) || (g.ld_src & 3)))
       return fail(KQ_ERR_ALIGNMENT, "gemm: src must be 16-byte aligned");
   }

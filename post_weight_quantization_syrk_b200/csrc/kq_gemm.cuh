@@ -6,8 +6,10 @@
 
 namespace kq {
 
-// Epilogues: C = AB;  partial[tile] = sum_ij (AB)_ij other_ij;  C = src - AB.
-enum GemmEpilogue { kEpiStore = 0, kEpiDot = 1, kEpiSubtract = 2 };
+// Epilogues: C = AB;  partial[tile] = sum_ij (AB)_ij other_ij;  C = src - AB;
+// C = tf32(AB), C_small = AB - tf32(AB) (the product stored ready to be the
+// A operand of another 3xTF32 product).
+enum GemmEpilogue { kEpiStore = 0, kEpiDot = 1, kEpiSubtract = 2, kEpiStoreSplit = 3 };
 
 // C[M, N] = A[M, K] B[K, N], each operand given as a tf32 "big" part and an
 // fp32 remainder "small" (see split_tf32), as AB ~ Ab Bb + Ab Bs + As Bb
@@ -26,7 +28,14 @@ struct Gemm3xTF32 {
   const float* bt_small = nullptr;
   int64_t ldbt = 0, bt_row0 = 0, bt_col0 = 0;
   int epilogue = kEpiStore;
-  float* C = nullptr;              // (m, n) at C[m * ldc + n]      (store, subtract)
+  // Upper block triangle (M == N, dot epilogue only): only the tiles whose
+  // 256-column block is at or right of the 256-row block holding their rows
+  // are formed, and the partials of tiles off the 256 x 256 block diagonal
+  // are doubled: for a symmetric AB, the dot over the whole matrix when
+  // `other` is symmetric too.
+  bool upper = false;
+  float* C = nullptr;              // (m, n) at C[m * ldc + n]      (store, subtract, split: tf32 part)
+  float* C_small = nullptr;        // (m, n) at C_small[m * ldc + n] (split: remainder)
   int64_t ldc = 0;
   const float* src = nullptr;      // (m, n) at src[m * ld_src + n] (subtract)
   int64_t ld_src = 0;
@@ -39,8 +48,8 @@ struct Gemm3xTF32 {
 
 // Output tiles of an M x N x K product as launched (`partial` holds 8 per
 // tile for kEpiDot), and the most tiles any M x N product can use.
-int64_t gemm_tiles(int64_t M, int64_t N, int64_t K);
-int64_t gemm_tiles_max(int64_t M, int64_t N);
+int64_t gemm_tiles(int64_t M, int64_t N, int64_t K, bool upper = false);
+int64_t gemm_tiles_max(int64_t M, int64_t N, bool upper = false);
 
 kq_status gemm_3xtf32(const Gemm3xTF32& g, cudaStream_t st);
 

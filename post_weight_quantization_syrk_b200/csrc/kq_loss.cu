@@ -3,13 +3,23 @@
 // KronQ review (romaanj.github.io/reviews/kronq), Background: H ~ H_X kron H_G;
 // Unified Hessian-Guided PTQ (hub.valency.io/works/W_r72x54u6), Appendix A.1:
 // the Kronecker-weighted norm of a perturbation is a trace of this form.
-// Using the symmetry of H_G, tr(dW H_X dW^T H_G) = sum_ij (dW H_X)_ij (H_G dW)_ij.
 //
-// kq_kron_loss runs the two products on the tensor cores in 3xTF32 (fp32
-// accuracy; plain TF32 or bf16 lose too much to cancellation here): split
-// dW, H_X, H_G into tf32 + remainder, A1 = dW H_X stored, then H_G dW with
-// the elementwise product against A1 reduced in the GEMM epilogue to fp64
-// partials, summed in a fixed order.
+// kq_kron_loss writes the trace as a Frobenius product with one symmetric
+// factor, taking the smaller Hessian into the product:
+//   d_in <= d_out:  loss = <P, H_G>,  P = dW H_X^T dW^T      (d_out x d_out)
+//   d_in >  d_out:  loss = <P, H_X>,  P = dW^T H_G^T dW      (d_in x d_in)
+//   H_G = I:        loss = <P, H_X>,  P = dW^T dW
+// (each is tr(dW H_X dW^T H_G) by the cyclic property and tr(M) = tr(M^T)).
+// With D = dW or dW^T (n2 x n1, n1 the smaller side) and H1 the smaller
+// Hessian, A1 = D H1^T is formed first (n2 n1^2 multiply-adds), then P =
+// A1 D^T is formed only in its upper block triangle, each off-diagonal tile
+// counting twice (P and H2 are symmetric): about n2^2 n1 / 2 more, against
+// d_out d_in (d_in + d_out) for forming dW H_X and H_G dW in full.  Both
+// products run on the tensor cores in 3xTF32 (fp32 accuracy; plain TF32 or
+// bf16 lose too much to cancellation here); A1 leaves the first product
+// already split into tf32 + remainder, and the elementwise product of P
+// with H2 is reduced in the second product's epilogue to fp64 partials,
+// summed in a fixed order.
 //
 // kq_kron_loss_noalloc (below) keeps a SIMT fp32 path whose only scratch is
 // one fp64 per 64x64 tile: each CTA forms one tile of both products and
@@ -115,66 +125,37 @@ __global__ void sum_kernel(const double* __restrict__ partial, int64_t n, double
 
 namespace {
 
-// sum_ij A1_ij (Db + Ds)_ij: the H_G = I case (dW = Db + Ds exactly).
-__global__ void __launch_bounds__(256) dot_rows_kernel(const float* __restrict__ A1, const float* __restrict__ Db,
-                                                       const float* __restrict__ Ds, int64_t ld, int64_t rows,
-                                                       int64_t cols, double* __restrict__ partial) {
-  __shared__ double red[256];
-  double s = 0.0;
-  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x)
-    for (int64_t c = threadIdx.x; c < cols; c += blockDim.x) {
-      const int64_t i = r * ld + c;
-      s += (double)A1[i] * (double)(Db[i] + Ds[i]);
-    }
-  red[threadIdx.x] = s;
-  __syncthreads();
-  for (int w = 128; w > 0; w >>= 1) {
-    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) partial[blockIdx.x] = red[0];
-}
 
-constexpr int kDotBlocks = 1024;
-
-// dW (as A of dW H_X), dW^T (as the transposed B of H_G dW), H_X^T, H_G, each
-// split into tf32 + remainder, then A1 = dW H_X and the partial sums.
+// D = dW or dW^T (n2 x n1) and A1 = D H1^T, each as tf32 + remainder (leading
+// dimension ldd); H1 likewise (leading dimension ldh); the fp64 partials of
+// the upper block triangle of P.  Sized for either orientation.
 struct LossWs {
-  float *Db, *Ds, *Dtb, *Dts, *Xb, *Xs, *Gb, *Gs, *A1;
+  float *Db, *Ds, *Ab, *As, *Hb, *Hs;
   double* partial;
-  int64_t ldd, ldt, ldx, ldg;
 };
 
+constexpr int64_t lead(int64_t n) { return (n + 3) / 4 * 4; }
+
 size_t loss_layout(int64_t d_out, int64_t d_in, LossWs* w, void* base) {
-  const int64_t ldd = (d_in + 3) / 4 * 4, ldx = ldd, ldg = (d_out + 3) / 4 * 4, ldt = ldg;
+  const int64_t n1 = std::min(d_out, d_in), n2 = std::max(d_out, d_in);
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
     off = kq::align_up(off + bytes, 256);
     return o;
   };
-  const size_t sd = (size_t)d_out * ldd * 4, st_ = (size_t)d_in * ldt * 4, sx = (size_t)d_in * ldx * 4,
-               sg = (size_t)d_out * ldg * 4;
-  size_t oDb = take(sd), oDs = take(sd), oTb = take(st_), oTs = take(st_), oXb = take(sx), oXs = take(sx),
-         oGb = take(sg), oGs = take(sg), oA = take(sd);
-  const int64_t np = std::max<int64_t>(8 * kq::gemm_tiles_max(d_out, d_in), kDotBlocks);
-  size_t oP = take((size_t)np * 8);
+  const size_t sd = (size_t)std::max(d_out * lead(d_in), d_in * lead(d_out)) * 4, sh = (size_t)n1 * lead(n1) * 4;
+  size_t oDb = take(sd), oDs = take(sd), oAb = take(sd), oAs = take(sd), oHb = take(sh), oHs = take(sh);
+  size_t oP = take((size_t)8 * kq::gemm_tiles_max(n2, n2, true) * 8);
   if (w && base) {
     char* b = static_cast<char*>(base);
     w->Db = reinterpret_cast<float*>(b + oDb);
     w->Ds = reinterpret_cast<float*>(b + oDs);
-    w->Dtb = reinterpret_cast<float*>(b + oTb);
-    w->Dts = reinterpret_cast<float*>(b + oTs);
-    w->Xb = reinterpret_cast<float*>(b + oXb);
-    w->Xs = reinterpret_cast<float*>(b + oXs);
-    w->Gb = reinterpret_cast<float*>(b + oGb);
-    w->Gs = reinterpret_cast<float*>(b + oGs);
-    w->A1 = reinterpret_cast<float*>(b + oA);
+    w->Ab = reinterpret_cast<float*>(b + oAb);
+    w->As = reinterpret_cast<float*>(b + oAs);
+    w->Hb = reinterpret_cast<float*>(b + oHb);
+    w->Hs = reinterpret_cast<float*>(b + oHs);
     w->partial = reinterpret_cast<double*>(b + oP);
-    w->ldd = ldd;
-    w->ldt = ldt;
-    w->ldx = ldx;
-    w->ldg = ldg;
   }
   return off;
 }
@@ -188,8 +169,9 @@ extern "C" size_t kq_kron_loss_workspace_size(int64_t d_out, int64_t d_in) {
 
 namespace {
 
-// One loss; the tf32 splits of H_X and H_G are formed here unless `split_h`
-// is false (then they are already in the workspace from an earlier call).
+// One loss; the tf32 split of the smaller Hessian is formed here unless
+// `split_h` is false (then it is already in the workspace from an earlier
+// call with the same H_X, H_G and shape).
 kq_status kron_loss_impl(const float* W, int64_t ldw, const float* W_hat, int64_t ldwh, int64_t d_out, int64_t d_in,
                          const float* H_X, int64_t ldhx, const float* H_G, int64_t ldhg, double* loss, void* ws,
                          size_t ws_bytes, kq_stream_t stream, bool split_h) {
@@ -203,47 +185,53 @@ kq_status kron_loss_impl(const float* W, int64_t ldw, const float* W_hat, int64_
   cudaStream_t st = (cudaStream_t)stream;
   LossWs w;
   loss_layout(d_out, d_in, &w, ws);
-  KQ_TRY(kq::split_tf32(W, ldw, W_hat, ldwh, d_out, d_in, w.Db, w.Ds, w.ldd, false, st));
-  if (split_h) KQ_TRY(kq::split_tf32(H_X, ldhx, nullptr, 0, d_in, d_in, w.Xb, w.Xs, w.ldx, true, st));
-  kq::Gemm3xTF32 g1;                 // A1 = dW H_X   (B^T = H_X^T)
-  g1.M = d_out;
-  g1.N = d_in;
-  g1.K = d_in;
-  g1.a_big = w.Db;
-  g1.a_small = w.Ds;
-  g1.lda = w.ldd;
-  g1.bt_big = w.Xb;
-  g1.bt_small = w.Xs;
-  g1.ldbt = w.ldx;
-  g1.epilogue = kq::kEpiStore;
-  g1.C = w.A1;
-  g1.ldc = w.ldd;
-  KQ_TRY(kq::gemm_3xtf32(g1, st));
-  int64_t np;
-  if (H_G) {
-    KQ_TRY(kq::split_tf32(W, ldw, W_hat, ldwh, d_out, d_in, w.Dtb, w.Dts, w.ldt, true, st));
-    if (split_h) KQ_TRY(kq::split_tf32(H_G, ldhg, nullptr, 0, d_out, d_out, w.Gb, w.Gs, w.ldg, false, st));
-    kq::Gemm3xTF32 g2;               // sum (H_G dW) .* A1   (B^T = dW^T)
-    g2.M = d_out;
-    g2.N = d_in;
-    g2.K = d_out;
-    g2.a_big = w.Gb;
-    g2.a_small = w.Gs;
-    g2.lda = w.ldg;
-    g2.bt_big = w.Dtb;
-    g2.bt_small = w.Dts;
-    g2.ldbt = w.ldt;
-    g2.epilogue = kq::kEpiDot;
-    g2.other = w.A1;
-    g2.ld_other = w.ldd;
-    g2.partial = w.partial;
-    KQ_TRY(kq::gemm_3xtf32(g2, st));
-    np = 8 * kq::gemm_tiles(d_out, d_in, d_out);
-  } else {
-    dot_rows_kernel<<<kDotBlocks, 256, 0, st>>>(w.A1, w.Db, w.Ds, w.ldd, d_out, d_in, w.partial);
-    KQ_TRY(kq::launch_check("kq_kron_loss dot"));
-    np = kDotBlocks;
+  // orientation: the smaller Hessian goes into the product (see the top of this file)
+  const bool g_first = !H_G || d_in > d_out;
+  const int64_t n2 = g_first ? d_in : d_out, n1 = g_first ? d_out : d_in, ldd = lead(n1);
+  const float* H1 = g_first ? H_G : H_X;
+  const int64_t ld1 = g_first ? ldhg : ldhx;
+  const float* H2 = g_first ? H_X : H_G;
+  const int64_t ld2 = g_first ? ldhx : ldhg;
+  // D = dW (rows d_out) or dW^T (rows d_in), split into tf32 + remainder
+  KQ_TRY(kq::split_tf32(W, ldw, W_hat, ldwh, d_out, d_in, w.Db, w.Ds, ldd, g_first, st));
+  const float *Pa_b = w.Db, *Pa_s = w.Ds;   // A operand of P = A D^T: A1, or D when H1 = I
+  if (H1) {
+    if (split_h) KQ_TRY(kq::split_tf32(H1, ld1, nullptr, 0, n1, n1, w.Hb, w.Hs, lead(n1), false, st));
+    kq::Gemm3xTF32 g1;                 // A1 = D H1^T   (B^T = H1 as stored)
+    g1.M = n2;
+    g1.N = n1;
+    g1.K = n1;
+    g1.a_big = w.Db;
+    g1.a_small = w.Ds;
+    g1.lda = ldd;
+    g1.bt_big = w.Hb;
+    g1.bt_small = w.Hs;
+    g1.ldbt = lead(n1);
+    g1.epilogue = kq::kEpiStoreSplit;
+    g1.C = w.Ab;
+    g1.C_small = w.As;
+    g1.ldc = ldd;
+    KQ_TRY(kq::gemm_3xtf32(g1, st));
+    Pa_b = w.Ab;
+    Pa_s = w.As;
   }
+  kq::Gemm3xTF32 g2;                   // sum over the upper block triangle of (A1 D^T) .* H2
+  g2.M = n2;
+  g2.N = n2;
+  g2.K = n1;
+  g2.a_big = Pa_b;
+  g2.a_small = Pa_s;
+  g2.lda = ldd;
+  g2.bt_big = w.Db;
+  g2.bt_small = w.Ds;
+  g2.ldbt = ldd;
+  g2.epilogue = kq::kEpiDot;
+  g2.upper = true;
+  g2.other = H2;
+  g2.ld_other = ld2;
+  g2.partial = w.partial;
+  KQ_TRY(kq::gemm_3xtf32(g2, st));
+  const int64_t np = 8 * kq::gemm_tiles(n2, n2, n1, true);
   sum_kernel<<<1, 1024, 0, st>>>(w.partial, np, loss);
   KQ_TRY(kq::launch_check("kq_kron_loss sum"));
   kq::clear_error();
