@@ -173,7 +173,7 @@ def run_kronq(a):
         tag = "".join(f"w{r.bits}" for r in results)
         lq.quantize_all(results)   # every bit-width, one operand split of Uc
         mark(f"quantize_{tag}")
-        lq.loss_all(results)       # every bit-width, one split of H_X and H_G
+        lq.loss_all(results)       # every bit-width, one split of the smaller Hessian
         mark(f"loss_{tag}")
         if timed:
             stage_events.append(marks)

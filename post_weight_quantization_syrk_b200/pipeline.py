@@ -109,7 +109,7 @@ class LayerQuantizer:
                                   self.gemm_mode, ws, self.info, stream)
 
     def loss_all(self, results, stream=None):
-        """Every result's Kronecker loss in one call (the H_X, H_G splits are shared)."""
+        """Every result's Kronecker loss in one call (the split of the smaller Hessian is shared)."""
         ws = self.workspace(K.kq_kron_loss_workspace_size(self.d_out, self.d_in))
         K.kq_kron_loss_multi(self.Wp, [r.W_hat for r in results], self.H_X, self.H_G, [r.loss for r in results], ws,
                              stream)
