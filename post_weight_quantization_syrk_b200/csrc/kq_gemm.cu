@@ -59,6 +59,7 @@ struct Params {
   const float* src;
   int64_t ld_src;
   const uint8_t* dead;
+  int dead_vec;    // `dead` 4-byte aligned: the mask read 4 columns at a time
   const float* other;
   int64_t ld_other;
   int other_vec;   // `other` rows can be read as float4 (16-byte aligned rows)
@@ -143,6 +144,11 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
   __syncthreads();
   fence_after();
   const uint32_t tmem = *tmem_slot;
+  // set-up done: from here on global memory that earlier kernels may write.
+  // No early trigger: the solver's in-block kernel that follows fits three
+  // CTAs per SM and would pile onto the SMs this grid leaves idle (measured
+  // 17 % slower at d_out = 4096); it starts as these CTAs exit instead.
+  pdl_wait();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -262,7 +268,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
         for (int g0 = 0; g0 < 128; g0 += 64) {
           const int64_t gj0 = n0 + cbase + g0;
           const bool any = row_ok && gj0 < p.N;
-          const bool fast = any && gj0 + 64 <= p.N && !(p.epilogue == kEpiSubtract && p.dead) &&
+          const bool fast = any && gj0 + 64 <= p.N && !(p.epilogue == kEpiSubtract && p.dead && !p.dead_vec) &&
                             !(p.epilogue == kEpiDot && !p.other_vec);
           float pre[64];
           if (fast && (p.epilogue == kEpiDot || p.epilogue == kEpiSubtract)) {
@@ -274,6 +280,16 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
               pre[q + 1] = w.y;
               pre[q + 2] = w.z;
               pre[q + 3] = w.w;
+            }
+            if (p.epilogue == kEpiSubtract && p.dead) {
+              // dead source columns read as zero; the same 64 flags for every lane
+              const uint32_t* dm = reinterpret_cast<const uint32_t*>(p.dead + gj0);
+#pragma unroll
+              for (int q = 0; q < 16; ++q) {
+                const uint32_t m = dm[q];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) pre[4 * q + u] = ((m >> (8 * u)) & 0xffu) ? 0.f : pre[4 * q + u];
+              }
             }
           }
 #pragma unroll
@@ -476,6 +492,7 @@ kq_status gemm_3xtf32(const Gemm3xTF32& g, cudaStream_t st) {
   p.src = g.src;
   p.ld_src = g.ld_src;
   p.dead = g.dead;
+  p.dead_vec = (g.dead && aligned(g.dead, 4)) ? 1 : 0;
   p.other = g.other;
   p.ld_other = g.ld_other;
   p.other_vec = (g.other && aligned(g.other, 16) && !(g.ld_other & 3)) ? 1 : 0;
@@ -497,8 +514,8 @@ kq_status gemm_3xtf32(const Gemm3xTF32& g, cudaStream_t st) {
   KQ_TRY(cuda_check(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev), "gemm: SM count"));
   KQ_TRY(cuda_check(cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES),
                     "gemm: smem attribute"));
-  gemm_kernel<<<std::min(p.num_tiles, sms), THREADS, SMEM_BYTES, st>>>(maps, p);
-  return launch_check("gemm_3xtf32");
+  return launch_ex("gemm_3xtf32", g.pdl, gemm_kernel, dim3((unsigned)std::min(p.num_tiles, sms)), dim3(THREADS),
+                   SMEM_BYTES, st, maps, p);
 }
 
 }  // namespace kq

@@ -44,6 +44,9 @@ struct Gemm3xTF32 {
   int64_t ld_other = 0;
   double* partial = nullptr;       // dot: 8 fp64 per output tile (one per epilogue warp)
   int32_t* info = nullptr;
+  // Launched as a programmatic dependent of the previous kernel on the
+  // stream, which must be a kernel of the same call (see pdl_wait).
+  bool pdl = false;
 };
 
 // Output tiles of an M x N x K product as launched (`partial` holds 8 per

@@ -126,9 +126,12 @@ __global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
   const bool row_ok = row < a.d_out;
   const int bw = a.bw;
   const int64_t i0 = a.i0;
+  kq::pdl_trigger();
 
   // the block of Uc: 16 asynchronous 16-byte copies per thread, all in
-  // flight while the row is loaded (bytes past the block are zero-filled)
+  // flight while the row is loaded (bytes past the block are zero-filled).
+  // No kernel of the solve writes Uc, so the copies may start before the
+  // previous kernel (a trailing update) has finished.
 #pragma unroll
   for (int u = 0; u < BLK * (BLK / 4) / IB_THREADS; ++u) {
     const int idx = t + IB_THREADS * u;
@@ -141,6 +144,7 @@ __global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(g), "r"(nbytes) : "memory");
   }
   asm volatile("cp.async.commit_group;" ::: "memory");
+  kq::pdl_wait();
 
   // this lane's 16 columns of the row
   float w[16];
@@ -467,8 +471,10 @@ kq_status quantize_impl(const float* W, int64_t d_out, int64_t d_in, int64_t ldw
     a.ldE = OUTER;
     a.e_col0 = i0 - o0;
     a.info = info;
-    inblock_kernel<<<(unsigned)kq::cdiv(d_out, IB_ROWS), IB_THREADS, IB_SMEM, st>>>(a);
-    return kq::launch_check("kq_quantize_layer inblock");
+    // after the first block the previous kernel is this solve's own trailing
+    // update, so the launch may overlap its tail (tensor-core mode)
+    return kq::launch_ex("kq_quantize_layer inblock", tc && i0 > 0, inblock_kernel,
+                         dim3((unsigned)kq::cdiv(d_out, IB_ROWS)), dim3(IB_THREADS), IB_SMEM, st, a);
   };
   // W_hat[:, c0:c0+N] = src[:, c0:c0+N] - E[:, e0:e0+K] Uc[k0:k0+K, c0:c0+N]; the
   // source is W (dead columns as zeros) while those columns are still untouched.
@@ -493,6 +499,7 @@ kq_status quantize_impl(const float* W, int64_t d_out, int64_t d_in, int64_t ldw
     g.ld_src = from_w ? ldw : ldwh;
     g.dead = from_w && dead_mask ? dead_mask + c0 : nullptr;
     g.info = info;
+    g.pdl = true;   // always follows this solve's in-block kernel
     return kq::gemm_3xtf32(g, st);
   };
   if (!tc) {
