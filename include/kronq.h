@@ -228,13 +228,22 @@ kq_status kq_quantize_layer(const float* W, int64_t d_out, int64_t d_in, int64_t
 
 /* kq_quantize_layer_multi - kq_quantize_layer for `count` settings of one
  * layer (the same W, Uc and dead mask; bit-width bits[i] and group group[i]
- * into codes[i], scales[i], zeros[i], W_hat[i]), run one after the other on
- * `stream`.  The 3xTF32 operand split of Uc is formed once for all settings
- * (KronQ paper page, authors' reply: one set of statistics serves every
- * bit-width).  The pointer arrays are HOST arrays of device pointers, read
- * during the call.  Workspace: kq_quantize_layer_workspace_size (the same as
- * for one setting).  Errors as kq_quantize_layer; count >= 1; every setting
- * is validated before any work is enqueued. */
+ * into codes[i], scales[i], zeros[i], W_hat[i]).  The 3xTF32 operand split
+ * of Uc is formed once for all settings (KronQ paper page, authors' reply:
+ * one set of statistics serves every bit-width).  With a workspace of
+ * kq_quantize_layer_multi_workspace_size(d_out, d_in, block, count) bytes
+ * up to 4 settings are solved side by side: setting i runs on lane i % 4,
+ * lane 0 being `stream` and the others internal streams of the library
+ * (created on the first such call of each host thread on each device)
+ * forked from and joined back into `stream` by events, so all the work is
+ * still ordered on `stream` as one call.  With a smaller workspace of at
+ * least kq_quantize_layer_workspace_size bytes the settings run one after
+ * the other on `stream`.  The results are the same either way, bit for bit.
+ * The pointer arrays are HOST arrays of device pointers, read during the
+ * call; no two settings may share an output buffer.  Errors as
+ * kq_quantize_layer; count >= 1; every setting is validated before any
+ * work is enqueued. */
+size_t kq_quantize_layer_multi_workspace_size(int64_t d_out, int64_t d_in, int block, int count);
 kq_status kq_quantize_layer_multi(const float* W, int64_t d_out, int64_t d_in, int64_t ldw,
                                   const float* Uc, int64_t lduc, const uint8_t* dead_mask,
                                   int count, const int* bits, const int* group, int block, int gemm_mode,

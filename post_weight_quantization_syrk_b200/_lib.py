@@ -32,7 +32,8 @@ EXPORTS = (
     "kq_sensitivity",
     "kq_rotate",
     "kq_chol_inv_workspace_size", "kq_chol_inv",
-    "kq_quantize_layer_workspace_size", "kq_quantize_layer", "kq_quantize_layer_multi",
+    "kq_quantize_layer_workspace_size", "kq_quantize_layer", "kq_quantize_layer_multi_workspace_size",
+    "kq_quantize_layer_multi",
     "kq_kron_loss_workspace_size", "kq_kron_loss", "kq_kron_loss_multi", "kq_kron_loss_noalloc",
     "kq_allocate_bits",
 )
@@ -65,6 +66,7 @@ _SIGS = {
     "kq_chol_inv_workspace_size": (_sz, [_i64]),
     "kq_chol_inv": (_i32, [_vp, _i64, _i64, _f32, _vp, _i64, _vp, _vp, _sz, _vp, _vp]),
     "kq_quantize_layer_workspace_size": (_sz, [_i64, _i64, _i32]),
+    "kq_quantize_layer_multi_workspace_size": (_sz, [_i64, _i64, _i32, _i32]),
     "kq_quantize_layer": (_i32, [_vp, _i64, _i64, _i64, _vp, _i64, _vp, _i32, _i32, _i32, _i32,
                                  _vp, _i64, _vp, _vp, _vp, _i64, _vp, _sz, _vp, _vp]),
     "kq_quantize_layer_multi": (_i32, [_vp, _i64, _i64, _i64, _vp, _i64, _vp, _i32, ctypes.POINTER(ctypes.c_int),
@@ -231,6 +233,11 @@ def kq_quantize_layer_workspace_size(d_out: int, d_in: int, block: int = 128) ->
     return int(load().kq_quantize_layer_workspace_size(int(d_out), int(d_in), int(block)))
 
 
+def kq_quantize_layer_multi_workspace_size(d_out: int, d_in: int, block: int = 128, count: int = 1) -> int:
+    """Workspace with which kq_quantize_layer_multi solves `count` settings side by side."""
+    return int(load().kq_quantize_layer_multi_workspace_size(int(d_out), int(d_in), int(block), int(count)))
+
+
 def kq_quantize_layer(W, Uc, dead_mask, bits, group, codes, scales, zeros, W_hat, block=128,
                       gemm_mode=KQ_GEMM_FP32, ws=None, info=None, stream=None):
     ldw = _mat(W, torch.float32, "W")
@@ -274,7 +281,7 @@ def kq_quantize_layer_multi(W, Uc, dead_mask, settings, codes, scales, zeros, W_
             if t.dtype != torch.float32 or not t.is_contiguous() or t.numel() < d_out * ng:
                 raise TypeError(f"{nm} must be contiguous float32 [d_out, n_groups]")
     if ws is None:
-        ws = workspace(kq_quantize_layer_workspace_size(d_out, d_in, block), W.device)
+        ws = workspace(kq_quantize_layer_multi_workspace_size(d_out, d_in, block, k), W.device)
     wp, wb = _buf(ws)
     bits = (ctypes.c_int * k)(*[int(b) for b, _ in settings])
     groups = (ctypes.c_int * k)(*[int(g) for _, g in settings])

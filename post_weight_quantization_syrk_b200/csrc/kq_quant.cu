@@ -369,28 +369,32 @@ namespace {
 // outer block one GEMM with K = OUTER updates all columns to its right.
 constexpr int OUTER = 1024;
 
-// Workspace: the errors (E^T of one block for the fp32 path, or E of one
-// outer block split in two for 3xTF32), then Uc^T split in two (3xTF32 only:
-// the tensor-core product reads its B operand transposed).
+// Workspace: per lane (one setting being solved at a time) the errors (E^T
+// of one block for the fp32 path, or E of one outer block split in two for
+// 3xTF32), then, shared by the lanes, Uc^T split in two (3xTF32 only: the
+// tensor-core product reads its B operand transposed).
 struct QuantWs {
   float *ET, *Eb, *Es, *Ub, *Us;
   int64_t ldu;
 };
 
-size_t quant_layout(int64_t d_out, int64_t d_in, QuantWs* w, void* base) {
+// Most settings kq_quantize_layer_multi solves side by side.
+constexpr int kMaxLanes = 4;
+
+size_t quant_layout(int64_t d_out, int64_t d_in, int lanes, int lane, QuantWs* w, void* base) {
   const int64_t ldu = (d_in + 3) / 4 * 4;
   const size_t se = kq::align_up((size_t)d_out * OUTER * sizeof(float), 256);
   const size_t su = kq::align_up((size_t)d_in * ldu * sizeof(float), 256);
   if (w && base) {
     char* b = static_cast<char*>(base);
-    w->ET = reinterpret_cast<float*>(b);
-    w->Eb = reinterpret_cast<float*>(b);
-    w->Es = reinterpret_cast<float*>(b + se);
-    w->Ub = reinterpret_cast<float*>(b + 2 * se);
-    w->Us = reinterpret_cast<float*>(b + 2 * se + su);
+    w->ET = reinterpret_cast<float*>(b + 2 * se * lane);
+    w->Eb = w->ET;
+    w->Es = reinterpret_cast<float*>(b + 2 * se * lane + se);
+    w->Ub = reinterpret_cast<float*>(b + 2 * se * lanes);
+    w->Us = reinterpret_cast<float*>(b + 2 * se * lanes + su);
     w->ldu = ldu;
   }
-  return 2 * se + 2 * su;
+  return 2 * se * lanes + 2 * su;
 }
 
 }  // namespace
@@ -398,18 +402,21 @@ size_t quant_layout(int64_t d_out, int64_t d_in, QuantWs* w, void* base) {
 extern "C" size_t kq_quantize_layer_workspace_size(int64_t d_out, int64_t d_in, int block) {
   (void)block;
   if (d_out < 1 || d_in < 1) return 0;
-  return quant_layout(d_out, d_in, nullptr, nullptr);
+  return quant_layout(d_out, d_in, 1, 0, nullptr, nullptr);
+}
+
+extern "C" size_t kq_quantize_layer_multi_workspace_size(int64_t d_out, int64_t d_in, int block, int count) {
+  (void)block;
+  if (d_out < 1 || d_in < 1 || count < 1) return 0;
+  return quant_layout(d_out, d_in, std::min(count, kMaxLanes), 0, nullptr, nullptr);
 }
 
 namespace {
 
-// One setting; the tf32 split of Uc^T (3xTF32 mode) is formed here unless
-// `split_uc` is false (then it is already in the workspace from an earlier
-// call with the same Uc).
-kq_status quantize_impl(const float* W, int64_t d_out, int64_t d_in, int64_t ldw, const float* Uc, int64_t lduc,
-                        const uint8_t* dead_mask, int bits, int group, int block, int gemm_mode, uint8_t* codes,
-                        int64_t ldq, float* scales, float* zeros, float* W_hat, int64_t ldwh, void* ws,
-                        size_t ws_bytes, int32_t* info, kq_stream_t stream, bool split_uc) {
+// Host-side checks of one setting (nothing is enqueued).
+kq_status check_args(const float* W, int64_t d_out, int64_t d_in, int64_t ldw, const float* Uc, int64_t lduc, int bits,
+                     int group, int block, int gemm_mode, const uint8_t* codes, int64_t ldq, const float* scales,
+                     const float* zeros, const float* W_hat, int64_t ldwh, const int32_t* info) {
   if (!W || !Uc || !codes || !scales || !zeros || !W_hat || !info)
     return kq::fail(KQ_ERR_INVALID_ARG, "kq_quantize_layer: NULL pointer");
   if (d_out < 1 || d_in < 1 || d_in > 65536) return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_quantize_layer: sizes");
@@ -425,11 +432,16 @@ kq_status quantize_impl(const float* W, int64_t d_out, int64_t d_in, int64_t ldw
   if (W == W_hat) return kq::fail(KQ_ERR_INVALID_ARG, "kq_quantize_layer: W and W_hat must not alias");
   if (!kq::aligned(W, 16) || !kq::aligned(W_hat, 16) || !kq::aligned(Uc, 16) || (ldw & 3) || (ldwh & 3) || (lduc & 3))
     return kq::fail(KQ_ERR_ALIGNMENT, "kq_quantize_layer: W, W_hat, Uc need 16-byte alignment and ld % 4 == 0");
-  if (!ws || !kq::aligned(ws, 256) || ws_bytes < kq_quantize_layer_workspace_size(d_out, d_in, block))
-    return kq::fail(KQ_ERR_WORKSPACE, "kq_quantize_layer: workspace too small or not 256-byte aligned");
-  cudaStream_t st = (cudaStream_t)stream;
-  QuantWs w;
-  quant_layout(d_out, d_in, &w, ws);
+  return KQ_OK;
+}
+
+// Enqueues one checked setting on `st` with the workspace lane `w`; the tf32
+// split of Uc^T (3xTF32 mode) is formed here unless `split_uc` is false
+// (then it is already in the workspace, from an earlier setting).
+kq_status enqueue_setting(const float* W, int64_t d_out, int64_t d_in, int64_t ldw, const float* Uc, int64_t lduc,
+                          const uint8_t* dead_mask, int bits, int group, int gemm_mode, uint8_t* codes, int64_t ldq,
+                          float* scales, float* zeros, float* W_hat, int64_t ldwh, const QuantWs& w, int32_t* info,
+                          cudaStream_t st, bool split_uc) {
   const bool tc = (gemm_mode == KQ_GEMM_3XTF32);
   if (tc && split_uc) KQ_TRY(kq::split_tf32(Uc, lduc, nullptr, 0, d_in, d_in, w.Ub, w.Us, w.ldu, true, st));
 
@@ -532,13 +544,57 @@ kq_status quantize_impl(const float* W, int64_t d_out, int64_t d_in, int64_t ldw
 
 }  // namespace
 
+namespace {
+
+// Streams and events for solving settings side by side: created on first
+// use by each host thread for each device, kept for the thread's lifetime.
+struct Lanes {
+  int device = -1;
+  cudaStream_t s[kMaxLanes - 1] = {};
+  cudaEvent_t fork = nullptr;
+  cudaEvent_t join[kMaxLanes - 1] = {};
+};
+
+kq_status side_lanes(Lanes** out) {
+  thread_local Lanes cache[16];
+  int dev = 0;
+  KQ_TRY(kq::cuda_check(cudaGetDevice(&dev), "kq_quantize_layer_multi: cudaGetDevice"));
+  Lanes* l = nullptr;
+  for (auto& c : cache)
+    if (c.device == dev) l = &c;
+  if (!l) {
+    for (auto& c : cache)
+      if (c.device < 0) {
+        l = &c;
+        break;
+      }
+    if (!l) return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_quantize_layer_multi: more than 16 devices");
+    for (auto& st : l->s)
+      KQ_TRY(kq::cuda_check(cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking), "kq_quantize_layer_multi: stream"));
+    KQ_TRY(kq::cuda_check(cudaEventCreateWithFlags(&l->fork, cudaEventDisableTiming), "kq_quantize_layer_multi: event"));
+    for (auto& e : l->join)
+      KQ_TRY(kq::cuda_check(cudaEventCreateWithFlags(&e, cudaEventDisableTiming), "kq_quantize_layer_multi: event"));
+    l->device = dev;
+  }
+  *out = l;
+  return KQ_OK;
+}
+
+}  // namespace
+
 extern "C" kq_status kq_quantize_layer(const float* W, int64_t d_out, int64_t d_in, int64_t ldw, const float* Uc,
                                        int64_t lduc, const uint8_t* dead_mask, int bits, int group, int block,
                                        int gemm_mode, uint8_t* codes, int64_t ldq, float* scales, float* zeros,
                                        float* W_hat, int64_t ldwh, void* ws, size_t ws_bytes, int32_t* info,
                                        kq_stream_t stream) {
-  return quantize_impl(W, d_out, d_in, ldw, Uc, lduc, dead_mask, bits, group, block, gemm_mode, codes, ldq, scales,
-                       zeros, W_hat, ldwh, ws, ws_bytes, info, stream, true);
+  KQ_TRY(check_args(W, d_out, d_in, ldw, Uc, lduc, bits, group, block, gemm_mode, codes, ldq, scales, zeros, W_hat,
+                    ldwh, info));
+  if (!ws || !kq::aligned(ws, 256) || ws_bytes < kq_quantize_layer_workspace_size(d_out, d_in, block))
+    return kq::fail(KQ_ERR_WORKSPACE, "kq_quantize_layer: workspace too small or not 256-byte aligned");
+  QuantWs w;
+  quant_layout(d_out, d_in, 1, 0, &w, ws);
+  return enqueue_setting(W, d_out, d_in, ldw, Uc, lduc, dead_mask, bits, group, gemm_mode, codes, ldq, scales, zeros,
+                         W_hat, ldwh, w, info, (cudaStream_t)stream, true);
 }
 
 extern "C" kq_status kq_quantize_layer_multi(const float* W, int64_t d_out, int64_t d_in, int64_t ldw,
@@ -551,16 +607,51 @@ extern "C" kq_status kq_quantize_layer_multi(const float* W, int64_t d_out, int6
     return kq::fail(KQ_ERR_INVALID_ARG, "kq_quantize_layer_multi: count < 1 or NULL array");
   // every setting is checked before any work is enqueued
   for (int i = 0; i < count; ++i) {
-    if (!codes[i] || !scales[i] || !zeros[i] || !W_hat[i])
-      return kq::fail(KQ_ERR_INVALID_ARG, "kq_quantize_layer_multi: NULL output of setting %d", i);
-    if (bits[i] < 2 || bits[i] > 8) return kq::fail(KQ_ERR_INVALID_ARG, "kq_quantize_layer_multi: bits outside 2..8");
-    if (group[i] < 0 || (group[i] && (group[i] % 32 || BLK % group[i])))
-      return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE,
-                      "kq_quantize_layer_multi: group must be 0 or a multiple of 32 dividing 128");
-    if (W == W_hat[i]) return kq::fail(KQ_ERR_INVALID_ARG, "kq_quantize_layer_multi: W and W_hat must not alias");
+    KQ_TRY(check_args(W, d_out, d_in, ldw, Uc, lduc, bits[i], group[i], block, gemm_mode, codes[i], ldq, scales[i],
+                      zeros[i], W_hat[i], ldwh, info));
+    for (int j = 0; j < i; ++j)
+      if (codes[j] == codes[i] || scales[j] == scales[i] || zeros[j] == zeros[i] || W_hat[j] == W_hat[i])
+        return kq::fail(KQ_ERR_INVALID_ARG, "kq_quantize_layer_multi: settings %d and %d share an output", j, i);
   }
-  for (int i = 0; i < count; ++i)
-    KQ_TRY(quantize_impl(W, d_out, d_in, ldw, Uc, lduc, dead_mask, bits[i], group[i], block, gemm_mode, codes[i], ldq,
-                         scales[i], zeros[i], W_hat[i], ldwh, ws, ws_bytes, info, stream, i == 0));
+  if (!ws || !kq::aligned(ws, 256))
+    return kq::fail(KQ_ERR_WORKSPACE, "kq_quantize_layer_multi: workspace NULL or not 256-byte aligned");
+  // side by side when the workspace holds a lane per setting (up to
+  // kMaxLanes), else one after the other in a single lane
+  int lanes = std::min(count, kMaxLanes);
+  if (ws_bytes < quant_layout(d_out, d_in, lanes, 0, nullptr, nullptr)) lanes = 1;
+  if (ws_bytes < quant_layout(d_out, d_in, lanes, 0, nullptr, nullptr))
+    return kq::fail(KQ_ERR_WORKSPACE, "kq_quantize_layer_multi: workspace too small");
+  QuantWs w[kMaxLanes];
+  for (int l = 0; l < lanes; ++l) quant_layout(d_out, d_in, lanes, l, &w[l], ws);
+  cudaStream_t st = (cudaStream_t)stream;
+  if (lanes == 1) {
+    for (int i = 0; i < count; ++i)
+      KQ_TRY(enqueue_setting(W, d_out, d_in, ldw, Uc, lduc, dead_mask, bits[i], group[i], gemm_mode, codes[i], ldq,
+                             scales[i], zeros[i], W_hat[i], ldwh, w[0], info, st, i == 0));
+    return KQ_OK;
+  }
+  Lanes* L = nullptr;
+  KQ_TRY(side_lanes(&L));
+  // the shared split of Uc^T on the caller's stream, then the fork
+  if (gemm_mode == KQ_GEMM_3XTF32)
+    KQ_TRY(kq::split_tf32(Uc, lduc, nullptr, 0, d_in, d_in, w[0].Ub, w[0].Us, w[0].ldu, true, st));
+  KQ_TRY(kq::cuda_check(cudaEventRecord(L->fork, st), "kq_quantize_layer_multi: record"));
+  for (int l = 1; l < lanes; ++l)
+    KQ_TRY(kq::cuda_check(cudaStreamWaitEvent(L->s[l - 1], L->fork, 0), "kq_quantize_layer_multi: wait"));
+  kq_status first = KQ_OK;
+  for (int i = 0; i < count && first == KQ_OK; ++i) {
+    const int l = i % lanes;
+    first = enqueue_setting(W, d_out, d_in, ldw, Uc, lduc, dead_mask, bits[i], group[i], gemm_mode, codes[i], ldq,
+                            scales[i], zeros[i], W_hat[i], ldwh, w[l], info, l ? L->s[l - 1] : st, false);
+  }
+  // the join is enqueued even after a failed launch, so that the caller's
+  // stream is ordered after everything that did get enqueued
+  for (int l = 1; l < lanes; ++l) {
+    cudaError_t e = cudaEventRecord(L->join[l - 1], L->s[l - 1]);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, L->join[l - 1], 0);
+    if (e != cudaSuccess && first == KQ_OK) first = kq::cuda_check(e, "kq_quantize_layer_multi: join");
+  }
+  if (first != KQ_OK) return first;
+  kq::clear_error();
   return KQ_OK;
 }

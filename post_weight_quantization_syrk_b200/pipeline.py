@@ -101,8 +101,9 @@ class LayerQuantizer:
         K.kq_kron_loss(self.Wp, res.W_hat, self.H_X, self.H_G, res.loss, ws, stream)
 
     def quantize_all(self, results, stream=None):
-        """Every setting of `results` in one call (the factor's operand split is shared)."""
-        ws = self.workspace(K.kq_quantize_layer_workspace_size(self.d_out, self.d_in, self.block))
+        """Every setting of `results` in one call: the factor's operand split is
+        shared and up to four settings are solved side by side."""
+        ws = self.workspace(K.kq_quantize_layer_multi_workspace_size(self.d_out, self.d_in, self.block, len(results)))
         K.kq_quantize_layer_multi(self.Wp, self.Uc, self.dead, [(r.bits, r.group) for r in results],
                                   [r.codes for r in results], [r.scales for r in results],
                                   [r.zeros for r in results], [r.W_hat for r in results], self.block,

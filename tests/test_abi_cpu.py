@@ -140,6 +140,18 @@ def test_workspace_sizes():
     assert P.kq_chol_inv_workspace_size(0) == 0
 
 
+def test_multi_workspace_sizes():
+    """One lane per setting up to four lanes; one lane is the single-setting size."""
+    one = P.kq_quantize_layer_workspace_size(4096, 4096)
+    sizes = [P.kq_quantize_layer_multi_workspace_size(4096, 4096, 128, c) for c in range(1, 7)]
+    assert sizes[0] == one
+    lane = sizes[1] - sizes[0]
+    assert lane >= 2 * 4096 * 1024 * 4
+    assert sizes[:4] == [one + k * lane for k in range(4)]
+    assert sizes[4] == sizes[5] == sizes[3]
+    assert P.kq_quantize_layer_multi_workspace_size(4096, 4096, 128, 0) == 0
+
+
 def test_multi_entry_points_validate_before_enqueue():
     """Host-side rejections of the multi-setting calls (no device work)."""
     import ctypes
@@ -154,3 +166,8 @@ def test_multi_entry_points_validate_before_enqueue():
     assert st == 1 and b"bits" in lib.kq_last_error()   # KQ_ERR_INVALID_ARG
     st = lib.kq_kron_loss_multi(dummy, 128, 0, arr, 128, 4, 128, dummy, 128, dummy, 4, arr, dummy, 1 << 30, None)
     assert st == 1   # KQ_ERR_INVALID_ARG
+    shared = (vp * 2)(vp(32), vp(32))        # both settings write the same W_hat
+    bits = (ctypes.c_int * 2)(3, 4)
+    st = lib.kq_quantize_layer_multi(dummy, 4, 128, 128, dummy, 128, None, 2, bits, groups, 128, 0, arr, 128, arr,
+                                     arr, shared, 128, dummy, 1 << 30, dummy, None)
+    assert st == 1 and b"share an output" in lib.kq_last_error()

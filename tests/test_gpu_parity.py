@@ -402,11 +402,15 @@ def test_layer512_whole_path_stagewise(P):
 
 # ------------------------------------------------------------------ multi-setting entry points
 
-def test_multi_entry_points_match_single_calls(P, rotated_small):
+@pytest.mark.parametrize("gemm_mode", ["3xtf32", "fp32"])
+def test_multi_entry_points_match_single_calls(P, rotated_small, gemm_mode):
     """kq_quantize_layer_multi / kq_kron_loss_multi share the operand splits
-    across settings and must return exactly what the single calls return."""
+    across settings and must return exactly what the single calls return,
+    whether the settings run side by side (four lanes, the fifth setting
+    reusing lane 0) or one after the other (single-setting workspace)."""
     lq = rotated_small[0]
-    settings = [(4, 0), (3, 128), (2, 0)]
+    mode = P.KQ_GEMM_3XTF32 if gemm_mode == "3xtf32" else P.KQ_GEMM_FP32
+    settings = [(4, 0), (3, 128), (2, 0), (3, 0), (4, 64)]
     d_out, d_in = lq.Wp.shape
 
     def outputs():
@@ -418,16 +422,21 @@ def test_multi_entry_points_match_single_calls(P, rotated_small):
                         torch.empty((d_out, d_in), device="cuda"), torch.zeros(1, dtype=torch.float64, device="cuda")))
         return res
 
-    one, many = outputs(), outputs()
+    one, many, seq = outputs(), outputs(), outputs()
     info = _info()
     for (b, g), (c, s, z, wh, l) in zip(settings, one):
-        P.kq_quantize_layer(lq.Wp, lq.Uc, lq.dead, b, g, c, s, z, wh, gemm_mode=P.KQ_GEMM_3XTF32, info=info)
+        P.kq_quantize_layer(lq.Wp, lq.Uc, lq.dead, b, g, c, s, z, wh, gemm_mode=mode, info=info)
         P.kq_kron_loss(lq.Wp, wh, lq.H_X, lq.H_G, l)
     P.kq_quantize_layer_multi(lq.Wp, lq.Uc, lq.dead, settings, [o[0] for o in many], [o[1] for o in many],
-                              [o[2] for o in many], [o[3] for o in many], gemm_mode=P.KQ_GEMM_3XTF32, info=info)
+                              [o[2] for o in many], [o[3] for o in many], gemm_mode=mode, info=info)
     P.kq_kron_loss_multi(lq.Wp, [o[3] for o in many], lq.H_X, lq.H_G, [o[4] for o in many])
+    ws1 = P.workspace(P.kq_quantize_layer_workspace_size(d_out, d_in), lq.Wp.device)
+    P.kq_quantize_layer_multi(lq.Wp, lq.Uc, lq.dead, settings, [o[0] for o in seq], [o[1] for o in seq],
+                              [o[2] for o in seq], [o[3] for o in seq], gemm_mode=mode, ws=ws1, info=info)
+    P.kq_kron_loss_multi(lq.Wp, [o[3] for o in seq], lq.H_X, lq.H_G, [o[4] for o in seq])
     torch.cuda.synchronize()
     assert _info_code(info)[0] == 0
-    for a, b in zip(one, many):
-        for x, y in zip(a, b):
+    for a, b, c in zip(one, many, seq):
+        for x, y, z in zip(a, b, c):
             assert torch.equal(x, y)
+            assert torch.equal(x, z)
