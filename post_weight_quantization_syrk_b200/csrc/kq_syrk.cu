@@ -60,6 +60,7 @@ struct Params {
   int accumulate;
   float* C;
   int64_t ldc;
+  int c_vec;        // C rows 16-byte aligned (C aligned, ldc % 4 == 0)
   float* partial;   // [splits][num_tiles][256][256] when splits > 1
   int32_t* info;
 };
@@ -269,43 +270,98 @@ __global__ void __launch_bounds__(THREADS, 1) syrk_tc_kernel(const __grid_consta
   }
 }
 
-// Sum the token splits of every lower tile in split order, apply alpha (and
-// the old C when accumulating), write the lower element and its mirror.
-// One CTA per (tile, 32-row band); 32x8 threads; the mirror goes through a
-// shared-memory transpose so both writes are coalesced.
+// Sum the token splits of every lower tile in split order (s = 0, then
+// s += split 0, 1, ... in fp32), apply alpha (and the old C when
+// accumulating), write the lower element and its mirror.  One CTA per
+// (tile, 32-row band); per 128-column half each of the 8 warps owns 4 rows
+// and each lane 4 adjacent columns, so the partials stream in as float4
+// loads, the four rows' loads of two splits in flight together; the mirror
+// goes through a shared-memory transpose so both writes are coalesced.
 __global__ void __launch_bounds__(256) split_reduce_kernel(Params p) {
-  __shared__ float t[32][33];
+  __shared__ float t[32][129];
   const int tile = blockIdx.x / 8;
   const int band = blockIdx.x % 8;  // 32-row band within the 256-row tile
   int ti, tj;
   tri_index(tile, &ti, &tj);
   const int64_t i0 = (int64_t)ti * TILE + band * 32, j0 = (int64_t)tj * TILE;
-  const int tx = threadIdx.x % 32, ty = threadIdx.x / 32;
-  for (int cb = 0; cb < TILE; cb += 32) {
-    const int64_t gj = j0 + cb + tx;
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+  const int64_t split_stride = (int64_t)p.num_tiles * TILE * TILE;
+  for (int h = 0; h < 2; ++h) {
+    const int cl = h * 128 + 4 * lane;   // first of this lane's 4 columns in the tile
+    const float* src = p.partial + ((int64_t)tile * TILE + band * 32 + warp) * TILE + cl;
+    float acc[4][4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[k][e] = 0.f;
+    int sp = 0;
+    for (; sp + 1 < p.splits; sp += 2) {
+      float4 v0[4], v1[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) v0[k] = *reinterpret_cast<const float4*>(src + sp * split_stride + 8 * k * TILE);
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        v1[k] = *reinterpret_cast<const float4*>(src + (sp + 1) * split_stride + 8 * k * TILE);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        acc[k][0] += v0[k].x;
+        acc[k][1] += v0[k].y;
+        acc[k][2] += v0[k].z;
+        acc[k][3] += v0[k].w;
+        acc[k][0] += v1[k].x;
+        acc[k][1] += v1[k].y;
+        acc[k][2] += v1[k].z;
+        acc[k][3] += v1[k].w;
+      }
+    }
+    if (sp < p.splits) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float4 v = *reinterpret_cast<const float4*>(src + sp * split_stride + 8 * k * TILE);
+        acc[k][0] += v.x;
+        acc[k][1] += v.y;
+        acc[k][2] += v.z;
+        acc[k][3] += v.w;
+      }
+    }
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const int rr = ty + 8 * k;
-      const int64_t gi = i0 + rr;
-      float s = 0.f;
-      for (int sp = 0; sp < p.splits; ++sp)
-        s += p.partial[(((int64_t)sp * p.num_tiles + tile) * TILE + band * 32 + rr) * TILE + cb + tx];
-      float val = p.alpha * s;
-      const bool keep = gi < p.d && gj < p.d && gj <= gi;
-      if (keep) {
-        if (p.accumulate) val += p.C[gi * p.ldc + gj];
-        if (!isfinite(val)) kq::report(p.info, KQ_ERR_NONFINITE, gi);
-        p.C[gi * p.ldc + gj] = val;
+      const int rr = warp + 8 * k;
+      const int64_t gi = i0 + rr, gj = j0 + cl;
+      float v[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[e] = p.alpha * acc[k][e];
+      if (gi < p.d) {
+        float* c = p.C + gi * p.ldc + gj;
+        if (p.c_vec && gj + 3 < p.d && gj + 3 <= gi) {
+          if (p.accumulate) {
+            const float4 o = *reinterpret_cast<const float4*>(c);
+            v[0] += o.x;
+            v[1] += o.y;
+            v[2] += o.z;
+            v[3] += o.w;
+          }
+          if (!(isfinite(v[0]) && isfinite(v[1]) && isfinite(v[2]) && isfinite(v[3])))
+            kq::report(p.info, KQ_ERR_NONFINITE, gi);
+          *reinterpret_cast<float4*>(c) = make_float4(v[0], v[1], v[2], v[3]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (gj + e < p.d && gj + e <= gi) {
+              if (p.accumulate) v[e] += c[e];
+              if (!isfinite(v[e])) kq::report(p.info, KQ_ERR_NONFINITE, gi);
+              c[e] = v[e];
+            }
+        }
       }
-      t[rr][tx] = val;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) t[rr][4 * lane + e] = v[e];
     }
     __syncthreads();
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int cc = ty + 8 * k;          // column within the 32-wide block
-      const int64_t gj2 = j0 + cb + cc;   // mirror row
-      const int64_t gi2 = i0 + tx;        // mirror column
-      if (gi2 < p.d && gj2 < p.d && gj2 < gi2) p.C[gj2 * p.ldc + gi2] = t[tx][cc];
+    // mirror: row j0 + h * 128 + c, columns i0 .. i0 + 31 (one per lane)
+    for (int c = warp; c < 128; c += 8) {
+      const int64_t gj2 = j0 + h * 128 + c, gi2 = i0 + lane;
+      if (gi2 < p.d && gj2 < p.d && gj2 < gi2) p.C[gj2 * p.ldc + gi2] = t[lane][c];
     }
     __syncthreads();
   }
@@ -412,6 +468,7 @@ extern "C" kq_status kq_accum_cov(const uint16_t* A, int64_t n, int64_t d, int64
   p.accumulate = accumulate ? 1 : 0;
   p.C = C;
   p.ldc = ldc;
+  p.c_vec = (kq::aligned(C, 16) && !(ldc & 3)) ? 1 : 0;
   p.partial = static_cast<float*>(ws);
   p.info = info;
 
