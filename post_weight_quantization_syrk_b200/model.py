@@ -12,10 +12,17 @@ Order (KronQ paper page, Abstract; KronQ review, Method and Comparison):
     share U and H_X, hence one damped Cholesky factor), then per linear the
     rotation of W and H_G, the blocked OBS solve at its allocated bit-width
     and its Kronecker loss.
-GPU time is taken with CUDA events around each phase; generating the
-synthetic inputs is reported separately and is not part of the quantization
-time.  On several ranks each takes the blocks of dist.shard and the score
-table is merged across ranks before the (identical) allocation.
+In pass 2 the linears of an input group start as soon as its factor is
+ready: the rotations of H_X and the Cholesky factorisations run on the
+caller's stream, each linear's rotations, solve and loss on a second
+stream, so the linears of one group overlap the factorisation of the next
+(the factorisations are a latency-bound chain).  GPU time is the elapsed
+time of pass 1 and of each block of pass 2, taken with CUDA events;
+generating the synthetic inputs is reported separately and is not part of
+it.  Phase seconds are each phase's own event time, summed over its calls
+(with the overlap they add up to more than the GPU time).  On several ranks
+each takes the blocks of dist.shard and the score table is merged across
+ranks before the (identical) allocation.
 """
 from __future__ import annotations
 
@@ -65,12 +72,15 @@ class ModelQuantizer:
     tensors of one block (X per input group, G and W per linear)."""
 
     def __init__(self, make_inputs, make_rht, n_tokens, n_blocks=N_BLOCKS, device="cuda",
-                 choices=(2, 3, 4), avg_bits=3.0, gemm_mode=K.KQ_GEMM_3XTF32, damp=0.01, rank=0, world=1):
+                 choices=(2, 3, 4), avg_bits=3.0, gemm_mode=K.KQ_GEMM_3XTF32, damp=0.01, rank=0, world=1,
+                 overlap=True):
         self.make_inputs, self.make_rht = make_inputs, make_rht
         self.n_tokens, self.n_blocks, self.dev = n_tokens, n_blocks, torch.device(device)
         self.choices, self.avg_bits, self.gemm_mode, self.damp = choices, avg_bits, gemm_mode, damp
         self.info = K.new_info(self.dev)
-        self.ws = K.workspace(256, self.dev)
+        self.overlap = overlap
+        self.ws = K.workspace(256, self.dev)        # calls on the caller's stream
+        self.ws_lin = None                          # calls of the linears (their stream)
         self.phases = {k: Phase() for k in ("statistics", "sensitivity", "rotate", "chol_inv", "quantize", "loss")}
         self.gen_s = 0.0
         self.rank, self.world = rank, world
@@ -80,6 +90,13 @@ class ModelQuantizer:
         if nbytes > self.ws.numel():
             self.ws = K.workspace(nbytes, self.dev)
         return self.ws
+
+    def _ws_lin(self, nbytes):
+        # allocated while the linears' stream is current, so that the caching
+        # allocator ties it to that stream
+        if self.ws_lin is None or nbytes > self.ws_lin.numel():
+            self.ws_lin = K.workspace(nbytes, self.dev)
+        return self.ws_lin
 
     def _timed(self, name, fn):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -104,8 +121,18 @@ class ModelQuantizer:
         bits = K.kq_allocate_bits([full[k][2] for k in keys], n_params, self.choices, self.avg_bits)
         return dict(zip(keys, bits)), full
 
+    def _span_start(self):
+        e = torch.cuda.Event(enable_timing=True)
+        e.record()
+        return e
+
+    def _span_end(self, e0):
+        e1 = torch.cuda.Event(enable_timing=True)
+        e1.record()
+        self._spans.append((e0, e1))
+
     def run(self):
-        self._events = []
+        self._events, self._spans = [], []
         dev = self.dev
         HX, HG, sens = {}, {}, {}
         sens_dev = {}
@@ -115,6 +142,7 @@ class ModelQuantizer:
             inp = self.make_inputs(b, stats_only=True)
             torch.cuda.synchronize()
             self.gen_s += time.perf_counter() - t0
+            span = self._span_start()
             for g, X in inp["X"].items():
                 d = X.shape[1]
                 H = torch.empty((d, d), dtype=torch.float32, device=dev)
@@ -132,6 +160,7 @@ class ModelQuantizer:
                 self._timed("sensitivity",
                             lambda: K.kq_sensitivity(HX[(b, INPUT_OF[lin])], HG[(b, lin)], out))
                 sens_dev[(b, lin)] = out
+            self._span_end(span)
             del inp
         torch.cuda.synchronize()
         K.check_info(self.info, "model statistics")
@@ -142,14 +171,18 @@ class ModelQuantizer:
         mine = [(b, lin) for b in self.blocks for lin in LINEARS]
 
         # ---------------- pass 2: BiIP, Cholesky, solver, loss (this rank's blocks)
+        main = torch.cuda.current_stream(dev)
+        lin_stream = torch.cuda.Stream(device=dev) if self.overlap else main
         results = {}
         for b in self.blocks:
             t0 = time.perf_counter()
             inp = self.make_inputs(b, stats_only=False)
             torch.cuda.synchronize()
             self.gen_s += time.perf_counter() - t0
+            span = self._span_start()
             U = {g: self.make_rht(b, "in:" + g, INPUT_WIDTH[g]) for g in INPUT_WIDTH}
-            Uc, dead = {}, {}
+            Uc, dead, ready = {}, {}, {}
+            # caller's stream: per input group the rotation of H_X and its factor
             for g in INPUT_WIDTH:
                 H = HX.pop((b, g))
                 self._timed("rotate", lambda: (K.kq_rotate(H, K.KQ_AXIS_COLS, U[g]),
@@ -160,37 +193,50 @@ class ModelQuantizer:
                 ws = self._ws(K.kq_chol_inv_workspace_size(n))
                 self._timed("chol_inv", lambda: K.kq_chol_inv(H, self.damp, Uc[g], dead[g], ws, self.info))
                 HX[(b, g)] = H
-            for lin in LINEARS:
-                g = INPUT_OF[lin]
-                d_out, d_in = SHAPE[lin]
-                V = self.make_rht(b, "out:" + lin, d_out)
-                W = inp["W"][lin]
-                Hg = HG.pop((b, lin))
-                self._timed("rotate", lambda: (K.kq_rotate(W, K.KQ_AXIS_COLS, U[g]), K.kq_rotate(W, K.KQ_AXIS_ROWS, V),
-                                               K.kq_rotate(Hg, K.KQ_AXIS_COLS, V),
-                                               K.kq_rotate(Hg, K.KQ_AXIS_ROWS, V)))
-                nb = alloc[(b, lin)]
-                codes = torch.empty((d_out, d_in), dtype=torch.uint8, device=dev)
-                scales = torch.empty((d_out, 1), dtype=torch.float32, device=dev)
-                zeros = torch.empty((d_out, 1), dtype=torch.float32, device=dev)
-                W_hat = torch.empty((d_out, d_in), dtype=torch.float32, device=dev)
-                loss = torch.zeros(1, dtype=torch.float64, device=dev)
-                ws = self._ws(K.kq_quantize_layer_workspace_size(d_out, d_in))
-                self._timed("quantize", lambda: K.kq_quantize_layer(W, Uc[g], dead[g], nb, 0, codes, scales, zeros,
-                                                                     W_hat, gemm_mode=self.gemm_mode, ws=ws,
-                                                                     info=self.info))
-                ws = self._ws(K.kq_kron_loss_workspace_size(d_out, d_in))
-                self._timed("loss", lambda: K.kq_kron_loss(W, W_hat, HX[(b, g)], Hg, loss, ws))
-                results[(b, lin)] = {"bits": nb, "loss": loss, "codes_bytes": codes.numel()}
-                del Hg, codes, W_hat
+                ready[g] = torch.cuda.Event()
+                ready[g].record(main)
+            # linears' stream: each linear once its group's factor is ready.
+            # Everything allocated here belongs to this stream; what the
+            # caller's stream allocated is freed only after the join below.
+            with torch.cuda.stream(lin_stream):
+                for lin in LINEARS:
+                    g = INPUT_OF[lin]
+                    lin_stream.wait_event(ready[g])
+                    d_out, d_in = SHAPE[lin]
+                    V = self.make_rht(b, "out:" + lin, d_out)
+                    W = inp["W"][lin]
+                    Hg = HG.pop((b, lin))
+                    self._timed("rotate", lambda: (K.kq_rotate(W, K.KQ_AXIS_COLS, U[g]),
+                                                   K.kq_rotate(W, K.KQ_AXIS_ROWS, V),
+                                                   K.kq_rotate(Hg, K.KQ_AXIS_COLS, V),
+                                                   K.kq_rotate(Hg, K.KQ_AXIS_ROWS, V)))
+                    nb = alloc[(b, lin)]
+                    codes = torch.empty((d_out, d_in), dtype=torch.uint8, device=dev)
+                    scales = torch.empty((d_out, 1), dtype=torch.float32, device=dev)
+                    zeros = torch.empty((d_out, 1), dtype=torch.float32, device=dev)
+                    W_hat = torch.empty((d_out, d_in), dtype=torch.float32, device=dev)
+                    loss = torch.zeros(1, dtype=torch.float64, device=dev)
+                    ws = self._ws_lin(max(K.kq_quantize_layer_workspace_size(d_out, d_in),
+                                          K.kq_kron_loss_workspace_size(d_out, d_in)))
+                    self._timed("quantize", lambda: K.kq_quantize_layer(W, Uc[g], dead[g], nb, 0, codes, scales,
+                                                                         zeros, W_hat, gemm_mode=self.gemm_mode,
+                                                                         ws=ws, info=self.info))
+                    self._timed("loss", lambda: K.kq_kron_loss(W, W_hat, HX[(b, g)], Hg, loss, ws))
+                    results[(b, lin)] = {"bits": nb, "loss": loss, "codes_bytes": codes.numel()}
+                    del Hg, codes, W_hat
+            if lin_stream is not main:
+                done = torch.cuda.Event()
+                done.record(lin_stream)
+                main.wait_event(done)
+            self._span_end(span)
             for g in INPUT_WIDTH:
                 del HX[(b, g)]
-            del inp, Uc, dead
+            del inp, U, Uc, dead
         torch.cuda.synchronize()
         K.check_info(self.info, "model quantization")
         for name, e0, e1 in self._events:
             self.phases[name].add(e0, e1)
-        total_ms = sum(p.ms for p in self.phases.values())
+        total_ms = sum(e0.elapsed_time(e1) for e0, e1 in self._spans)
         # the job's GPU time is the slowest rank's
         total_s = D.all_max(total_ms / 1e3, self.dev)
         n_weights = sum(SHAPE[lin][0] * SHAPE[lin][1] for _, lin in keys)

@@ -33,3 +33,19 @@ def test_one_block_model():
         assert math.isfinite(x["loss"]) and x["loss"] > 0
         assert abs(x["score"] - x["tr_X"] * x["tr_G"]) <= 1e-12 * abs(x["score"])
     assert r["gpu_seconds"] > 0
+
+
+def test_overlapped_linears_match_sequential():
+    """Pass 2 runs each linear on a second stream once its input group's
+    factor is ready; two blocks (buffers freed and reused across the join)
+    must give exactly the bits and losses of the one-stream order."""
+    if not torch.cuda.is_available():
+        pytest.fail("needs a CUDA GPU")
+    from post_weight_quantization_syrk_b200.model import synthetic_model
+    a = synthetic_model(n_tokens=2048, n_blocks=2, overlap=True).run()
+    b = synthetic_model(n_tokens=2048, n_blocks=2, overlap=False).run()
+    assert len(a["per_linear"]) == len(b["per_linear"]) == 14
+    for x, y in zip(a["per_linear"], b["per_linear"]):
+        assert (x["block"], x["linear"], x["bits"]) == (y["block"], y["linear"], y["bits"])
+        assert x["loss"] == y["loss"], (x, y)
+    assert a["gpu_seconds"] > 0 and b["gpu_seconds"] > 0
