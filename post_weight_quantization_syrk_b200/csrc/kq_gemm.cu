@@ -4,9 +4,10 @@
 // fp32 accuracy at tensor-core speed: each fp32 operand x is split into its
 // tf32 rounding b = tf32(x) and the remainder s = x - b (exact in fp32), and
 // A B ~ Ab Bb + Ab Bs + As Bb: the dropped As Bs term and the tf32 reading of
-// the remainders are ~2^-22 relative.  The products the path needs (dW H_X,
-// H_G dW for the Kronecker loss, E Uc for the solver's trailing update) lose
-// up to ~60x to cancellation, which rules out plain TF32 or bf16 there.
+// the remainders are ~2^-22 relative.  The products the path needs (dW H1^T
+// and its product with dW^T for the Kronecker loss, E Uc for the solver's
+// trailing update) lose up to ~60x to cancellation, which rules out plain
+// TF32 or bf16 there.
 //
 // Structure (same as the covariance SYRK): persistent CTAs, one per SM, walk
 // the output tiles in one of two shapes chosen per launch: wide tiles of
