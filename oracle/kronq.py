@@ -44,6 +44,7 @@ __all__ = [
     "chol_inv_reversed", "fit_grid", "quantize_codes", "dequantize",
     "QuantResult", "quantize_layer", "kron_loss", "gptq_loss",
     "allocate_bits", "budget_units", "quantize_linear",
+    "pack_codes", "unpack_codes", "dequantize_layer", "reverted_apply",
 ]
 
 
@@ -458,3 +459,87 @@ def quantize_linear(W, X, G, T_in, T_out, bits, group=0, block=128, damp_frac=0.
         "Uc": Uc, "dead": dead, "lam": lam, "quant": q,
         "loss": kron_loss(Wp, q.W_hat, HXp, HGp), "loss_gptq": gptq_loss(Wp, q.W_hat, HXp),
     }
+
+
+# ---------------------------------------------------------------------------
+# Inference side: packed codes and the online reversion of U and V
+# ---------------------------------------------------------------------------
+
+def pack_codes(codes, bits):
+    """The codes of a [rows, cols] layer packed `bits` bits each into uint32.
+
+    [REV] Limitations (third limitation): inference runs from the low-bit
+    weights and reverts the orthogonal transforms online; the pages give no
+    storage format.  Reading R15: each row is padded with zero codes to a
+    multiple of 32; the 32 codes of group g of a row fill `bits` consecutive
+    32-bit words (row r, words g*bits .. g*bits + bits - 1), code k of the
+    group at bits bits*k .. bits*k + bits - 1 of the group's little-endian
+    bit stream (word w of the group holds stream bits 32w .. 32w + 31).
+    Returns uint32 [rows, ceil(cols / 32) * bits].
+    """
+    codes = np.asarray(codes)
+    if codes.ndim != 2:
+        raise ValueError("codes must be [rows, cols]")
+    bits = int(bits)
+    if not 1 <= bits <= 8:
+        raise ValueError("bits must be 1..8")
+    if codes.size and (codes.min() < 0 or codes.max() >= (1 << bits)):
+        raise ValueError("a code does not fit in the bit-width")
+    rows, cols = codes.shape
+    groups = -(-cols // 32)
+    out = np.zeros((rows, groups * bits), dtype=np.uint32)
+    c = np.arange(cols)
+    r = np.arange(rows)[:, None]
+    q = codes.astype(np.uint32)
+    for t in range(bits):                      # bit t of every code
+        pos = bits * (c % 32) + t              # its place in the group's stream
+        word = (c // 32) * bits + pos // 32
+        one = ((q >> np.uint32(t)) & np.uint32(1)) << (pos % 32).astype(np.uint32)
+        np.bitwise_or.at(out, (np.broadcast_to(r, q.shape), np.broadcast_to(word, q.shape)), one)
+    return out
+
+
+def unpack_codes(packed, bits, cols):
+    """Inverse of pack_codes: uint8 codes [rows, cols] (the padding dropped)."""
+    packed = np.asarray(packed, dtype=np.uint32)
+    bits = int(bits)
+    rows = packed.shape[0]
+    if packed.shape[1] != -(-cols // 32) * bits:
+        raise ValueError("packed width does not match cols and bits")
+    c = np.arange(cols)
+    codes = np.zeros((rows, cols), dtype=np.uint32)
+    for t in range(bits):
+        pos = bits * (c % 32) + t
+        word = (c // 32) * bits + pos // 32
+        bit = (packed[:, word] >> (pos % 32).astype(np.uint32)) & np.uint32(1)
+        codes |= bit << np.uint32(t)
+    return codes.astype(np.uint8)
+
+
+def dequantize_layer(codes, scales, zeros, group=0):
+    """W_hat[r, c] = scale[r, g] * (code[r, c] - zero[r, g]), g = 0 per channel
+    or c // group for grouped grids (the solver's grid layout)."""
+    codes = np.asarray(codes, dtype=np.float64)
+    scales = np.asarray(scales, dtype=np.float64)
+    zeros = np.asarray(zeros, dtype=np.float64)
+    rows, cols = codes.shape
+    g = np.zeros(cols, dtype=np.int64) if not group else np.arange(cols) // int(group)
+    return scales.reshape(rows, -1)[:, g] * (codes - zeros.reshape(rows, -1)[:, g])
+
+
+def reverted_apply(packed, scales, zeros, bits, group, T_in, T_out, x):
+    """y = V^T (W_hat' (U x)) for x [d_in] or [d_in, B]: the quantized layer in
+    the rotated basis applied between the forward input rotation U = T_in and
+    the reverted output rotation V^T = T_out^T.
+
+    [REV] Method (1): W' = V W U^T, so V^T W' U = W and the layer keeps its
+    function; Limitations (third limitation): at inference U and V are
+    reverted online, Theta(d_in log d_in + d_out log d_out) per layer with the
+    fast transform (applied here as dense float64 matrices).
+    """
+    T_in = np.asarray(T_in, dtype=np.float64)
+    T_out = np.asarray(T_out, dtype=np.float64)
+    codes = unpack_codes(packed, bits, T_in.shape[0])
+    W_hat = dequantize_layer(codes, scales, zeros, group)
+    xr = T_in @ np.asarray(x, dtype=np.float64)
+    return T_out.T @ (W_hat @ xr)
