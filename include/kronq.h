@@ -335,6 +335,41 @@ kq_status kq_allocate_bits(const double* sens, const int64_t* n_params, int n_la
                            const int* choices, int n_choices, double avg_bits,
                            int* bits_out);
 
+/* --------------------------------------------------------------------------
+ * Inference side: packed codes and the matvec with U and V reverted online.
+ *
+ * KronQ review, Limitations (third limitation): at inference the orthogonal
+ * transforms U and V are reverted online, Theta(d_in log d_in + d_out log
+ * d_out) per layer; Method (1): W' = V W U^T, so V^T W_hat' U stands for the
+ * layer.  The pages give no packed format; this one: each row padded with
+ * zero codes to a multiple of 32, the 32 codes of a group in `bits`
+ * consecutive 32-bit words (row r, words g*bits .. g*bits + bits - 1), code
+ * k of the group at bits bits*k .. bits*k + bits - 1 of the group's
+ * little-endian bit stream.
+ *
+ * kq_pack_codes: uint8 codes [rows, cols] (ldq >= cols) -> uint32 packed
+ *   [rows, ceil(cols/32) * bits] (ldp >= that), 1 <= bits <= 8.  A code that
+ *   does not fit in `bits` is masked and reported in `info`
+ *   (KQ_ERR_INVALID_ARG, index = row).
+ * kq_reverted_matvec: Y[b, :] = V^T (W_hat' (U X[b, :])) for b < batch
+ *   (1..8), W_hat'[r, c] = scales[r, g] (code[r, c] - zeros[r, g]) with
+ *   g = 0 (group == 0, scales/zeros [d_out, 1]) or c / group (group a
+ *   multiple of 32, [d_out, ceil(d_in/group)]), i.e. the layout
+ *   kq_quantize_layer writes.  T_in (order d_in) / T_out (order d_out) as
+ *   for kq_rotate; NULL means the identity (the plain dequantized matvec).
+ *   X fp32 [batch, d_in] (ldx >= d_in), Y fp32 [batch, d_out] (ldy >=
+ *   d_out; 16-byte aligned with ldy % 4 == 0 when T_out is given).
+ *   ws: kq_reverted_matvec_workspace_size(d_in, batch) bytes.
+ * ------------------------------------------------------------------------ */
+kq_status kq_pack_codes(const uint8_t* codes, int64_t rows, int64_t cols, int64_t ldq, int bits,
+                        uint32_t* packed, int64_t ldp, int32_t* info, kq_stream_t stream);
+size_t kq_reverted_matvec_workspace_size(int64_t d_in, int batch);
+kq_status kq_reverted_matvec(const uint32_t* packed, int64_t d_out, int64_t d_in, int64_t ldp, int bits,
+                             const float* scales, const float* zeros, int group,
+                             const kq_rht* T_in, const kq_rht* T_out,
+                             const float* X, int64_t ldx, int batch, float* Y, int64_t ldy,
+                             void* ws, size_t ws_bytes, kq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

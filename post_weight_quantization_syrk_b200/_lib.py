@@ -29,6 +29,7 @@ KQ_GEMM_FP32, KQ_GEMM_3XTF32 = 0, 1
 EXPORTS = (
     "kq_status_string", "kq_last_error", "kq_version", "kq_launch_count",
     "kq_accum_cov_workspace_size", "kq_accum_cov",
+    "kq_pack_codes", "kq_reverted_matvec_workspace_size", "kq_reverted_matvec",
     "kq_sensitivity",
     "kq_rotate",
     "kq_chol_inv_workspace_size", "kq_chol_inv",
@@ -78,6 +79,10 @@ _SIGS = {
                                   ctypes.POINTER(_vp), _vp, _sz, _vp]),
     "kq_kron_loss": (_i32, [_vp, _i64, _vp, _i64, _i64, _i64, _vp, _i64, _vp, _i64, _vp, _vp, _sz, _vp]),
     "kq_kron_loss_noalloc": (_i32, [_vp, _i64, _vp, _i64, _i64, _i64, _vp, _i64, _vp, _i64, _vp, _vp]),
+    "kq_pack_codes": (_i32, [_vp, _i64, _i64, _i64, _i32, _vp, _i64, _vp, _vp]),
+    "kq_reverted_matvec_workspace_size": (_sz, [_i64, _i32]),
+    "kq_reverted_matvec": (_i32, [_vp, _i64, _i64, _i64, _i32, _vp, _vp, _i32, ctypes.POINTER(kq_rht),
+                                  ctypes.POINTER(kq_rht), _vp, _i64, _i32, _vp, _i64, _vp, _sz, _vp]),
     "kq_allocate_bits": (_i32, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), _i32,
                                 ctypes.POINTER(ctypes.c_int), _i32, _f64, ctypes.POINTER(ctypes.c_int)]),
 }
@@ -354,3 +359,49 @@ def kq_allocate_bits(sens, n_params, choices=(2, 3, 4), avg_bits=3.0):
     out = (ctypes.c_int * max(k, 1))()
     _check(load().kq_allocate_bits(s, n, k, c, len(choices), float(avg_bits), out), "kq_allocate_bits")
     return [int(out[i]) for i in range(k)]
+
+
+def kq_pack_codes(codes, bits, packed=None, info=None, stream=None):
+    """uint8 codes [rows, cols] -> packed words [rows, ceil(cols / 32) * bits]
+    (int32 storage of the uint32 words; layout in kronq.h)."""
+    ldq = _mat(codes, torch.uint8, "codes")
+    rows, cols = codes.shape
+    words = -(-cols // 32) * int(bits)
+    if packed is None:
+        packed = torch.empty((rows, words), dtype=torch.int32, device=codes.device)
+    ldp = _mat(packed, torch.int32, "packed")
+    if packed.shape[0] != rows or packed.shape[1] < words:
+        raise ValueError("packed must be [rows, >= ceil(cols / 32) * bits]")
+    if info is None:
+        info = new_info(codes.device)
+    _check(load().kq_pack_codes(_ptr(codes), rows, cols, ldq, int(bits), _ptr(packed), ldp, _ptr(info),
+                                _stream(stream)), "kq_pack_codes")
+    return packed
+
+
+def kq_reverted_matvec_workspace_size(d_in: int, batch: int) -> int:
+    return int(load().kq_reverted_matvec_workspace_size(int(d_in), int(batch)))
+
+
+def kq_reverted_matvec(packed, bits, scales, zeros, group, T_in, T_out, X, Y, ws=None, stream=None):
+    """Y = V^T (W_hat' (U X^T))^T for X [batch, d_in]: the packed layer with its
+    rotations reverted (T_in / T_out None: the identity)."""
+    ldp = _mat(packed, torch.int32, "packed")
+    ldx = _mat(X, torch.float32, "X")
+    ldy = _mat(Y, torch.float32, "Y")
+    batch, d_in = X.shape
+    d_out = Y.shape[1]
+    if Y.shape[0] != batch or packed.shape[0] != d_out:
+        raise ValueError("X [batch, d_in], Y [batch, d_out], packed [d_out, words]")
+    for t, nm in ((scales, "scales"), (zeros, "zeros")):
+        if t.dtype != torch.float32 or not t.is_contiguous() or not t.is_cuda:
+            raise TypeError(f"{nm} must be a contiguous CUDA float32 tensor")
+    if ws is None:
+        ws = workspace(kq_reverted_matvec_workspace_size(d_in, batch), X.device)
+    wp, wb = _buf(ws)
+    _check(load().kq_reverted_matvec(_ptr(packed), d_out, d_in, ldp, int(bits), _ptr(scales), _ptr(zeros), int(group),
+                                     None if T_in is None else ctypes.byref(T_in.c),
+                                     None if T_out is None else ctypes.byref(T_out.c),
+                                     _ptr(X), ldx, batch, _ptr(Y), ldy, wp, wb, _stream(stream)),
+           "kq_reverted_matvec")
+    return Y
