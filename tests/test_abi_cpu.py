@@ -171,3 +171,31 @@ def test_multi_entry_points_validate_before_enqueue():
     st = lib.kq_quantize_layer_multi(dummy, 4, 128, 128, dummy, 128, None, 2, bits, groups, 128, 0, arr, 128, arr,
                                      arr, shared, 128, dummy, 1 << 30, dummy, None)
     assert st == 1 and b"share an output" in lib.kq_last_error()
+
+
+def test_inference_entry_points_validate_before_enqueue():
+    """Host-side rejections of kq_pack_codes / kq_reverted_matvec (nothing is
+    launched: every check fails before a CUDA call)."""
+    import ctypes
+    lib = P.load()
+    vp = ctypes.c_void_p
+    d = vp(256)   # never dereferenced
+    # kq_pack_codes: NULL codes, bits outside 1..8, packed row too short
+    assert lib.kq_pack_codes(None, 4, 64, 64, 4, d, 8, d, None) == 1
+    assert lib.kq_pack_codes(d, 4, 64, 64, 9, d, 18, d, None) == 1
+    st = lib.kq_pack_codes(d, 4, 64, 64, 3, d, 5, d, None)      # needs 2 groups x 3 words
+    assert st == 1 and b"leading dimension" in lib.kq_last_error()
+    # kq_reverted_matvec
+    T_ok = K.kq_rht(64, 6, 1, 256, None)
+    T_bad = K.kq_rht(32, 5, 1, 256, None)
+    def call(bits=4, group=0, batch=1, T_in=T_ok, ws_bytes=1 << 20, ldp=8):
+        return lib.kq_reverted_matvec(d, 16, 64, ldp, bits, d, d, group, ctypes.byref(T_in), None, d, 64, batch, d,
+                                      16, d, ws_bytes, None)
+    assert call(bits=0) == 1
+    assert call(batch=9) == 2 and b"batch" in lib.kq_last_error()
+    assert call(group=48) == 2
+    assert call(T_in=T_bad) == 1 and b"rotation order" in lib.kq_last_error()
+    assert call(ldp=7) == 1
+    assert call(ws_bytes=16) == 4
+    assert P.kq_reverted_matvec_workspace_size(64, 3) >= 3 * 64 * 4
+    assert P.kq_reverted_matvec_workspace_size(0, 1) == 0
