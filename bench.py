@@ -274,7 +274,7 @@ def run_kronq(a):
 # ncu capture summarised in profiles/syrk_tc_kernel_attn4096_traffic.md; valid
 # only for the kernel sources it was taken on.
 SYRK_TRAFFIC = {"attn4096": 5.00e9}
-SYRK_SOURCE_SHA = {"kq_syrk.cu": "3097a3ef9da3a5d7", "kq_tc.cuh": "f59b54090d782541"}
+SYRK_SOURCE_SHA = {"kq_syrk.cu": "219987dcfe1d0668", "kq_tc.cuh": "f59b54090d782541"}
 
 
 def syrk_traffic(workload):

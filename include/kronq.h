@@ -210,7 +210,7 @@ kq_status kq_chol_inv(const float* H, int64_t n, int64_t ldh, float damp_frac,
  *   gemm_mode trailing-update precision: KQ_GEMM_FP32 (SIMT fp32) or
  *            KQ_GEMM_3XTF32 (tcgen05 tensor cores, operands split into tf32 +
  *            remainder, fp32-level accuracy).
- *   codes    uint8 [d_out, d_in], ldq >= d_in.
+ *   codes    uint8 [d_out, d_in], ldq >= d_in; 4-byte aligned, ldq % 4 == 0.
  *   scales, zeros  fp32 [d_out, n_groups], n_groups = 1 or ceil(d_in / group).
  *   W_hat    fp32 [d_out, d_in] dequantized weights (rotated coordinates),
  *            ldwh >= d_in; also used as the running copy of W.

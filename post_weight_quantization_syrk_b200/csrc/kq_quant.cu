@@ -431,7 +431,10 @@ kq_status check_args(const float* W, int64_t d_out, int64_t d_in, int64_t ldw, c
     return kq::fail(KQ_ERR_INVALID_ARG, "kq_quantize_layer: gemm_mode must be KQ_GEMM_FP32 or KQ_GEMM_3XTF32");
   if (W == W_hat) return kq::fail(KQ_ERR_INVALID_ARG, "kq_quantize_layer: W and W_hat must not alias");
   if (!kq::aligned(W, 16) || !kq::aligned(W_hat, 16) || !kq::aligned(Uc, 16) || (ldw & 3) || (ldwh & 3) || (lduc & 3))
-    return kq::fail(KQ_ERR_ALIGNMENT, "kq_quantize_layer: W, W_hat, Uc need 16-byte alignment and ld % 4 == 0");
+    return kq::fail(KQ_ERR_ALIGNMENT, "kq_quantize_layer: W, W_hat, Uc need 16-byte alignment and ld %% 4 == 0");
+  // the in-block kernel stores four codes at a time
+  if (!kq::aligned(codes, 4) || (ldq & 3))
+    return kq::fail(KQ_ERR_ALIGNMENT, "kq_quantize_layer: codes need 4-byte alignment and ldq %% 4 == 0");
   return KQ_OK;
 }
 

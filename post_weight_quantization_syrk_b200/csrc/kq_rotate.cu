@@ -346,7 +346,7 @@ extern "C" kq_status kq_rotate(float* M, int64_t rows, int64_t cols, int64_t ld,
   if (n != (axis == KQ_AXIS_ROWS ? rows : cols))
     return kq::fail(KQ_ERR_INVALID_ARG, "kq_rotate: T->n does not match the rotated dimension");
   if (!kq::aligned(M, 16) || (ld & 3) || !kq::aligned(T->signs, 16))
-    return kq::fail(KQ_ERR_ALIGNMENT, "kq_rotate: M and signs must be 16-byte aligned and ld % 4 == 0");
+    return kq::fail(KQ_ERR_ALIGNMENT, "kq_rotate: M and signs must be 16-byte aligned and ld %% 4 == 0");
   if (rows == 0 || cols == 0) return KQ_OK;
   cudaStream_t st = (cudaStream_t)stream;
   const int p = 1 << lp;

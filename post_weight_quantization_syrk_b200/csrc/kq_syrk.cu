@@ -438,7 +438,7 @@ extern "C" kq_status kq_accum_cov(const uint16_t* A, int64_t n, int64_t d, int64
   if (n > ((int64_t)1 << 31) - BK) return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_accum_cov: n above 2^31 - 64");
   if (lda < d || ldc < d) return kq::fail(KQ_ERR_INVALID_ARG, "kq_accum_cov: leading dimension too small");
   if ((n > 0 && !kq::aligned(A, 16)) || (lda & 7))
-    return kq::fail(KQ_ERR_ALIGNMENT, "kq_accum_cov: A 16-byte aligned, lda % 8 == 0");
+    return kq::fail(KQ_ERR_ALIGNMENT, "kq_accum_cov: A 16-byte aligned, lda %% 8 == 0");
   if (!isfinite(alpha)) return kq::fail(KQ_ERR_INVALID_ARG, "kq_accum_cov: alpha not finite");
   cudaStream_t st = (cudaStream_t)stream;
   if (n == 0) {

@@ -199,3 +199,21 @@ def test_inference_entry_points_validate_before_enqueue():
     assert call(ws_bytes=16) == 4
     assert P.kq_reverted_matvec_workspace_size(64, 3) >= 3 * 64 * 4
     assert P.kq_reverted_matvec_workspace_size(0, 1) == 0
+
+
+def test_code_buffer_alignment_and_message_text():
+    """The solver stores four codes at a time: a code buffer that is not
+    4-byte aligned, or whose ldq is not a multiple of 4, is refused before
+    anything is enqueued; error texts render their percent signs literally."""
+    import ctypes
+    lib = P.load()
+    vp = ctypes.c_void_p
+    d = vp(256)
+    def quant(codes, ldq):
+        return lib.kq_quantize_layer(d, 4, 128, 128, d, 128, None, 3, 0, 128, 0, codes, ldq, d, d, vp(512), 128, d,
+                                     1 << 30, d, None)
+    assert quant(vp(258), 128) == 3 and b"ldq % 4 == 0" in lib.kq_last_error()
+    assert quant(vp(256), 129) == 3
+    T = K.kq_rht(4, 2, 1, 256, None)
+    st = lib.kq_rotate(vp(4), 4, 4, 4, P.KQ_AXIS_COLS, ctypes.byref(T), 0, None)
+    assert st == 3 and b"ld % 4 == 0" in lib.kq_last_error()
