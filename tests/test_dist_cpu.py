@@ -1,4 +1,4 @@
-"""The multi-rank plumbing on CPU (gloo, world size 2): blocks of the
+"""The multi-rank plumbing on CPU (gloo, world sizes 2 and 3): blocks of the
 7B-shaped model are sharded over ranks without overlap, each rank fills the
 sensitivity table for its own blocks, the merged table gives every rank the
 same bit allocation as one process with the whole table, and the job's time
@@ -46,8 +46,8 @@ def _worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_two_rank_sharding_and_allocation():
-    world = 2
+@pytest.mark.parametrize("world", [2, 3])
+def test_rank_sharding_and_allocation(world):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
@@ -60,9 +60,11 @@ def test_two_rank_sharding_and_allocation():
         assert p.exitcode == 0
     out.sort()
     blocks = [o[1] for o in out]
-    assert sorted(blocks[0] + blocks[1]) == list(range(N_BLOCKS)) and not set(blocks[0]) & set(blocks[1])
-    # both ranks see the full table and allocate identically
-    assert out[0][2] == out[1][2] and out[0][3] == out[1][3]
+    # every block on exactly one rank
+    assert sorted(b for bl in blocks for b in bl) == list(range(N_BLOCKS))
+    assert all(not set(blocks[i]) & set(blocks[j]) for i in range(world) for j in range(i))
+    # every rank sees the full table and allocates identically
+    assert all(o[2] == out[0][2] and o[3] == out[0][3] for o in out)
     # ... and that allocation equals a single process's from the whole table
     from post_weight_quantization_syrk_b200.model import LINEARS, ModelQuantizer
     single = ModelQuantizer(None, None, n_tokens=1, n_blocks=N_BLOCKS, device="cpu")
@@ -70,4 +72,4 @@ def test_two_rank_sharding_and_allocation():
     assert out[0][2] == sorted(alloc1.items())
     assert all(abs(a[1][2] - b[1][2]) == 0 for a, b in zip(out[0][3], sorted(full1.items())))
     # the job's time is the slowest rank's
-    assert out[0][4] == out[1][4] == 20.0
+    assert all(o[4] == 10.0 * world for o in out)
