@@ -1,7 +1,8 @@
 """Latency of the inference-side matvec with U and V reverted online against
 the same packed matvec without rotations.
 
-    python -m post_weight_quantization_syrk_b200.infer_bench
+    python -m post_weight_quantization_syrk_b200.infer_bench    (from the repository root:
+                                                                it draws the rotations with synth/)
 
 For each layer shape of the 7B model (4-bit, per-channel grid) and batch 1
 and 8, it cycles through 24 distinct packed layers (more bytes than L2, so
