@@ -87,6 +87,18 @@ int kq_version(void);
  * (all host threads); a diagnostic for counting device work per step. */
 unsigned long long kq_launch_count(void);
 
+/* Time limit of the device waits in the tensor-core kernels (kq_accum_cov,
+ * and the products inside kq_quantize_layer and kq_kron_loss): a pipeline
+ * wait that has not completed after `ns` nanoseconds gives up, the kernel
+ * records KQ_ERR_TIMEOUT in `info` (index = the wait's site), lets its own
+ * copies and products finish (with the fixed default bound), frees its
+ * tensor memory and returns.  ns == 0 makes a wait give up at the first poll
+ * that finds it incomplete: a test of this failure path, whose results are
+ * then garbage.  Process-wide, read by each call when it enqueues; returns
+ * the previous limit.  Default KQ_WAIT_LIMIT_DEFAULT_NS (4 s). */
+#define KQ_WAIT_LIMIT_DEFAULT_NS 4000000000ull
+unsigned long long kq_set_wait_limit_ns(unsigned long long ns);
+
 /* --------------------------------------------------------------------------
  * kq_accum_cov - covariance accumulation (steps a1/a2).
  *
@@ -294,16 +306,18 @@ kq_status kq_kron_loss_multi(const float* W, int64_t ldw, int count, const float
  * that cannot allocate device memory: code embedded in a host application
  * that owns every device allocation through its own pool, or a latency-bound
  * loop where the implicit synchronisation of cudaMalloc/cudaFree is not
- * acceptable.  It computes the same loss (all of H_X and H_G read, no
- * symmetry assumed) with an fp32 CUDA-core kernel that forms one 64 x 64 tile
- * of dW H_X and of H_G dW per CTA, and keeps the per-tile partial sums in a
+ * acceptable.  It computes the same loss with an fp32 CUDA-core kernel that
+ * forms one 64 x 64 tile of dW H_X and of H_G^T dW per CTA and sums their
+ * elementwise product, which is tr(dW H_X dW^T H_G) exactly for any H_X and
+ * H_G (all of both read, no symmetry assumed), and keeps the per-tile partial sums in a
  * fixed array inside the library (static device memory: KQ_KRON_LOSS_NOALLOC_MAX_TILES fp64
  * values, 512 KiB, held by every GPU that loads the library until the
  * process exits).  It calls no cudaMalloc, cudaFree or allocating routine.
  *
  *   Arguments as kq_kron_loss, without ws/ws_bytes.
  *   Limit: ceil(d_out / 64) * ceil(d_in / 64) <= KQ_KRON_LOSS_NOALLOC_MAX_TILES
- *          (e.g. 8192 x 28672 fits); larger layers get KQ_ERR_UNSUPPORTED_SHAPE.
+ *          (e.g. 8192 x 28672 fits) and ceil(d_out / 64) <= 65535; larger
+ *          layers get KQ_ERR_UNSUPPORTED_SHAPE.
  *   The stream must belong to the current device.  The first call on a
  *   device looks up the array's device address (cudaGetSymbolAddress) with
  *   that device current; make that first call before any stream capture.

@@ -447,7 +447,14 @@ def allocate_bits(sens, n_params, choices=(2, 3, 4), avg_bits=3.0):
 
 def quantize_linear(W, X, G, T_in, T_out, bits, group=0, block=128, damp_frac=0.01):
     """Covariances -> sensitivity -> BiIP -> damped Cholesky of the inverse ->
-    blocked OBS -> Kronecker loss, all in float64 from the same inputs."""
+    blocked OBS -> Kronecker loss, all in float64 from the same inputs.
+
+    Pinned as a whole (tests/test_oracle_linear_pins.py) by quantities formed
+    by other routes: the loss against the sample double sum
+    (1/N^2) sum_{t,s} (g_t^T dW x_s)^2 with dW = W - V^T W_hat' U in original
+    coordinates, the factor against the residual of the rotated covariance
+    formed by loops, the rotated weights by function preservation, and a
+    dead-column case."""
     H_X = covariance(X)
     H_G = covariance(G)
     sens = sensitivity(H_X, H_G)

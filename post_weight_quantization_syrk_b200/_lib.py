@@ -27,7 +27,7 @@ KQ_GEMM_FP32, KQ_GEMM_3XTF32 = 0, 1
 
 # Every symbol the header declares.
 EXPORTS = (
-    "kq_status_string", "kq_last_error", "kq_version", "kq_launch_count",
+    "kq_status_string", "kq_last_error", "kq_version", "kq_launch_count", "kq_set_wait_limit_ns",
     "kq_accum_cov_workspace_size", "kq_accum_cov",
     "kq_pack_codes", "kq_reverted_matvec_workspace_size", "kq_reverted_matvec",
     "kq_sensitivity",
@@ -60,6 +60,7 @@ _SIGS = {
     "kq_last_error": (ctypes.c_char_p, []),
     "kq_version": (_i32, []),
     "kq_launch_count": (ctypes.c_ulonglong, []),
+    "kq_set_wait_limit_ns": (ctypes.c_ulonglong, [ctypes.c_ulonglong]),
     "kq_accum_cov_workspace_size": (_sz, [_i64, _i64]),
     "kq_accum_cov": (_i32, [_vp, _i64, _i64, _i64, _vp, _i64, _f32, _i32, _vp, _sz, _vp, _vp]),
     "kq_sensitivity": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _vp, _vp]),
@@ -405,3 +406,13 @@ def kq_reverted_matvec(packed, bits, scales, zeros, group, T_in, T_out, X, Y, ws
                                      _ptr(X), ldx, batch, _ptr(Y), ldy, wp, wb, _stream(stream)),
            "kq_reverted_matvec")
     return Y
+
+
+KQ_WAIT_LIMIT_DEFAULT_NS = 4_000_000_000
+
+
+def kq_set_wait_limit_ns(ns):
+    """Set the time limit of the tensor-core kernels' device waits (process
+    wide); 0 makes a wait give up at its first incomplete poll.  Returns the
+    previous limit."""
+    return int(load().kq_set_wait_limit_ns(int(ns)))

@@ -66,6 +66,7 @@ struct Params {
   int other_vec;   // `other` rows can be read as float4 (16-byte aligned rows)
   double* partial;
   int32_t* info;
+  unsigned long long wait_ns;   // limit of each pipeline wait (kq_set_wait_limit_ns)
 };
 
 // Operand layout in shared memory (K-major): one 16 (k) x 256 TMA box per
@@ -164,7 +165,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
         walk.at(p, bm, t, tm, tn, rb);
         const int m0 = tm * bm, n0 = tn * BN;
         for (int kb = 0; kb < p.kblocks; ++kb) {
-          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.info, 11)) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.info, 11, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -199,10 +200,10 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       int local = 0;
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++local) {
         const int buf = p.wide ? 0 : (local & 1);
-        if (!mbar_wait(accempty0 + 8 * buf, ((acc_bits >> buf) & 1u) ^ 1u, abort_flag, p.info, 12)) break;
+        if (!mbar_wait(accempty0 + 8 * buf, ((acc_bits >> buf) & 1u) ^ 1u, abort_flag, p.info, 12, p.wait_ns)) break;
         fence_after();
         for (int kb = 0; kb < p.kblocks; ++kb) {
-          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, p.info, 13)) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, p.info, 13, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -256,7 +257,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       const int64_t m0 = (int64_t)tm * bm, n0 = (int64_t)tn * BN;
       // one lane waits, the warp follows: every lane leaves together on abort
       bool ready = true;
-      if (lane == 0) ready = mbar_wait(accfull0 + 8 * buf, (acc_bits >> buf) & 1u, abort_flag, p.info, 14);
+      if (lane == 0) ready = mbar_wait(accfull0 + 8 * buf, (acc_bits >> buf) & 1u, abort_flag, p.info, 14, p.wait_ns);
       if (!__shfl_sync(0xffffffffu, ready ? 1 : 0, 0)) break;
       __syncwarp();
       fence_after();
@@ -499,6 +500,7 @@ kq_status gemm_3xtf32(const Gemm3xTF32& g, cudaStream_t st) {
   p.other_vec = (g.other && aligned(g.other, 16) && !(g.ld_other & 3)) ? 1 : 0;
   p.partial = g.partial;
   p.info = g.info;
+  p.wait_ns = kq::wait_limit_ns();
   if (g.upper && (g.M != g.N || g.epilogue != kEpiDot))
     return fail(KQ_ERR_INVALID_ARG, "gemm: the upper block triangle needs M == N and the dot epilogue");
   if (g.epilogue == kEpiDot) {

@@ -28,6 +28,9 @@ void clear_error() { g_last_error[0] = 0; }
 static std::atomic<unsigned long long> g_launches{0};
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
+static std::atomic<unsigned long long> g_wait_limit_ns{KQ_WAIT_LIMIT_DEFAULT_NS};
+unsigned long long wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
+
 kq_status fail(kq_status s, const char* fmt, ...) {
   va_list ap;
   va_start(ap, fmt);
@@ -56,6 +59,10 @@ const char* kq_status_string(kq_status s) {
 }
 
 const char* kq_last_error(void) { return kq::g_last_error; }
+
+unsigned long long kq_set_wait_limit_ns(unsigned long long ns) {
+  return kq::g_wait_limit_ns.exchange(ns, std::memory_order_relaxed);
+}
 
 int kq_version(void) { return 100; }  // 0.1.0
 

@@ -26,6 +26,9 @@ inline kq_status cuda_check(cudaError_t e, const char* what) {
 // Counts kernel launches enqueued by this library (see kq_launch_count).
 void count_launch();
 
+// Current limit of the tensor-core kernels' device waits (kq_set_wait_limit_ns).
+unsigned long long wait_limit_ns();
+
 // Launch-error check after a kernel launch; also counts the launch.
 inline kq_status launch_check(const char* what) {
   count_launch();

@@ -22,8 +22,8 @@
 // summed in a fixed order.
 //
 // kq_kron_loss_noalloc (below) keeps a SIMT fp32 path whose only scratch is
-// one fp64 per 64x64 tile: each CTA forms one tile of both products and
-// reduces their elementwise product.
+// one fp64 per 64x64 tile: each CTA forms one tile of dW H_X and of
+// H_G^T dW and reduces their elementwise product (exact for any H_X, H_G).
 #include <algorithm>
 #include <mutex>
 
@@ -84,8 +84,10 @@ __global__ void __launch_bounds__(256) loss_tile_kernel(const float* __restrict_
   tile_product(A, d_in, [&](int r, int64_t k) { return D(r0 + r, k); },
                [&](int64_t k, int c) { return (c0 + c < d_in) ? HX[k * ldhx + c0 + c] : 0.f; });
   if (HG) {
-    // B = H_G dW (K = d_out)
-    tile_product(B, d_out, [&](int r, int64_t k) { return (r0 + r < d_out) ? HG[(r0 + r) * ldhg + k] : 0.f; },
+    // B = H_G^T dW (K = d_out): H_G read by columns, so that the sum below is
+    // sum (dW H_X) .* (H_G^T dW) = tr((dW H_X)^T H_G^T dW) = tr(dW H_X dW^T H_G)
+    // exactly, for any H_X and H_G (no symmetry used)
+    tile_product(B, d_out, [&](int r, int64_t k) { return (r0 + r < d_out) ? HG[k * ldhg + r0 + r] : 0.f; },
                  [&](int64_t k, int c) { return D(k, c0 + c); });
   } else {
 #pragma unroll
@@ -302,6 +304,9 @@ extern "C" kq_status kq_kron_loss_noalloc(const float* W, int64_t ldw, const flo
   if (ldw < d_in || ldwh < d_in || ldhx < d_in || (H_G && ldhg < d_out))
     return kq::fail(KQ_ERR_INVALID_ARG, "kq_kron_loss_noalloc: leading dimension too small");
   const int64_t tiles = kq::cdiv(d_out, T) * kq::cdiv(d_in, T);
+  if (kq::cdiv(d_out, T) > 65535)   // the tile rows are the grid's y extent
+    return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_kron_loss_noalloc: ceil(d_out/64) = %lld exceeds 65535",
+                    (long long)kq::cdiv(d_out, T));
   if (tiles > KQ_KRON_LOSS_NOALLOC_MAX_TILES)
     return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE,
                     "kq_kron_loss_noalloc: ceil(d_out/64) * ceil(d_in/64) = %lld tiles exceeds the fixed scratch of %d "

@@ -63,6 +63,7 @@ struct Params {
   int c_vec;        // C rows 16-byte aligned (C aligned, ldc % 4 == 0)
   float* partial;   // [splits][num_tiles][256][256] when splits > 1
   int32_t* info;
+  unsigned long long wait_ns;   // limit of each pipeline wait (kq_set_wait_limit_ns)
 };
 
 using namespace kq::tc;
@@ -136,7 +137,7 @@ __global__ void __launch_bounds__(THREADS, 1) syrk_tc_kernel(const __grid_consta
         const int kb1 = min(p.kblocks, kb0 + p.kb_per_split);
         const bool diag = (ti == tj);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.info, 1)) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.info, 1, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -176,13 +177,13 @@ __global__ void __launch_bounds__(THREADS, 1) syrk_tc_kernel(const __grid_consta
         const int kb0 = sp * p.kb_per_split;
         const int kb1 = min(p.kblocks, kb0 + p.kb_per_split);
         const bool diag = (ti == tj);
-        if (!mbar_wait(accempty, acc_phase ^ 1u, abort_flag, p.info, 2)) {
+        if (!mbar_wait(accempty, acc_phase ^ 1u, abort_flag, p.info, 2, p.wait_ns)) {
           ok = false;
           break;
         }
         fence_after();
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, p.info, 3)) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, p.info, 3, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -223,7 +224,7 @@ __global__ void __launch_bounds__(THREADS, 1) syrk_tc_kernel(const __grid_consta
       unit_coords(p, u, &ti, &tj, &sp);
       // one lane waits, the warp follows: every lane leaves together on abort
       bool ready = true;
-      if (lane == 0) ready = mbar_wait(accfull, acc_phase, abort_flag, p.info, 4);
+      if (lane == 0) ready = mbar_wait(accfull, acc_phase, abort_flag, p.info, 4, p.wait_ns);
       if (!__shfl_sync(0xffffffffu, ready ? 1 : 0, 0)) break;
       __syncwarp();
       fence_after();
@@ -471,6 +472,7 @@ extern "C" kq_status kq_accum_cov(const uint16_t* A, int64_t n, int64_t d, int64
   p.c_vec = (kq::aligned(C, 16) && !(ldc & 3)) ? 1 : 0;
   p.partial = static_cast<float*>(ws);
   p.info = info;
+  p.wait_ns = kq::wait_limit_ns();
 
   int dev = 0, sms = ASSUMED_SMS;
   KQ_TRY(kq::cuda_check(cudaGetDevice(&dev), "kq_accum_cov: cudaGetDevice"));

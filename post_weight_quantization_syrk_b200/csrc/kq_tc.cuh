@@ -13,8 +13,9 @@
 namespace kq {
 namespace tc {
 
-// A wait that lasts longer than this is treated as a deadlock.
-constexpr unsigned long long kTimeoutNs = 4000000000ull;
+// Bound of the drains after an abort (a pipeline wait's own limit is a
+// kernel parameter, kq_set_wait_limit_ns).
+constexpr unsigned long long kTimeoutNs = KQ_WAIT_LIMIT_DEFAULT_NS;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -54,18 +55,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Bounded wait for the phase with the given parity.  Returns false (after
 // setting the CTA's abort flag and recording KQ_ERR_TIMEOUT with `where`)
-// when the limit expires, or when another role of the CTA already aborted.
+// when `limit_ns` has passed (limit 0: at the first poll that finds the phase
+// incomplete), or when another role of the CTA already aborted.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int32_t* info,
-                                          int where) {
+                                          int where, unsigned long long limit_ns) {
   unsigned long long t0 = 0;
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (*abort_flag) return false;
       unsigned long long now = globaltimer();
-      if (it == 0) {
-        t0 = now;
-      } else if (now - t0 > kTimeoutNs) {
+      if (it == 0) t0 = now;
+      if (it == 0 ? limit_ns == 0 : now - t0 > limit_ns) {
         *abort_flag = 1;
         report(info, KQ_ERR_TIMEOUT, where);
         return false;

@@ -47,6 +47,12 @@ def test_status_strings_and_version():
         assert P.kq_status_string(code) == name
 
 
+def test_wait_limit_is_process_wide_and_returns_the_previous_value():
+    assert P.kq_set_wait_limit_ns(123) == P.KQ_WAIT_LIMIT_DEFAULT_NS
+    assert P.kq_set_wait_limit_ns(0) == 123
+    assert P.kq_set_wait_limit_ns(P.KQ_WAIT_LIMIT_DEFAULT_NS) == 0
+
+
 def test_allocation_matches_oracle_bit_exact():
     rng = np.random.default_rng(0)
     for _ in range(200):

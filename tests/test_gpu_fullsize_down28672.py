@@ -4,7 +4,8 @@ launch configuration, checked against the oracle where it can follow:
 a sampled covariance block; the trailing 2048 x 2048 corner of the Cholesky
 factor of the damped inverse, which depends only on the same corner of H_X'
 and on lambda (for the reversed factorisation Uc = J L^-1 J, L = chol(J H J),
-the leading block of L is the Cholesky factor of the leading block of J H J);
+the leading block of L is the Cholesky factor of the leading block of J H J),
+and a residual check of the whole factor on sampled columns;
 sampled solver rows on the GPU's W' and Uc; the whole Kronecker loss; the
 sensitivity.  Tolerances as in test_gpu_parity.py.
 """
@@ -80,6 +81,40 @@ def test_cholesky_trailing_corner(layer):
     # and Uc is upper triangular with a positive diagonal everywhere
     assert bool((torch.diagonal(lq.Uc) > 0).all())
     assert float(torch.tril(lq.Uc, -1).abs().max()) == 0.0
+
+
+def test_cholesky_residual_sampled_columns(layer):
+    """A residual pin of the WHOLE factor, leading rows included: for sampled
+    columns j (the first 64, the last 64 and 64 at random),
+    ||(Uc^T Uc (H_X' + lambda I) - I) e_j|| <= 2e-6, evaluated in fp64.  The
+    exact factor of a Student-t layer of this shape, rounded to fp32, leaves
+    1.4e-7 (1024 and 2048 channels) to 1.7e-7 (4096) here, so the bound
+    catches any row of Uc off by more than about 1e-5 relative."""
+    lq = layer["lq"]
+    n = layer["spec"].d_in
+    H = lq.H_X
+    dev = H.device
+    diag = torch.diagonal(H).double()
+    dead = diag == 0
+    lam = 0.01 * float(torch.where(dead, torch.ones_like(diag), diag).mean())
+    rng = np.random.default_rng(29)
+    S = np.unique(np.r_[np.arange(64), np.arange(n - 64, n), rng.choice(n, 64, replace=False)])
+    St = torch.from_numpy(S).to(dev)
+    # column j of the symmetric matrix the factor is defined from (its upper
+    # triangle): rows i <= j from H[i, j], rows i > j from H[j, i]
+    up = H[:, St].double()
+    lo = H[St, :].double().T
+    rows = torch.arange(n, device=dev)[:, None]
+    Hs = torch.where(rows <= St[None, :], up, lo)
+    k = torch.arange(len(S), device=dev)
+    Hs[St, k] = torch.where(dead[St], torch.ones_like(diag[St]), diag[St]) + lam
+    Uc = lq.Uc.double()
+    R = Uc.T @ (Uc @ Hs)
+    R[St, k] -= 1.0
+    r = torch.linalg.vector_norm(R, dim=0).cpu().numpy()
+    del Uc, R
+    torch.cuda.empty_cache()
+    assert r.max() <= 2e-6, (float(r.max()), int(S[int(np.argmax(r))]))
 
 
 def test_solver_sampled_rows(layer):

@@ -100,6 +100,35 @@ def test_accum_cov_nonfinite_reported(P):
     assert code == 7
 
 
+def test_accum_cov_wait_timeout_reported_then_recovers(P):
+    """Failure detection without a fault: with the device-wait limit at 0 the
+    SYRK's pipeline waits give up at their first incomplete poll, the call
+    records KQ_ERR_TIMEOUT (index = the wait's site) in info, and the kernel
+    drains its own copies and products with the normal bound before it frees
+    its tensor memory and returns.  The context stays usable: the next call
+    with the default limit matches the oracle."""
+    X = synth.activations(SMALL, 7).cuda()
+    n = X.shape[0]
+    C = torch.zeros((704, 704), device="cuda")
+    info = _info()
+    old = P.kq_set_wait_limit_ns(0)
+    try:
+        P.kq_accum_cov(X, C, 1.0 / n, False, None, info)
+        torch.cuda.synchronize()
+    finally:
+        P.kq_set_wait_limit_ns(old)
+    assert old == P.KQ_WAIT_LIMIT_DEFAULT_NS
+    code, where = _info_code(info)
+    assert code == 8 and where in (1, 2, 3, 4), (code, where)
+    info.zero_()
+    C.fill_(float("nan"))
+    P.kq_accum_cov(X, C, 1.0 / n, False, None, info)
+    torch.cuda.synchronize()
+    assert _info_code(info)[0] == 0
+    fro, ent = cov_close(np64(C), O.covariance(X.cpu().float().numpy()))
+    assert fro <= 1e-4 and ent <= 1e-4, (fro, ent)
+
+
 # ------------------------------------------------------------------ sensitivity
 
 def test_sensitivity_parity(P):
