@@ -16,6 +16,16 @@ With N > 1 (torchrun) every rank quantizes its own layer (weak scaling, no
 data-path collective); timing is the max over ranks.  Rank 0 prints one JSON
 line.  --impl reference times the float64 CPU oracle on a bounded sample of
 the same workload on the host cores and prints the same line for it.
+
+Besides the headline the line carries, all measured outside the timed
+region: `roofline` for the dominant kernel (the covariance SYRK, against the
+measured burst bf16 peak: the runs hold the maximum SM clock);
+`stage_roofline`, every stage of the step against its own bound (SYRK and
+trailing-update GEMMs on the tensor pipe, rotations and the quantize pass
+against HBM, the Cholesky against an fp64 DGEMM measured in the same run);
+`configs`, the per-layer numbers of the other workloads (the 512 x 512
+layer, the MLP gate/up and down layers, the 70B-shaped down projection);
+`model_7b`, the whole 7B-shaped model.
 """
 from __future__ import annotations
 
@@ -50,6 +60,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-model", action="store_true", help="skip the whole 7B-shaped model run")
     ap.add_argument("--model-blocks", type=int, default=32)
+    ap.add_argument("--configs", default="layer512,mlp_up11008,mlp_down11008,down28672",
+                    help="other workloads reported per layer (comma list; empty for none)")
+    ap.add_argument("--no-diag", action="store_true", help="skip the untimed per-kernel-class diagnostics")
     a = ap.parse_args()
     a.warmup = max(a.warmup, 3)
     return a
@@ -62,6 +75,120 @@ def peaks():
         return p, "measured"
     except OSError:
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def tf32x3_peak(pk, src):
+    """Effective peak of a 3xTF32 product: dense tf32 runs at half the bf16
+    rate (1.1 against 2.25 PFLOP/s nominal), and every product issues three
+    tf32 MMAs (big*big + big*small + small*big)."""
+    return {"value": pk["bf16_tflops"] / 2.0 / 3.0, "unit": "TFLOP/s",
+            "source": f"{src} burst bf16 {pk['bf16_tflops']} / 2 (tf32 : bf16 nominal) / 3 (MMAs per product)"}
+
+
+def fp64_peak(dev):
+    """fp64 denominator for the Cholesky: a cuBLAS DGEMM (torch.matmul, 8192^3)
+    timed here with CUDA events, best of 5; MEASURED_PEAKS.json has no fp64
+    figure.  A library GEMM is used only as this yardstick."""
+    import torch
+    n = 8192
+    a = torch.randn((n, n), dtype=torch.float64, device=dev)
+    b = torch.randn((n, n), dtype=torch.float64, device=dev)
+    torch.matmul(a, b)
+    best = None
+    for _ in range(5):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        torch.matmul(a, b)
+        e.record()
+        torch.cuda.synchronize()
+        ms = s.elapsed_time(e)
+        best = ms if best is None else min(best, ms)
+    del a, b
+    return {"value": 2.0 * n ** 3 / (best / 1e3) / 1e12, "unit": "TFLOP/s",
+            "source": "cuBLAS DGEMM 8192^3 (torch.matmul fp64) measured in this run, best of 5"}
+
+
+def stage_roofline(spec, settings, stages_ms, pk, src, fp64):
+    """Every stage of one step against its own bound.  Algorithmic work per
+    unit (one layer): SYRK N d (d + 1) flops per covariance (lower triangle);
+    rotations 8 bytes per element per pass, 2 passes each for W, H_X, H_G;
+    Cholesky n^3/3 + n^3/3 fp64 flops; quantize pass 13 bytes per weight per
+    setting (W slab read; W_hat, codes, errors written); Kronecker loss
+    2 d_out d_in (min + max/2) flops per setting as formed (2 d_out d_in
+    (d_in + d_out) if both products of the trace were formed in full, also
+    reported)."""
+    d_out, d_in, N, k = spec.d_out, spec.d_in, spec.n_tokens, len(settings)
+    hbm = pk["hbm_gbs"]
+    x3 = tf32x3_peak(pk, src)
+    q_ms = next(v for n, v in stages_ms.items() if n.startswith("quantize"))
+    l_ms = next(v for n, v in stages_ms.items() if n.startswith("loss"))
+    out = {}
+
+    def put(name, work, unit, ms, peak, peak_unit, peak_src, note):
+        ach = work / (ms / 1e3) / (1e12 if peak_unit == "TFLOP/s" else 1e9)
+        out[name] = {"ms": ms, "work": work, "work_unit": unit, "achieved": ach, "unit": peak_unit, "peak": peak,
+                     "frac": ach / peak, "peak_source": peak_src, "note": note}
+
+    put("syrk", float(N) * (d_in * (d_in + 1) + d_out * (d_out + 1)), "flop", stages_ms["syrk_x2"],
+        pk["bf16_tflops"], "TFLOP/s", f"{src} burst bf16", "both covariances incl. the fixed-order split sum")
+    put("rotate", 8.0 * 2 * (d_out * d_in + d_in * d_in + d_out * d_out), "byte", stages_ms["rotate"], hbm, "GB/s",
+        f"{src} HBM copy", "6 algorithmic passes (W, H_X, H_G 2 each); the column transform takes 2 passes, so "
+                           "9 passes move 1.5x these bytes")
+    put("chol_inv", 2.0 * d_in ** 3 / 3.0, "flop", stages_ms["chol_inv"], fp64["value"], "TFLOP/s",
+        fp64["source"], "fp64 throughout (DMMA trailing updates, serial 64-column diagonal chain)")
+    put("quantize", 13.0 * d_out * d_in * k, "byte", q_ms, hbm, "GB/s", f"{src} HBM copy",
+        f"{k} settings solved side by side (grid fit, in-block recursion, trailing updates)")
+    lo, hi = min(d_in, d_out), max(d_in, d_out)
+    put("loss", 2.0 * d_out * d_in * (lo + hi / 2.0) * k, "flop", l_ms, x3["value"], "TFLOP/s", x3["source"],
+        "3xTF32; work = the products as formed, one Hessian in the first product and the upper block triangle "
+        "of the second: 2 d_out d_in (min + max/2) flops per setting")
+    full = 2.0 * d_out * d_in * (d_in + d_out) * k
+    out["loss"]["work_both_products_full"] = full
+    out["loss"]["achieved_vs_full_products"] = full / (l_ms / 1e3) / 1e12
+    return out
+
+
+def run_layer_steps(P, LayerQuantizer, spec, settings, seed, dev, steps, warmup, gemm_mode):
+    """Generate one layer, run `warmup` + `steps` whole-path steps with CUDA
+    events per stage; returns (ms per step, stage ms, the quantizer)."""
+    import torch
+    import synth
+    with torch.no_grad():
+        W = synth.weights(spec, seed, dev)
+        X = synth.activations(spec, seed, dev)
+        G = synth.gradients(spec, seed, dev)
+    Ti, To = synth.rht_params(spec.d_in, seed * 2 + 11), synth.rht_params(spec.d_out, seed * 2 + 12)
+    T_in = P.RHT(Ti.n, Ti.log2_p, Ti.m, Ti.signs.to(dev), None if Ti.Qm is None else Ti.Qm.to(dev))
+    T_out = P.RHT(To.n, To.log2_p, To.m, To.signs.to(dev), None if To.Qm is None else To.Qm.to(dev))
+    lq = LayerQuantizer(spec.d_out, spec.d_in, dev, gemm_mode=gemm_mode)
+    results = [lq.alloc_result(b, g) for b, g in settings]
+    stream = torch.cuda.current_stream()
+    names = ["syrk_x2", "sensitivity", "rotate", "chol_inv", "quantize", "loss"]
+    per = {n: [] for n in names}
+    total = 0.0
+    for it in range(warmup + steps):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+        ev[0].record(stream)
+        lq.statistics(X, G)
+        ev[1].record(stream)
+        lq.sensitivity()
+        ev[2].record(stream)
+        lq.rotate(W, T_in, T_out)
+        ev[3].record(stream)
+        lq.factor(0.01)
+        ev[4].record(stream)
+        lq.quantize_all(results)
+        ev[5].record(stream)
+        lq.loss_all(results)
+        ev[6].record(stream)
+        torch.cuda.synchronize()
+        if it >= warmup:
+            for i, n in enumerate(names):
+                per[n].append(ev[i].elapsed_time(ev[i + 1]))
+            total += ev[0].elapsed_time(ev[-1])
+    lq.check(spec.name)
+    del X, G
+    return total / steps, {n: statistics.mean(v) for n, v in per.items()}, lq, results, W, T_in, T_out
 
 
 # ----------------------------------------------------------------- clocks
@@ -219,6 +346,73 @@ def run_kronq(a):
     if not a.no_e2e:
         e2e = run_e2e(a, lq, results, W, X, G, T_in, T_out, spec, settings, world, dev)
 
+    # ---- untimed diagnostics: fp64 yardstick, solver split by kernel class,
+    # host enqueue time per stage
+    pk, src = peaks()
+    fp64 = fp64_peak(dev)
+    solver = None
+    host_ms = None
+    if not a.no_diag:
+        solver = {k: 0.0 for k in ("grid_ms", "inblock_ms", "update_ms", "grid_launches", "inblock_launches",
+                                   "update_launches", "update_flops", "inblock_bytes")}
+        for r in results:   # one setting at a time: no overlap between lanes
+            P.kq_solver_timing(True)
+            lq.quantize(r)
+            t = P.kq_solver_timing(False)
+            for k_ in solver:
+                solver[k_] += t[k_]
+        torch.cuda.synchronize()
+        host_ms = {}
+        c0 = time.perf_counter()
+        for name, fn in (("statistics", lambda: lq.statistics(X, G)), ("sensitivity", lq.sensitivity),
+                         ("rotate", lambda: lq.rotate(W, T_in, T_out)), ("chol_inv", lambda: lq.factor(0.01)),
+                         ("quantize", lambda: lq.quantize_all(results)), ("loss", lambda: lq.loss_all(results))):
+            t0 = time.perf_counter()
+            fn()
+            host_ms[name] = (time.perf_counter() - t0) * 1e3
+        host_ms["total"] = (time.perf_counter() - c0) * 1e3
+        torch.cuda.synchronize()
+        lq.check("diagnostics")
+    sr = stage_roofline(spec, settings, stages_ms, pk, src, fp64)
+    if solver:
+        x3 = tf32x3_peak(pk, src)
+        ib_ach = solver["inblock_bytes"] / (solver["inblock_ms"] / 1e3) / 1e9
+        up_ach = solver["update_flops"] / (solver["update_ms"] / 1e3) / 1e12
+        sr["solver_inblock"] = {
+            "ms": solver["inblock_ms"], "launches": int(solver["inblock_launches"]),
+            "us_per_launch": 1e3 * solver["inblock_ms"] / max(1, solver["inblock_launches"]),
+            "work": solver["inblock_bytes"], "work_unit": "byte", "achieved": ib_ach, "unit": "GB/s",
+            "peak": pk["hbm_gbs"], "frac": ib_ach / pk["hbm_gbs"], "peak_source": f"{src} HBM copy",
+            "note": "per-launch CUDA events, one setting at a time (untimed diagnostic pass)"}
+        sr["solver_trailing_gemm"] = {
+            "ms": solver["update_ms"], "launches": int(solver["update_launches"]), "work": solver["update_flops"],
+            "work_unit": "flop", "achieved": up_ach, "unit": "TFLOP/s", "peak": x3["value"],
+            "frac": up_ach / x3["value"], "peak_source": x3["source"],
+            "note": "3xTF32 trailing updates, per-launch CUDA events, one setting at a time"}
+        sr["solver_grid"] = {"ms": solver["grid_ms"], "launches": int(solver["grid_launches"])}
+
+    # ---- the other workloads, per layer (untimed by the headline; each its
+    # own short run with per-stage CUDA events)
+    configs = {}
+    cfg_settings = {"layer512": [(3, 0)], "mlp_up11008": [(3, 128), (2, 0)], "mlp_down11008": [(3, 128), (2, 0)],
+                    "down28672": [(2, 0)]}
+    cfg_index = {"layer512": 1, "mlp_up11008": 3, "mlp_down11008": 3, "down28672": 4}
+    for name in [c for c in a.configs.split(",") if c]:
+        cspec = synth.WORKLOADS[name]
+        cset = cfg_settings.get(name, settings)
+        small = cspec.d_out * cspec.d_in <= 1 << 20
+        ms_c, st_c, lq_c, res_c, W_c, Ti_c, To_c = run_layer_steps(
+            P, LayerQuantizer, cspec, cset, synth.layer_seed(cfg_index.get(name, 9), rank), dev,
+            steps=10 if small else 2, warmup=3 if small else 1, gemm_mode=gemm_mode)
+        configs[name] = {
+            "workload": f"{name}: W {cspec.d_out}x{cspec.d_in}, N={cspec.n_tokens} tokens, "
+                        + "+".join(f"W{b}" + (f" g{g}" if g else "") for b, g in cset),
+            "ms_per_step": ms_c, "weights_per_s": cspec.d_out * cspec.d_in * len(cset) / (ms_c / 1e3),
+            "stages_ms": st_c, "stage_roofline": stage_roofline(cspec, cset, st_c, pk, src, fp64),
+            "losses": [float(r.loss.item()) for r in res_c], "steps": 10 if small else 2}
+        del lq_c, res_c, W_c
+        torch.cuda.empty_cache()
+
     # ---- the whole 7B-shaped model (32 blocks x 7 linears); on N ranks each
     # takes every N-th block and the sensitivity table is merged for the
     # allocation (the model's total work is fixed: strong scaling)
@@ -236,13 +430,12 @@ def run_kronq(a):
                          "allocation, BiIP, Cholesky, solver, loss), the slowest rank's when sharded; phase "
                          "seconds are rank 0's; synthetic inputs generated per block, untimed")
 
-    pk, src = peaks()
     flops = spec.n_tokens * spec.d_in * (spec.d_in + 1)    # one SYRK launch on X (d_out == d_in here)
     traffic = syrk_traffic(a.workload)
     syrk_avg = statistics.mean(syrk_ms)
     achieved = flops / (syrk_avg / 1e3) / 1e12
-    peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
-    burst = pk.get("bf16_tflops") or peak
+    peak = pk.get("bf16_tflops")
+    sustained = pk.get("bf16_tflops_sustained") or peak
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
         "ms_per_step": ms_max / a.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -254,12 +447,15 @@ def run_kronq(a):
                    "l2": "inputs larger than L2 (X, G 2 GiB each); no flush"},
         "roofline": {"kernel": "kq_accum_cov (SYRK)", "bound": "tensor", "achieved": achieved, "peak": peak,
                      "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                     "peak_source": f"{src} bf16 sustained",
-                     # the burst figure too: the sustained one was taken at power-capped clocks
-                     "burst_peak": burst, "frac_of_burst": achieved / burst,
+                     "peak_source": f"{src} bf16 burst (the step runs at the maximum SM clock, see clocks)",
+                     # the sustained figure too: it was taken at power-capped clocks
+                     "sustained_peak": sustained, "frac_of_sustained": achieved / sustained,
                      "algorithmic_flops_per_launch": flops,
                      "avg_launch_ms": syrk_avg},
         "stages_ms": stages_ms,
+        "stage_roofline": sr,
+        "host_enqueue_ms": host_ms,
+        "configs": configs,
         "gpu_launches": launches,
         "clocks": clk,
         "e2e": e2e,
@@ -274,11 +470,12 @@ def run_kronq(a):
         print(json.dumps(out), flush=True)
 
 
-# DRAM bytes (read + write) of one kq_accum_cov call at 262144 x 4096, from the
-# ncu capture summarised in profiles/syrk_tc_kernel_attn4096_traffic.md; valid
-# only for the kernel sources it was taken on.
+# DRAM bytes (read + write, both launches) of one kq_accum_cov call at
+# 262144 x 4096, from one ncu capture of dram__bytes_read.sum and
+# dram__bytes_write.sum; valid only for the kernel sources it was taken on
+# (their hashes), else the bench reports null.
 SYRK_TRAFFIC = {"attn4096": 5.00e9}
-SYRK_SOURCE_SHA = {"kq_syrk.cu": "219987dcfe1d0668", "kq_tc.cuh": "f59b54090d782541"}
+SYRK_SOURCE_SHA = {"kq_syrk.cu": "a457aac871c196f3", "kq_tc.cuh": "91f487fc41a449d7"}
 
 
 def syrk_traffic(workload):

@@ -263,6 +263,27 @@ kq_status kq_quantize_layer_multi(const float* W, int64_t d_out, int64_t d_in, i
                                   float* const* zeros, float* const* W_hat, int64_t ldwh,
                                   void* ws, size_t ws_bytes, int32_t* info, kq_stream_t stream);
 
+/* kq_solver_timing - diagnostic timing of the solver's kernel classes.
+ *
+ * kq_solver_timing(1, NULL) makes this host thread's following
+ * kq_quantize_layer / kq_quantize_layer_multi calls record a pair of CUDA
+ * events around each launch of the grid fit, the in-block recursion and the
+ * trailing update (on the stream it goes to); kq_solver_timing(0, out)
+ * synchronises those events, writes the summed times and counts to `out`
+ * (may be NULL) and stops recording.  The events sit between launches that
+ * would otherwise overlap (programmatic dependent launches), so a recorded
+ * solve runs slightly slower than an unrecorded one: use it to split a
+ * solve's time by kernel class, not to time the solve.  Host memory. */
+typedef struct kq_solver_times {
+  double grid_ms, inblock_ms, update_ms;               /* summed event intervals per class */
+  long long grid_launches, inblock_launches, update_launches;
+  double update_flops;   /* algorithmic flops of the trailing updates: sum of 2 M N K */
+  double inblock_bytes;  /* algorithmic bytes of the in-block launches: W slab read, W_hat slab,
+                            codes and errors written (4 + 4 + 1 + 4 bytes per weight, the
+                            errors 8 when kept as a tf32 split for the tensor cores) */
+} kq_solver_times;
+kq_status kq_solver_timing(int enable, kq_solver_times* out);
+
 /* --------------------------------------------------------------------------
  * kq_kron_loss - Kronecker loss (a10).
  *

@@ -10,6 +10,7 @@ from ._lib import (  # noqa: F401
     kq_accum_cov_workspace_size, kq_allocate_bits, kq_chol_inv, kq_chol_inv_workspace_size, kq_kron_loss,
     kq_kron_loss_multi, kq_kron_loss_workspace_size, kq_launch_count, kq_pack_codes, kq_quantize_layer,
     kq_quantize_layer_multi, kq_reverted_matvec, kq_reverted_matvec_workspace_size, kq_set_wait_limit_ns, KQ_WAIT_LIMIT_DEFAULT_NS,
+    kq_solver_timing,
     kq_quantize_layer_multi_workspace_size, kq_quantize_layer_workspace_size, kq_rotate, kq_sensitivity,
     kq_status_string, kq_version, load, new_info, workspace,
 )

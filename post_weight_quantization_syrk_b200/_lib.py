@@ -34,7 +34,7 @@ EXPORTS = (
     "kq_rotate",
     "kq_chol_inv_workspace_size", "kq_chol_inv",
     "kq_quantize_layer_workspace_size", "kq_quantize_layer", "kq_quantize_layer_multi_workspace_size",
-    "kq_quantize_layer_multi",
+    "kq_quantize_layer_multi", "kq_solver_timing",
     "kq_kron_loss_workspace_size", "kq_kron_loss", "kq_kron_loss_multi", "kq_kron_loss_noalloc",
     "kq_allocate_bits",
 )
@@ -45,6 +45,13 @@ class KronqError(RuntimeError):
         self.status = int(status)
         self.name = STATUS_NAMES.get(int(status), f"status {status}")
         super().__init__(f"{where}: {self.name}: {detail}" if where else f"{self.name}: {detail}")
+
+
+class kq_solver_times(ctypes.Structure):
+    _fields_ = [("grid_ms", ctypes.c_double), ("inblock_ms", ctypes.c_double), ("update_ms", ctypes.c_double),
+                ("grid_launches", ctypes.c_longlong), ("inblock_launches", ctypes.c_longlong),
+                ("update_launches", ctypes.c_longlong), ("update_flops", ctypes.c_double),
+                ("inblock_bytes", ctypes.c_double)]
 
 
 class kq_rht(ctypes.Structure):
@@ -75,6 +82,7 @@ _SIGS = {
                                        ctypes.POINTER(ctypes.c_int), _i32, _i32, ctypes.POINTER(_vp), _i64,
                                        ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i64, _vp, _sz,
                                        _vp, _vp]),
+    "kq_solver_timing": (_i32, [_i32, ctypes.POINTER(kq_solver_times)]),
     "kq_kron_loss_workspace_size": (_sz, [_i64, _i64]),
     "kq_kron_loss_multi": (_i32, [_vp, _i64, _i32, ctypes.POINTER(_vp), _i64, _i64, _i64, _vp, _i64, _vp, _i64,
                                   ctypes.POINTER(_vp), _vp, _sz, _vp]),
@@ -416,3 +424,14 @@ def kq_set_wait_limit_ns(ns):
     wide); 0 makes a wait give up at its first incomplete poll.  Returns the
     previous limit."""
     return int(load().kq_set_wait_limit_ns(int(ns)))
+
+
+def kq_solver_timing(enable):
+    """Diagnostic: kq_solver_timing(True) starts recording CUDA events around
+    this thread's solver launches; kq_solver_timing(False) synchronises and
+    returns the per-class sums as a dict."""
+    t = kq_solver_times()
+    _check(load().kq_solver_timing(1 if enable else 0, None if enable else ctypes.byref(t)), "kq_solver_timing")
+    if enable:
+        return None
+    return {f: getattr(t, f) for f, _ in kq_solver_times._fields_}

@@ -24,6 +24,7 @@
 // (round half to even); errors e = (w - w_hat) * (1/Uc[j][j]).  The grid
 // itself (scale, zero) uses IEEE fp32 division.
 #include <algorithm>
+#include <vector>
 
 #include "kq_gemm.cuh"
 #include "kq_internal.cuh"
@@ -364,6 +365,45 @@ __global__ void __launch_bounds__(256) trailing_fp32_kernel(const float* __restr
 
 namespace {
 
+// Diagnostic timing (kq_solver_timing): event pairs around each launch,
+// recorded per host thread while enabled.
+enum TimedClass { kClassGrid = 0, kClassInblock = 1, kClassUpdate = 2 };
+struct TimedLaunch {
+  int cls;
+  cudaEvent_t a, b;
+  double flops, bytes;
+};
+struct SolverTiming {
+  bool on = false;
+  std::vector<TimedLaunch> recs;
+  std::vector<cudaEvent_t> pool;
+};
+thread_local SolverTiming g_timing;
+
+kq_status timing_event(cudaEvent_t* e) {
+  if (!g_timing.pool.empty()) {
+    *e = g_timing.pool.back();
+    g_timing.pool.pop_back();
+    return KQ_OK;
+  }
+  return kq::cuda_check(cudaEventCreate(e), "kq_solver_timing: event");
+}
+
+// Runs `launch` (a kq_status-returning callable) between two recorded events
+// when timing is on; otherwise just runs it.
+template <typename F>
+kq_status timed(int cls, double flops, double bytes, cudaStream_t st, F&& launch) {
+  if (!g_timing.on) return launch();
+  TimedLaunch r{cls, nullptr, nullptr, flops, bytes};
+  KQ_TRY(timing_event(&r.a));
+  KQ_TRY(timing_event(&r.b));
+  KQ_TRY(kq::cuda_check(cudaEventRecord(r.a, st), "kq_solver_timing: record"));
+  const kq_status s = launch();
+  KQ_TRY(kq::cuda_check(cudaEventRecord(r.b, st), "kq_solver_timing: record"));
+  g_timing.recs.push_back(r);
+  return s;
+}
+
 // Outer block of the two-level lazy update (3xTF32 path): after each
 // 128-column block only the rest of its outer block is updated; after each
 // outer block one GEMM with K = OUTER updates all columns to its right.
@@ -452,9 +492,11 @@ kq_status enqueue_setting(const float* W, int64_t d_out, int64_t d_in, int64_t l
   const int64_t n_groups = group ? kq::cdiv(d_in, group) : 1;
 
   if (!group) {
-    grid_rows_kernel<<<(unsigned)kq::cdiv(d_out, 8), 256, 0, st>>>(W, ldw, d_out, d_in, dead_mask, nl, scales, zeros,
-                                                                   info);
-    KQ_TRY(kq::launch_check("kq_quantize_layer grid"));
+    KQ_TRY(timed(kClassGrid, 0.0, 4.0 * d_out * d_in, st, [&]() -> kq_status {
+      grid_rows_kernel<<<(unsigned)kq::cdiv(d_out, 8), 256, 0, st>>>(W, ldw, d_out, d_in, dead_mask, nl, scales,
+                                                                     zeros, info);
+      return kq::launch_check("kq_quantize_layer grid");
+    }));
   }
   KQ_TRY(kq::cuda_check(cudaFuncSetAttribute(inblock_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, IB_SMEM),
                         "kq_quantize_layer: smem attribute"));
@@ -488,8 +530,10 @@ kq_status enqueue_setting(const float* W, int64_t d_out, int64_t d_in, int64_t l
     a.info = info;
     // after the first block the previous kernel is this solve's own trailing
     // update, so the launch may overlap its tail (tensor-core mode)
-    return kq::launch_ex("kq_quantize_layer inblock", tc && i0 > 0, inblock_kernel,
-                         dim3((unsigned)kq::cdiv(d_out, IB_ROWS)), dim3(IB_THREADS), IB_SMEM, st, a);
+    return timed(kClassInblock, 0.0, (double)d_out * bw * (tc ? 17.0 : 13.0), st, [&]() {
+      return kq::launch_ex("kq_quantize_layer inblock", tc && i0 > 0, inblock_kernel,
+                           dim3((unsigned)kq::cdiv(d_out, IB_ROWS)), dim3(IB_THREADS), IB_SMEM, st, a);
+    });
   };
   // W_hat[:, c0:c0+N] = src[:, c0:c0+N] - E[:, e0:e0+K] Uc[k0:k0+K, c0:c0+N]; the
   // source is W (dead columns as zeros) while those columns are still untouched.
@@ -515,7 +559,7 @@ kq_status enqueue_setting(const float* W, int64_t d_out, int64_t d_in, int64_t l
     g.dead = from_w && dead_mask ? dead_mask + c0 : nullptr;
     g.info = info;
     g.pdl = true;   // always follows this solve's in-block kernel
-    return kq::gemm_3xtf32(g, st);
+    return timed(kClassUpdate, 2.0 * d_out * N * K, 0.0, st, [&]() { return kq::gemm_3xtf32(g, st); });
   };
   if (!tc) {
     for (int64_t i0 = 0; i0 < d_in; i0 += BLK) {
@@ -525,9 +569,11 @@ kq_status enqueue_setting(const float* W, int64_t d_out, int64_t d_in, int64_t l
       const int64_t cstart = i0 + bw;
       if (cstart < d_in) {
         dim3 grid((unsigned)kq::cdiv(d_in - cstart, TN), (unsigned)kq::cdiv(d_out, TM));
-        trailing_fp32_kernel<<<grid, 256, 0, st>>>(first ? W : W_hat, first ? ldw : ldwh, W_hat, ldwh, w.ET, Uc,
-                                                  lduc, first ? dead_mask : nullptr, d_out, d_in, i0, bw, cstart);
-        KQ_TRY(kq::launch_check("kq_quantize_layer trailing"));
+        KQ_TRY(timed(kClassUpdate, 2.0 * d_out * bw * (d_in - cstart), 0.0, st, [&]() -> kq_status {
+          trailing_fp32_kernel<<<grid, 256, 0, st>>>(first ? W : W_hat, first ? ldw : ldwh, W_hat, ldwh, w.ET, Uc,
+                                                    lduc, first ? dead_mask : nullptr, d_out, d_in, i0, bw, cstart);
+          return kq::launch_check("kq_quantize_layer trailing");
+        }));
       }
     }
   } else {
@@ -657,4 +703,39 @@ extern "C" kq_status kq_quantize_layer_multi(const float* W, int64_t d_out, int6
   if (first != KQ_OK) return first;
   kq::clear_error();
   return KQ_OK;
+}
+
+extern "C" kq_status kq_solver_timing(int enable, kq_solver_times* out) {
+  if (enable) {
+    g_timing.on = true;
+    return KQ_OK;
+  }
+  g_timing.on = false;
+  kq_solver_times t = {};
+  kq_status st = KQ_OK;
+  for (const TimedLaunch& r : g_timing.recs) {
+    float ms = 0.f;
+    if (st == KQ_OK) {
+      st = kq::cuda_check(cudaEventSynchronize(r.b), "kq_solver_timing: synchronize");
+      if (st == KQ_OK) st = kq::cuda_check(cudaEventElapsedTime(&ms, r.a, r.b), "kq_solver_timing: elapsed");
+    }
+    if (r.cls == kClassGrid) {
+      t.grid_ms += ms;
+      ++t.grid_launches;
+    } else if (r.cls == kClassInblock) {
+      t.inblock_ms += ms;
+      ++t.inblock_launches;
+      t.inblock_bytes += r.bytes;
+    } else {
+      t.update_ms += ms;
+      ++t.update_launches;
+      t.update_flops += r.flops;
+    }
+    g_timing.pool.push_back(r.a);
+    g_timing.pool.push_back(r.b);
+  }
+  g_timing.recs.clear();
+  if (out) *out = t;
+  if (st == KQ_OK) kq::clear_error();
+  return st;
 }

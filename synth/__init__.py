@@ -70,6 +70,10 @@ WORKLOADS = {
     # captures: inputs still larger than L2, a few GB on the device).
     "attn4096_n65536": LayerSpec("attn4096_n65536", 4096, 4096, 65536, w_std=0.02, x_sigma=1.5,
                                  x_massive=8, g_lo=1e-4),
+    # The MLP gate/up layer with 16384 tokens (profiling captures of the
+    # 11008-wide rotations: H_G is 485 MB, larger than L2; about 2.5 GB on
+    # the device in all).
+    "mlp_up11008_n16384": LayerSpec("mlp_up11008_n16384", 11008, 4096, 16384, x_sigma=1.0, g_lo=1e-3),
     # Llama-70B-shaped down projection: 28672 -> 8192, 65536 tokens, Student-t(3).
     "down28672": LayerSpec("down28672", 8192, 28672, 65536, w_std=0.01,
                            x_kind="student_t3", g_lo=1e-4),
