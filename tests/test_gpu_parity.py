@@ -143,7 +143,7 @@ def test_sensitivity_parity(P):
 
 # ------------------------------------------------------------------ rotations
 
-@pytest.mark.parametrize("n", [512, 704, 352, 43 * 256, 7 * 4096 // 8, 96, 5])
+@pytest.mark.parametrize("n", [512, 704, 352, 43 * 256, 7 * 4096 // 8, 96, 5, 4096, 2048, 16, 8, 7 * 1024, 8192])
 @pytest.mark.parametrize("axis", ["rows", "cols"])
 @pytest.mark.parametrize("inverse", [False, True])
 def test_rotate_parity(P, n, axis, inverse):
