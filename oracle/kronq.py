@@ -45,6 +45,8 @@ __all__ = [
     "QuantResult", "quantize_layer", "kron_loss", "gptq_loss",
     "allocate_bits", "budget_units", "quantize_linear",
     "pack_codes", "unpack_codes", "dequantize_layer", "reverted_apply",
+    "balance_permutation", "permutation_matrix", "hg_blockwise", "hg_lowrank", "block_rht_matrix",
+    "blockwise_kron_loss", "weight_cv",
 ]
 
 
@@ -550,3 +552,100 @@ def reverted_apply(packed, scales, zeros, bits, group, T_in, T_out, x):
     W_hat = dequantize_layer(codes, scales, zeros, group)
     xr = T_in @ np.asarray(x, dtype=np.float64)
     return T_out.T @ (W_hat @ xr)
+
+
+# ---------------------------------------------------------------------------
+# Output side without the full d_out x d_out H_G (next-step row: blockwise and
+# low-rank H_G), and an output rotation informed by H_G
+# ---------------------------------------------------------------------------
+# [REV] Limitations (second limitation): BiIP holds H_G as a full
+# d_out x d_out matrix, a transient peak of memory; the research thread's
+# "Sparks" list asks how much of the output-side flattening survives low-rank
+# or blockwise approximations of H_G.  [ABS] Abstract (1): the output-side
+# rotation extends the input-side one "using the gradient covariance".
+# Readings taken here (listed with the others in the design notes):
+#   * blockwise H_G: only its k x k diagonal blocks are kept (memory d_out k);
+#     the output rotation is then block diagonal, the same randomised
+#     Hadamard T_k in every block, so that V H_G V^T stays block diagonal and
+#     is formed block by block;
+#   * low-rank H_G: its best rank-r approximation (top r eigenpairs);
+#   * the H_G-informed factor: a permutation P_G of the output channels from
+#     diag(H_G) ahead of the Hadamard, V = T P_G.  Channels are ranked by
+#     descending diag(H_G) (ties: lower index) and dealt round-robin to the
+#     d_out / k blocks, so every block receives the same share of large and
+#     small gradient energy before the Hadamard mixes within it.
+
+def balance_permutation(diag_hg, k):
+    """perm with new channel i = old channel perm[i]: the channel of rank q
+    (descending diag(H_G), ties by lower index) goes to block q mod nb,
+    position q div nb, nb = d / k blocks of k channels."""
+    d = np.asarray(diag_hg).shape[0]
+    k = int(k)
+    if k < 1 or d % k:
+        raise ValueError("k must divide the number of channels")
+    nb = d // k
+    order = sorted(range(d), key=lambda j: (-float(diag_hg[j]), j))
+    perm = np.empty(d, dtype=np.int64)
+    for q, old in enumerate(order):
+        perm[(q % nb) * k + q // nb] = old
+    return perm
+
+
+def permutation_matrix(perm):
+    """P with (P x)[i] = x[perm[i]]."""
+    d = len(perm)
+    P = np.zeros((d, d))
+    P[np.arange(d), np.asarray(perm)] = 1.0
+    return P
+
+
+def hg_blockwise(H_G, k):
+    """H_G with everything outside its k x k diagonal blocks set to zero."""
+    H = np.asarray(H_G, dtype=np.float64)
+    d = H.shape[0]
+    if d % int(k):
+        raise ValueError("k must divide d")
+    out = np.zeros_like(H)
+    for b in range(0, d, int(k)):
+        out[b:b + k, b:b + k] = H[b:b + k, b:b + k]
+    return out
+
+
+def hg_lowrank(H_G, r):
+    """Best rank-r approximation of the symmetric H_G: sum of its r largest
+    eigenpairs lambda_i q_i q_i^T (library eigensolver as one step)."""
+    H = np.asarray(H_G, dtype=np.float64)
+    w, Q = np.linalg.eigh(0.5 * (H + H.T))
+    idx = np.argsort(w)[::-1][:int(r)]
+    return (Q[:, idx] * w[idx][None, :]) @ Q[:, idx].T
+
+
+def block_rht_matrix(n, k, log2_p, signs, Qm=None):
+    """Block diagonal I_{n/k} kron T_k with T_k = rht_matrix(k, log2_p, signs, Qm)."""
+    if n % k:
+        raise ValueError("k must divide n")
+    return np.kron(np.eye(n // k), rht_matrix(k, log2_p, signs, Qm))
+
+
+def blockwise_kron_loss(W, W_hat, H_X, HG_blocks):
+    """sum_b tr(dW_b H_X dW_b^T H_G,b) over the row blocks dW_b of dW = W - W_hat
+    with the k x k blocks HG_blocks[b] (array [nb, k, k]): the Kronecker loss
+    of the block-diagonal H_G they form."""
+    D = np.asarray(W, dtype=np.float64) - np.asarray(W_hat, dtype=np.float64)
+    Hb = np.asarray(HG_blocks, dtype=np.float64)
+    nb, k, _ = Hb.shape
+    s = 0.0
+    for b in range(nb):
+        Db = D[b * k:(b + 1) * k]
+        s += float(np.trace(Db @ np.asarray(H_X, dtype=np.float64) @ Db.T @ Hb[b]))
+    return s
+
+
+def weight_cv(W, axis):
+    """Coefficient of variation (std / mean) of the L2 norms of W's rows
+    (axis 'out': one norm per output channel) or columns (axis 'in'): the
+    flattening diagnostic of [REV] Method (1) (weight-magnitude variance
+    across input and output dimensions)."""
+    W = np.asarray(W, dtype=np.float64)
+    norms = np.linalg.norm(W, axis=1 if axis == "out" else 0)
+    return float(np.std(norms) / np.mean(norms))
