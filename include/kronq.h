@@ -125,6 +125,54 @@ kq_status kq_accum_cov(const uint16_t* A, int64_t n, int64_t d, int64_t lda,
                        float* C, int64_t ldc, float alpha, int accumulate,
                        void* ws, size_t ws_bytes, int32_t* info, kq_stream_t stream);
 
+/* kq_accum_cov_blocks - only the k x k diagonal blocks of the covariance.
+ *
+ * The blockwise approximation of H_G that keeps BiIP's memory at d k instead
+ * of d^2 floats (KronQ review, Limitations, second limitation: the full
+ * d_out x d_out H_G is a transient peak; research thread, "Sparks": blockwise
+ * H_G).  Block b (rows and columns b k .. b k + k - 1 of alpha A^T A) is
+ * written (or added, accumulate != 0) to rows b k .. of C, which is d x k
+ * (ldc >= k): C[b k + i][j] = alpha sum_t A[t][b k + i] A[t][b k + j].
+ * Same kernel and accuracy as kq_accum_cov; k a multiple of 256 dividing d.
+ * Workspace: kq_accum_cov_blocks_workspace_size(n, d, k) bytes (0 when
+ * the shape is unsupported). */
+size_t kq_accum_cov_blocks_workspace_size(int64_t n, int64_t d, int64_t k);
+kq_status kq_accum_cov_blocks(const uint16_t* A, int64_t n, int64_t d, int64_t lda, int64_t k, float* C,
+                              int64_t ldc, float alpha, int accumulate, void* ws, size_t ws_bytes,
+                              int32_t* info, kq_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * Output rotation informed by H_G: V = T P_G.
+ *
+ * KronQ paper page, Abstract (1): the output-side rotation extends the
+ * input-side one "using the gradient covariance"; KronQ review, Limitations
+ * (second limitation) and research thread ("Sparks"): blockwise H_G.  P_G
+ * permutes the output channels: ranked by descending diag(H_G) (ties: lower
+ * index), the channel of rank q goes to block q mod nb, slot q div nb, of the
+ * nb = d / k blocks of a blockwise rotation, so that every block holds the
+ * same share of large and small gradient energies.
+ *
+ * kq_channel_energy: out[j] = alpha sum_t A[t][j]^2 (the diagonal of
+ *   alpha A^T A without forming it) for bf16 A [n, d] (lda >= d); fp64 sums
+ *   over 64 token slices added in a fixed order; out fp32 [d] device.
+ *   Workspace kq_channel_energy_workspace_size(d).  KQ_ERR_NONFINITE in info.
+ * kq_balance_permutation: perm[(q % nb) k + q / nb] = channel of rank q by
+ *   descending energy[j] (ties: lower j); energy fp32 [d], perm int64 [d],
+ *   both device; k divides d, d <= 65536.
+ * kq_gather: out[i][j] = M[row_idx[i]][col_idx[j]] (either index array may
+ *   be NULL: the identity) for rows x cols matrices of 2- or 4-byte elements
+ *   (ldm, ldo >= cols; out must not alias M); an index outside 0..rows-1 or
+ *   0..cols-1 is skipped and reported as KQ_ERR_INVALID_ARG (index = row i).
+ *   Row gather: P_G W (or P_G^T with the inverse permutation); both: P_G H
+ *   P_G^T; columns of bf16 G: G P_G^T, whose covariance is P_G H_G P_G^T.
+ * ------------------------------------------------------------------------ */
+size_t kq_channel_energy_workspace_size(int64_t d);
+kq_status kq_channel_energy(const uint16_t* A, int64_t n, int64_t d, int64_t lda, float alpha, float* out,
+                            void* ws, size_t ws_bytes, int32_t* info, kq_stream_t stream);
+kq_status kq_balance_permutation(const float* energy, int64_t d, int64_t k, int64_t* perm, kq_stream_t stream);
+kq_status kq_gather(const void* M, int64_t ldm, int elem_bytes, const int64_t* row_idx, const int64_t* col_idx,
+                    int64_t rows, int64_t cols, void* out, int64_t ldo, int32_t* info, kq_stream_t stream);
+
 /* --------------------------------------------------------------------------
  * kq_sensitivity - trace sensitivity (step a3).
  *
@@ -139,6 +187,11 @@ kq_status kq_accum_cov(const uint16_t* A, int64_t n, int64_t d, int64_t lda,
 kq_status kq_sensitivity(const float* H_X, int64_t d_in, int64_t ldhx,
                          const float* H_G, int64_t d_out, int64_t ldhg,
                          double* out3, kq_stream_t stream);
+/* The same with H_G in the block-diagonal layout of kq_accum_cov_blocks
+ * (d_out x k, block b in rows b k .., ldhgb >= k): tr(H_G) is the sum of
+ * the blocks' traces. */
+kq_status kq_sensitivity_blocks(const float* H_X, int64_t d_in, int64_t ldhx, const float* H_Gb,
+                                int64_t d_out, int64_t k, int64_t ldhgb, double* out3, kq_stream_t stream);
 
 /* --------------------------------------------------------------------------
  * kq_rotate - randomised Hadamard rotation (steps a4/a5, BiIP).
@@ -319,6 +372,20 @@ kq_status kq_kron_loss_multi(const float* W, int64_t ldw, int count, const float
                              int64_t ldwh, int64_t d_out, int64_t d_in,
                              const float* H_X, int64_t ldhx, const float* H_G, int64_t ldhg,
                              double* const* loss, void* ws, size_t ws_bytes, kq_stream_t stream);
+
+/* kq_kron_loss_blocks - the Kronecker loss with the blockwise H_G of
+ * kq_accum_cov_blocks: sum over the row blocks b of
+ * tr(dW_b H_X dW_b^T H_G,b), dW_b = rows b k .. b k + k - 1 of W - W_hat and
+ * H_G,b = rows b k .. of H_Gb (d_out x k, ldhgb >= k): the loss of the
+ * block-diagonal matrix the blocks form (KronQ review, Limitations, second
+ * limitation; research thread, "Sparks": blockwise H_G).  Each block as
+ * kq_kron_loss (3xTF32 products, same symmetry reading), the partials of all
+ * blocks summed in one fixed order.  k divides d_out.  Workspace
+ * kq_kron_loss_blocks_workspace_size(d_out, d_in, k). */
+size_t kq_kron_loss_blocks_workspace_size(int64_t d_out, int64_t d_in, int64_t k);
+kq_status kq_kron_loss_blocks(const float* W, int64_t ldw, const float* W_hat, int64_t ldwh, int64_t d_out,
+                              int64_t d_in, const float* H_X, int64_t ldhx, const float* H_Gb, int64_t k,
+                              int64_t ldhgb, double* loss, void* ws, size_t ws_bytes, kq_stream_t stream);
 
 /* --------------------------------------------------------------------------
  * kq_kron_loss_noalloc - kq_kron_loss without a caller workspace.

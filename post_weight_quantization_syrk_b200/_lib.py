@@ -28,14 +28,16 @@ KQ_GEMM_FP32, KQ_GEMM_3XTF32 = 0, 1
 # Every symbol the header declares.
 EXPORTS = (
     "kq_status_string", "kq_last_error", "kq_version", "kq_launch_count", "kq_set_wait_limit_ns",
-    "kq_accum_cov_workspace_size", "kq_accum_cov",
+    "kq_accum_cov_workspace_size", "kq_accum_cov", "kq_accum_cov_blocks_workspace_size", "kq_accum_cov_blocks",
+    "kq_channel_energy_workspace_size", "kq_channel_energy", "kq_balance_permutation", "kq_gather",
     "kq_pack_codes", "kq_reverted_matvec_workspace_size", "kq_reverted_matvec",
-    "kq_sensitivity",
+    "kq_sensitivity", "kq_sensitivity_blocks",
     "kq_rotate",
     "kq_chol_inv_workspace_size", "kq_chol_inv",
     "kq_quantize_layer_workspace_size", "kq_quantize_layer", "kq_quantize_layer_multi_workspace_size",
     "kq_quantize_layer_multi", "kq_solver_timing",
     "kq_kron_loss_workspace_size", "kq_kron_loss", "kq_kron_loss_multi", "kq_kron_loss_noalloc",
+    "kq_kron_loss_blocks_workspace_size", "kq_kron_loss_blocks",
     "kq_allocate_bits",
 )
 
@@ -71,6 +73,13 @@ _SIGS = {
     "kq_accum_cov_workspace_size": (_sz, [_i64, _i64]),
     "kq_accum_cov": (_i32, [_vp, _i64, _i64, _i64, _vp, _i64, _f32, _i32, _vp, _sz, _vp, _vp]),
     "kq_sensitivity": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _vp, _vp]),
+    "kq_sensitivity_blocks": (_i32, [_vp, _i64, _i64, _vp, _i64, _i64, _i64, _vp, _vp]),
+    "kq_accum_cov_blocks_workspace_size": (_sz, [_i64, _i64, _i64]),
+    "kq_accum_cov_blocks": (_i32, [_vp, _i64, _i64, _i64, _i64, _vp, _i64, _f32, _i32, _vp, _sz, _vp, _vp]),
+    "kq_channel_energy_workspace_size": (_sz, [_i64]),
+    "kq_channel_energy": (_i32, [_vp, _i64, _i64, _i64, _f32, _vp, _vp, _sz, _vp, _vp]),
+    "kq_balance_permutation": (_i32, [_vp, _i64, _i64, _vp, _vp]),
+    "kq_gather": (_i32, [_vp, _i64, _i32, _vp, _vp, _i64, _i64, _vp, _i64, _vp, _vp]),
     "kq_rotate": (_i32, [_vp, _i64, _i64, _i64, _i32, ctypes.POINTER(kq_rht), _i32, _vp]),
     "kq_chol_inv_workspace_size": (_sz, [_i64]),
     "kq_chol_inv": (_i32, [_vp, _i64, _i64, _f32, _vp, _i64, _vp, _vp, _sz, _vp, _vp]),
@@ -84,6 +93,8 @@ _SIGS = {
                                        _vp, _vp]),
     "kq_solver_timing": (_i32, [_i32, ctypes.POINTER(kq_solver_times)]),
     "kq_kron_loss_workspace_size": (_sz, [_i64, _i64]),
+    "kq_kron_loss_blocks_workspace_size": (_sz, [_i64, _i64, _i64]),
+    "kq_kron_loss_blocks": (_i32, [_vp, _i64, _vp, _i64, _i64, _i64, _vp, _i64, _vp, _i64, _i64, _vp, _vp, _sz, _vp]),
     "kq_kron_loss_multi": (_i32, [_vp, _i64, _i32, ctypes.POINTER(_vp), _i64, _i64, _i64, _vp, _i64, _vp, _i64,
                                   ctypes.POINTER(_vp), _vp, _sz, _vp]),
     "kq_kron_loss": (_i32, [_vp, _i64, _vp, _i64, _i64, _i64, _vp, _i64, _vp, _i64, _vp, _vp, _sz, _vp]),
@@ -193,6 +204,72 @@ def kq_accum_cov(A, C, alpha, accumulate=False, ws=None, info=None, stream=None)
     wp, wb = _buf(ws)
     _check(load().kq_accum_cov(_ptr(A), n, d, lda, _ptr(C), ldc, float(alpha), int(bool(accumulate)),
                                wp, wb, _ptr(info), _stream(stream)), "kq_accum_cov")
+
+
+def kq_sensitivity_blocks(H_X, H_Gb, out3, stream=None):
+    """out3 = tr H_X, tr H_G, product, with H_G in the block layout [d_out, k]."""
+    ldx = _mat(H_X, torch.float32, "H_X")
+    ldg = _mat(H_Gb, torch.float32, "H_Gb")
+    if out3.dtype != torch.float64 or out3.numel() < 3 or not out3.is_cuda:
+        raise TypeError("out3 must be a CUDA float64 tensor of 3 elements")
+    _check(load().kq_sensitivity_blocks(_ptr(H_X), H_X.shape[0], ldx, _ptr(H_Gb), H_Gb.shape[0], H_Gb.shape[1], ldg,
+                                        _ptr(out3), _stream(stream)), "kq_sensitivity_blocks")
+
+
+def kq_accum_cov_blocks_workspace_size(n: int, d: int, k: int) -> int:
+    return int(load().kq_accum_cov_blocks_workspace_size(int(n), int(d), int(k)))
+
+
+def kq_accum_cov_blocks(A, k, C, alpha, accumulate=False, ws=None, info=None, stream=None):
+    """The k x k diagonal blocks of alpha * A^T A into C fp32 [d, k] (block b in rows b k ..)."""
+    lda = _mat(A, torch.bfloat16, "A")
+    ldc = _mat(C, torch.float32, "C")
+    n, d = A.shape
+    if C.shape != (d, k):
+        raise ValueError("C must be [d, k]")
+    if ws is None:
+        ws = workspace(kq_accum_cov_blocks_workspace_size(n, d, k), A.device)
+    wp, wb = _buf(ws)
+    _check(load().kq_accum_cov_blocks(_ptr(A), n, d, lda, int(k), _ptr(C), ldc, float(alpha), int(bool(accumulate)),
+                                      wp, wb, _ptr(info), _stream(stream)), "kq_accum_cov_blocks")
+
+
+def kq_channel_energy(A, out, alpha, ws=None, info=None, stream=None):
+    """out fp32 [d] = alpha * sum_t A[t, j]^2 for bf16 A [n, d]."""
+    lda = _mat(A, torch.bfloat16, "A")
+    n, d = A.shape
+    if out.dtype != torch.float32 or not out.is_cuda or out.numel() < d:
+        raise TypeError("out must be a CUDA float32 tensor of d elements")
+    if ws is None:
+        ws = workspace(int(load().kq_channel_energy_workspace_size(d)), A.device)
+    wp, wb = _buf(ws)
+    _check(load().kq_channel_energy(_ptr(A), n, d, lda, float(alpha), _ptr(out), wp, wb, _ptr(info),
+                                    _stream(stream)), "kq_channel_energy")
+
+
+def kq_balance_permutation(energy, k, perm, stream=None):
+    """perm int64 [d]: output channels dealt to d/k blocks by descending energy."""
+    d = energy.numel()
+    if energy.dtype != torch.float32 or perm.dtype != torch.int64 or perm.numel() < d:
+        raise TypeError("energy float32 [d], perm int64 [d]")
+    _check(load().kq_balance_permutation(_ptr(energy), d, int(k), _ptr(perm), _stream(stream)),
+           "kq_balance_permutation")
+
+
+def kq_gather(M, out, row_idx=None, col_idx=None, info=None, stream=None):
+    """out[i, j] = M[row_idx[i], col_idx[j]] (either index may be None) for
+    float32 or bf16 matrices of the same shape."""
+    if M.dtype != out.dtype or M.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("M and out must both be float32 or both bf16")
+    ldm = _mat(M, M.dtype, "M")
+    ldo = _mat(out, out.dtype, "out")
+    if M.shape != out.shape:
+        raise ValueError("M and out must have the same shape")
+    for ix in (row_idx, col_idx):
+        if ix is not None and (ix.dtype != torch.int64 or not ix.is_cuda):
+            raise TypeError("indices must be CUDA int64 tensors")
+    _check(load().kq_gather(_ptr(M), ldm, M.element_size(), _ptr(row_idx), _ptr(col_idx), M.shape[0], M.shape[1],
+                            _ptr(out), ldo, _ptr(info), _stream(stream)), "kq_gather")
 
 
 def kq_sensitivity(H_X, H_G, out3, stream=None):
@@ -344,6 +421,29 @@ def kq_kron_loss_multi(W, W_hats, H_X, H_G, losses, ws=None, stream=None):
     wp, wb = _buf(ws)
     _check(load().kq_kron_loss_multi(_ptr(W), ldw, k, _ptrs(W_hats), ldh, d_out, d_in, _ptr(H_X), ldx, _ptr(H_G), ldg,
                                      _ptrs(losses), wp, wb, _stream(stream)), "kq_kron_loss_multi")
+
+
+def kq_kron_loss_blocks_workspace_size(d_out: int, d_in: int, k: int) -> int:
+    return int(load().kq_kron_loss_blocks_workspace_size(int(d_out), int(d_in), int(k)))
+
+
+def kq_kron_loss_blocks(W, W_hat, H_X, H_Gb, loss, ws=None, stream=None):
+    """Kronecker loss with the block-diagonal H_G given as H_Gb [d_out, k]."""
+    ldw = _mat(W, torch.float32, "W")
+    ldh = _mat(W_hat, torch.float32, "W_hat")
+    ldx = _mat(H_X, torch.float32, "H_X")
+    ldg = _mat(H_Gb, torch.float32, "H_Gb")
+    d_out, d_in = W.shape
+    k = H_Gb.shape[1]
+    if H_Gb.shape[0] != d_out:
+        raise ValueError("H_Gb must be [d_out, k]")
+    if loss.dtype != torch.float64 or not loss.is_cuda:
+        raise TypeError("loss must be a CUDA float64 tensor")
+    if ws is None:
+        ws = workspace(kq_kron_loss_blocks_workspace_size(d_out, d_in, k), W.device)
+    wp, wb = _buf(ws)
+    _check(load().kq_kron_loss_blocks(_ptr(W), ldw, _ptr(W_hat), ldh, d_out, d_in, _ptr(H_X), ldx, _ptr(H_Gb), k, ldg,
+                                      _ptr(loss), wp, wb, _stream(stream)), "kq_kron_loss_blocks")
 
 
 def kq_kron_loss_noalloc(W, W_hat, H_X, H_G, loss, stream=None):

@@ -171,22 +171,18 @@ extern "C" size_t kq_kron_loss_workspace_size(int64_t d_out, int64_t d_in) {
 
 namespace {
 
-// One loss; the tf32 split of the smaller Hessian is formed here unless
-// `split_h` is false (then it is already in the workspace from an earlier
-// call with the same H_X, H_G and shape).
-kq_status kron_loss_impl(const float* W, int64_t ldw, const float* W_hat, int64_t ldwh, int64_t d_out, int64_t d_in,
-                         const float* H_X, int64_t ldhx, const float* H_G, int64_t ldhg, double* loss, void* ws,
-                         size_t ws_bytes, kq_stream_t stream, bool split_h) {
-  if (!W || !W_hat || !H_X || !loss) return kq::fail(KQ_ERR_INVALID_ARG, "kq_kron_loss: NULL pointer");
-  if (d_out < 1 || d_in < 1) return kq::fail(KQ_ERR_INVALID_ARG, "kq_kron_loss: sizes must be >= 1");
-  if (d_out > 65536 || d_in > 65536) return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_kron_loss: sizes above 65536");
-  if (ldw < d_in || ldwh < d_in || ldhx < d_in || (H_G && ldhg < d_out))
-    return kq::fail(KQ_ERR_INVALID_ARG, "kq_kron_loss: leading dimension too small");
-  if (!ws || !kq::aligned(ws, 256) || ws_bytes < kq_kron_loss_workspace_size(d_out, d_in))
-    return kq::fail(KQ_ERR_WORKSPACE, "kq_kron_loss: workspace too small or not 256-byte aligned");
+// The products of one loss, their fp64 partials written from `partial`
+// (or the workspace's own region when NULL); *np_out = how many.  The tf32
+// split of the smaller Hessian is formed here unless `split_h` is false
+// (then it is already in the workspace from an earlier call with the same
+// H_X, H_G and shape).
+kq_status kron_loss_products(const float* W, int64_t ldw, const float* W_hat, int64_t ldwh, int64_t d_out,
+                             int64_t d_in, const float* H_X, int64_t ldhx, const float* H_G, int64_t ldhg, void* ws,
+                             kq_stream_t stream, bool split_h, double* partial, int64_t* np_out) {
   cudaStream_t st = (cudaStream_t)stream;
   LossWs w;
   loss_layout(d_out, d_in, &w, ws);
+  if (partial) w.partial = partial;
   // orientation: the smaller Hessian goes into the product (see the top of this file)
   const bool g_first = !H_G || d_in > d_out;
   const int64_t n2 = g_first ? d_in : d_out, n1 = g_first ? d_out : d_in, ldd = lead(n1);
@@ -233,7 +229,27 @@ kq_status kron_loss_impl(const float* W, int64_t ldw, const float* W_hat, int64_
   g2.ld_other = ld2;
   g2.partial = w.partial;
   KQ_TRY(kq::gemm_3xtf32(g2, st));
-  const int64_t np = 8 * kq::gemm_tiles(n2, n2, n1, true);
+  *np_out = 8 * kq::gemm_tiles(n2, n2, n1, true);
+  return KQ_OK;
+}
+
+// One loss; see kron_loss_products for `split_h`.
+kq_status kron_loss_impl(const float* W, int64_t ldw, const float* W_hat, int64_t ldwh, int64_t d_out, int64_t d_in,
+                         const float* H_X, int64_t ldhx, const float* H_G, int64_t ldhg, double* loss, void* ws,
+                         size_t ws_bytes, kq_stream_t stream, bool split_h) {
+  if (!W || !W_hat || !H_X || !loss) return kq::fail(KQ_ERR_INVALID_ARG, "kq_kron_loss: NULL pointer");
+  if (d_out < 1 || d_in < 1) return kq::fail(KQ_ERR_INVALID_ARG, "kq_kron_loss: sizes must be >= 1");
+  if (d_out > 65536 || d_in > 65536) return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_kron_loss: sizes above 65536");
+  if (ldw < d_in || ldwh < d_in || ldhx < d_in || (H_G && ldhg < d_out))
+    return kq::fail(KQ_ERR_INVALID_ARG, "kq_kron_loss: leading dimension too small");
+  if (!ws || !kq::aligned(ws, 256) || ws_bytes < kq_kron_loss_workspace_size(d_out, d_in))
+    return kq::fail(KQ_ERR_WORKSPACE, "kq_kron_loss: workspace too small or not 256-byte aligned");
+  cudaStream_t st = (cudaStream_t)stream;
+  int64_t np = 0;
+  KQ_TRY(kron_loss_products(W, ldw, W_hat, ldwh, d_out, d_in, H_X, ldhx, H_G, ldhg, ws, stream, split_h, nullptr,
+                            &np));
+  LossWs w;
+  loss_layout(d_out, d_in, &w, ws);
   sum_kernel<<<1, 1024, 0, st>>>(w.partial, np, loss);
   KQ_TRY(kq::launch_check("kq_kron_loss sum"));
   kq::clear_error();
@@ -241,6 +257,48 @@ kq_status kron_loss_impl(const float* W, int64_t ldw, const float* W_hat, int64_
 }
 
 }  // namespace
+
+// Blockwise loss: the products of every row block into one partial region
+// after the per-block workspace, then one fixed-order sum.
+size_t blocks_partial_offset(int64_t d_in, int64_t k) {
+  return kq::align_up(loss_layout(k, d_in, nullptr, nullptr), 256);
+}
+
+extern "C" size_t kq_kron_loss_blocks_workspace_size(int64_t d_out, int64_t d_in, int64_t k) {
+  if (d_out < 1 || d_in < 1 || k < 1 || d_out % k) return 0;
+  const int64_t n2 = std::max(k, d_in), n1 = std::min(k, d_in);
+  return blocks_partial_offset(d_in, k) + (size_t)(d_out / k) * 8 * kq::gemm_tiles(n2, n2, n1, true) * sizeof(double);
+}
+
+extern "C" kq_status kq_kron_loss_blocks(const float* W, int64_t ldw, const float* W_hat, int64_t ldwh, int64_t d_out,
+                                         int64_t d_in, const float* H_X, int64_t ldhx, const float* H_Gb, int64_t k,
+                                         int64_t ldhgb, double* loss, void* ws, size_t ws_bytes,
+                                         kq_stream_t stream) {
+  if (!W || !W_hat || !H_X || !H_Gb || !loss) return kq::fail(KQ_ERR_INVALID_ARG, "kq_kron_loss_blocks: NULL pointer");
+  if (d_out < 1 || d_in < 1 || k < 1 || d_out % k)
+    return kq::fail(KQ_ERR_INVALID_ARG, "kq_kron_loss_blocks: sizes must be >= 1 and k must divide d_out");
+  if (d_out > 65536 || d_in > 65536) return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_kron_loss_blocks: sizes above 65536");
+  if (ldw < d_in || ldwh < d_in || ldhx < d_in || ldhgb < k)
+    return kq::fail(KQ_ERR_INVALID_ARG, "kq_kron_loss_blocks: leading dimension too small");
+  if (!ws || !kq::aligned(ws, 256) || ws_bytes < kq_kron_loss_blocks_workspace_size(d_out, d_in, k))
+    return kq::fail(KQ_ERR_WORKSPACE, "kq_kron_loss_blocks: workspace too small or not 256-byte aligned");
+  cudaStream_t st = (cudaStream_t)stream;
+  double* partial = reinterpret_cast<double*>(static_cast<char*>(ws) + blocks_partial_offset(d_in, k));
+  int64_t total = 0;
+  for (int64_t b = 0; b < d_out / k; ++b) {
+    int64_t np = 0;
+    // the smaller Hessian of a block is its H_G block when k < d_in: split
+    // it for every block; H_X (k >= d_in) only once
+    const bool split = (k < d_in) || b == 0;
+    KQ_TRY(kron_loss_products(W + b * k * ldw, ldw, W_hat + b * k * ldwh, ldwh, k, d_in, H_X, ldhx, H_Gb + b * k * ldhgb,
+                              ldhgb, ws, stream, split, partial + total, &np));
+    total += np;
+  }
+  sum_kernel<<<1, 1024, 0, st>>>(partial, total, loss);
+  KQ_TRY(kq::launch_check("kq_kron_loss_blocks sum"));
+  kq::clear_error();
+  return KQ_OK;
+}
 
 extern "C" kq_status kq_kron_loss(const float* W, int64_t ldw, const float* W_hat, int64_t ldwh, int64_t d_out,
                                   int64_t d_in, const float* H_X, int64_t ldhx, const float* H_G, int64_t ldhg,

@@ -9,14 +9,16 @@ namespace {
 
 constexpr int kThreads = 512;
 
+// H_G's diagonal entry i at HG[i * ldg + i % kg]: kg = dg for the whole
+// matrix, kg = k for the block-diagonal d x k layout (block b in rows b k ..).
 __global__ void __launch_bounds__(kThreads) trace_kernel(const float* __restrict__ HX, int64_t dx, int64_t ldx,
                                                           const float* __restrict__ HG, int64_t dg, int64_t ldg,
-                                                          double* __restrict__ out3) {
+                                                          int64_t kg, double* __restrict__ out3) {
   __shared__ double sx[kThreads];
   __shared__ double sg[kThreads];
   double ax = 0.0, ag = 0.0;
   for (int64_t i = threadIdx.x; i < dx; i += kThreads) ax += (double)HX[i * ldx + i];
-  for (int64_t i = threadIdx.x; i < dg; i += kThreads) ag += (double)HG[i * ldg + i];
+  for (int64_t i = threadIdx.x; i < dg; i += kThreads) ag += (double)HG[i * ldg + i % kg];
   sx[threadIdx.x] = ax;
   sg[threadIdx.x] = ag;
   __syncthreads();
@@ -41,8 +43,20 @@ extern "C" kq_status kq_sensitivity(const float* H_X, int64_t d_in, int64_t ldhx
   if (!H_X || !H_G || !out3) return kq::fail(KQ_ERR_INVALID_ARG, "kq_sensitivity: NULL pointer");
   if (d_in < 1 || d_out < 1) return kq::fail(KQ_ERR_INVALID_ARG, "kq_sensitivity: sizes must be >= 1");
   if (ldhx < d_in || ldhg < d_out) return kq::fail(KQ_ERR_INVALID_ARG, "kq_sensitivity: leading dimension too small");
-  trace_kernel<<<1, kThreads, 0, (cudaStream_t)stream>>>(H_X, d_in, ldhx, H_G, d_out, ldhg, out3);
+  trace_kernel<<<1, kThreads, 0, (cudaStream_t)stream>>>(H_X, d_in, ldhx, H_G, d_out, ldhg, d_out, out3);
   KQ_TRY(kq::launch_check("kq_sensitivity"));
+  kq::clear_error();
+  return KQ_OK;
+}
+
+extern "C" kq_status kq_sensitivity_blocks(const float* H_X, int64_t d_in, int64_t ldhx, const float* H_Gb,
+                                           int64_t d_out, int64_t k, int64_t ldhgb, double* out3, kq_stream_t stream) {
+  if (!H_X || !H_Gb || !out3) return kq::fail(KQ_ERR_INVALID_ARG, "kq_sensitivity_blocks: NULL pointer");
+  if (d_in < 1 || d_out < 1 || k < 1 || d_out % k)
+    return kq::fail(KQ_ERR_INVALID_ARG, "kq_sensitivity_blocks: sizes must be >= 1 and k must divide d_out");
+  if (ldhx < d_in || ldhgb < k) return kq::fail(KQ_ERR_INVALID_ARG, "kq_sensitivity_blocks: leading dimension too small");
+  trace_kernel<<<1, kThreads, 0, (cudaStream_t)stream>>>(H_X, d_in, ldhx, H_Gb, d_out, ldhgb, k, out3);
+  KQ_TRY(kq::launch_check("kq_sensitivity_blocks"));
   kq::clear_error();
   return KQ_OK;
 }

@@ -62,6 +62,9 @@ struct Params {
   int64_t ldc;
   int c_vec;        // C rows 16-byte aligned (C aligned, ldc % 4 == 0)
   float* partial;   // [splits][num_tiles][256][256] when splits > 1
+  int kt;           // block-diagonal mode: tiles per diagonal block side (0: whole lower triangle)
+  int tiles_per_block;  // kt (kt + 1) / 2
+  int64_t blk;      // block-diagonal mode: block size k = 256 kt; C is [d, k], block b in rows b k ..
   int32_t* info;
   unsigned long long wait_ns;   // limit of each pipeline wait (kq_set_wait_limit_ns)
 };
@@ -83,10 +86,30 @@ __device__ __forceinline__ void tri_index(int64_t l, int* ti, int* tj) {
   *tj = (int)(l - t * (t + 1) / 2);
 }
 
+// Tile number -> (tile row, tile column): the lower triangle of the whole
+// matrix, or (block-diagonal mode) the lower triangles of the diagonal
+// blocks one after the other.
+__device__ __forceinline__ void tile_coords(const Params& p, int l, int* ti, int* tj) {
+  if (p.kt) {
+    const int b = l / p.tiles_per_block;
+    tri_index(l % p.tiles_per_block, ti, tj);
+    *ti += b * p.kt;
+    *tj += b * p.kt;
+  } else {
+    tri_index(l, ti, tj);
+  }
+}
+
+// Column of element (row gi, column gj <= gi of the same block) in C: the
+// block-diagonal mode stores each block's rows from column 0.
+__device__ __forceinline__ int64_t c_col(const Params& p, int64_t gi, int64_t gj) {
+  return p.kt ? gj - (gi / p.blk) * p.blk : gj;
+}
+
 // unit -> (tile, split); units of the same split are adjacent.
 __device__ __forceinline__ void unit_coords(const Params& p, int u, int* ti, int* tj, int* split) {
   *split = u / p.num_tiles;
-  tri_index(u % p.num_tiles, ti, tj);
+  tile_coords(p, u % p.num_tiles, ti, tj);
 }
 
 // ------------------------------------------------------------------ kernel
@@ -249,10 +272,10 @@ __global__ void __launch_bounds__(THREADS, 1) syrk_tc_kernel(const __grid_consta
               const int64_t gj = j0 + c0 + q;
               if (gj >= p.d || gj > gi) continue;
               float val = p.alpha * v[q];
-              if (p.accumulate) val += p.C[gi * p.ldc + gj];
+              if (p.accumulate) val += p.C[gi * p.ldc + c_col(p, gi, gj)];
               if (!isfinite(val)) kq::report(p.info, KQ_ERR_NONFINITE, gi);
-              p.C[gi * p.ldc + gj] = val;
-              p.C[gj * p.ldc + gi] = val;
+              p.C[gi * p.ldc + c_col(p, gi, gj)] = val;
+              p.C[gj * p.ldc + c_col(p, gj, gi)] = val;
             }
           }
         }
@@ -283,7 +306,7 @@ __global__ void __launch_bounds__(256) split_reduce_kernel(Params p) {
   const int tile = blockIdx.x / 8;
   const int band = blockIdx.x % 8;  // 32-row band within the 256-row tile
   int ti, tj;
-  tri_index(tile, &ti, &tj);
+  tile_coords(p, tile, &ti, &tj);
   const int64_t i0 = (int64_t)ti * TILE + band * 32, j0 = (int64_t)tj * TILE;
   const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
   const int64_t split_stride = (int64_t)p.num_tiles * TILE * TILE;
@@ -333,7 +356,7 @@ __global__ void __launch_bounds__(256) split_reduce_kernel(Params p) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) v[e] = p.alpha * acc[k][e];
       if (gi < p.d) {
-        float* c = p.C + gi * p.ldc + gj;
+        float* c = p.C + gi * p.ldc + c_col(p, gi, gj);
         if (p.c_vec && gj + 3 < p.d && gj + 3 <= gi) {
           if (p.accumulate) {
             const float4 o = *reinterpret_cast<const float4*>(c);
@@ -362,18 +385,18 @@ __global__ void __launch_bounds__(256) split_reduce_kernel(Params p) {
     // mirror: row j0 + h * 128 + c, columns i0 .. i0 + 31 (one per lane)
     for (int c = warp; c < 128; c += 8) {
       const int64_t gj2 = j0 + h * 128 + c, gi2 = i0 + lane;
-      if (gi2 < p.d && gj2 < p.d && gj2 < gi2) p.C[gj2 * p.ldc + gi2] = t[lane][c];
+      if (gi2 < p.d && gj2 < p.d && gj2 < gi2) p.C[gj2 * p.ldc + c_col(p, gj2, gi2)] = t[lane][c];
     }
     __syncthreads();
   }
 }
 
-__global__ void scale_or_zero_kernel(float* C, int64_t d, int64_t ldc, int accumulate) {
-  // n == 0: C = 0 (overwrite) or unchanged (accumulate)
+__global__ void scale_or_zero_kernel(float* C, int64_t d, int64_t cols, int64_t ldc, int accumulate) {
+  // n == 0: C = 0 (overwrite) or unchanged (accumulate); C is d x cols
   if (accumulate) return;
-  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < d * d;
+  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < d * cols;
        idx += (int64_t)gridDim.x * blockDim.x)
-    C[(idx / d) * ldc + idx % d] = 0.f;
+    C[(idx / cols) * ldc + idx % cols] = 0.f;
 }
 
 // ------------------------------------------------------------------ host
@@ -393,10 +416,14 @@ constexpr int kMaxKbPerSplit = 192;   // 12288 tokens
 // Token splits per tile: minimise (waves / splits) x full-tile MMA time plus
 // the partial-tile round trip through HBM, with waves counted on 148 SMs,
 // subject to the chain-length cap above.
-Plan make_plan(int64_t n, int64_t d) {
+Plan make_plan(int64_t n, int64_t d, int64_t blk = 0) {
   Plan pl;
   pl.T = (int)kq::cdiv(d, TILE);
   pl.num_tiles = pl.T * (pl.T + 1) / 2;
+  if (blk) {   // block-diagonal mode: d / blk blocks of (blk / 256)^2 / 2 tiles
+    const int kt = (int)(blk / TILE);
+    pl.num_tiles = (int)(d / blk) * (kt * (kt + 1) / 2);
+  }
   pl.kblocks = (int)kq::cdiv(n, BK);
   const double tile_s = 2.0 * TILE * TILE * (double)n / (1.4e15 / ASSUMED_SMS);
   double best = 1e300;
@@ -424,34 +451,40 @@ Plan make_plan(int64_t n, int64_t d) {
 
 }  // namespace
 
-extern "C" size_t kq_accum_cov_workspace_size(int64_t n, int64_t d) {
+namespace {
+
+size_t accum_ws_size(int64_t n, int64_t d, int64_t blk) {
   if (n <= 0 || d < 1) return 0;
-  Plan pl = make_plan(n, d);
+  Plan pl = make_plan(n, d, blk);
   if (pl.splits == 1) return 0;
   return kq::align_up((size_t)pl.num_units * TILE * TILE * sizeof(float), 256);
 }
 
-extern "C" kq_status kq_accum_cov(const uint16_t* A, int64_t n, int64_t d, int64_t lda, float* C, int64_t ldc,
-                                  float alpha, int accumulate, void* ws, size_t ws_bytes, int32_t* info,
-                                  kq_stream_t stream) {
-  if ((!A && n > 0) || !C || !info) return kq::fail(KQ_ERR_INVALID_ARG, "kq_accum_cov: NULL pointer");
-  if (n < 0 || d < 1 || d > 65536) return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_accum_cov: need n >= 0, 1 <= d <= 65536");
-  if (n > ((int64_t)1 << 31) - BK) return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_accum_cov: n above 2^31 - 64");
-  if (lda < d || ldc < d) return kq::fail(KQ_ERR_INVALID_ARG, "kq_accum_cov: leading dimension too small");
+// C (+)= alpha A^T A: the whole symmetric matrix (blk == 0) or only its
+// blk x blk diagonal blocks (blk a multiple of 256 dividing d), C then being
+// d x blk with block b in rows b blk .. b blk + blk - 1.
+kq_status accum_cov_impl(const char* name, const uint16_t* A, int64_t n, int64_t d, int64_t lda, float* C,
+                         int64_t ldc, float alpha, int accumulate, void* ws, size_t ws_bytes, int32_t* info,
+                         kq_stream_t stream, int64_t blk) {
+  const int64_t cols = blk ? blk : d;
+  if ((!A && n > 0) || !C || !info) return kq::fail(KQ_ERR_INVALID_ARG, "%s: NULL pointer", name);
+  if (n < 0 || d < 1 || d > 65536) return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "%s: need n >= 0, 1 <= d <= 65536", name);
+  if (n > ((int64_t)1 << 31) - BK) return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "%s: n above 2^31 - 64", name);
+  if (lda < d || ldc < cols) return kq::fail(KQ_ERR_INVALID_ARG, "%s: leading dimension too small", name);
   if ((n > 0 && !kq::aligned(A, 16)) || (lda & 7))
-    return kq::fail(KQ_ERR_ALIGNMENT, "kq_accum_cov: A 16-byte aligned, lda %% 8 == 0");
-  if (!isfinite(alpha)) return kq::fail(KQ_ERR_INVALID_ARG, "kq_accum_cov: alpha not finite");
+    return kq::fail(KQ_ERR_ALIGNMENT, "%s: A 16-byte aligned, lda %% 8 == 0", name);
+  if (!isfinite(alpha)) return kq::fail(KQ_ERR_INVALID_ARG, "%s: alpha not finite", name);
   cudaStream_t st = (cudaStream_t)stream;
   if (n == 0) {
-    scale_or_zero_kernel<<<256, 256, 0, st>>>(C, d, ldc, accumulate);
-    KQ_TRY(kq::launch_check("kq_accum_cov zero"));
+    scale_or_zero_kernel<<<256, 256, 0, st>>>(C, d, cols, ldc, accumulate);
+    KQ_TRY(kq::launch_check(name));
     kq::clear_error();
     return KQ_OK;
   }
-  Plan pl = make_plan(n, d);
-  const size_t need = kq_accum_cov_workspace_size(n, d);
+  Plan pl = make_plan(n, d, blk);
+  const size_t need = accum_ws_size(n, d, blk);
   if (need && (!ws || !kq::aligned(ws, 256) || ws_bytes < need))
-    return kq::fail(KQ_ERR_WORKSPACE, "kq_accum_cov: workspace of %zu bytes needed", need);
+    return kq::fail(KQ_ERR_WORKSPACE, "%s: workspace of %zu bytes needed", name, need);
 
   CUtensorMap tmap;
   KQ_TRY(make_map_2d(&tmap, A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, n, lda, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B));
@@ -471,6 +504,9 @@ extern "C" kq_status kq_accum_cov(const uint16_t* A, int64_t n, int64_t d, int64
   p.ldc = ldc;
   p.c_vec = (kq::aligned(C, 16) && !(ldc & 3)) ? 1 : 0;
   p.partial = static_cast<float*>(ws);
+  p.kt = blk ? (int)(blk / TILE) : 0;
+  p.tiles_per_block = p.kt * (p.kt + 1) / 2;
+  p.blk = blk;
   p.info = info;
   p.wait_ns = kq::wait_limit_ns();
 
@@ -481,11 +517,35 @@ extern "C" kq_status kq_accum_cov(const uint16_t* A, int64_t n, int64_t d, int64
                         "kq_accum_cov: smem attribute"));
   const int grid = std::min(pl.num_units, sms);
   syrk_tc_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(tmap, p);
-  KQ_TRY(kq::launch_check("kq_accum_cov"));
+  KQ_TRY(kq::launch_check(name));
   if (pl.splits > 1) {
     split_reduce_kernel<<<pl.num_tiles * 8, 256, 0, st>>>(p);
-    KQ_TRY(kq::launch_check("kq_accum_cov reduce"));
+    KQ_TRY(kq::launch_check(name));
   }
   kq::clear_error();
   return KQ_OK;
+}
+
+}  // namespace
+
+extern "C" size_t kq_accum_cov_workspace_size(int64_t n, int64_t d) { return accum_ws_size(n, d, 0); }
+
+extern "C" kq_status kq_accum_cov(const uint16_t* A, int64_t n, int64_t d, int64_t lda, float* C, int64_t ldc,
+                                  float alpha, int accumulate, void* ws, size_t ws_bytes, int32_t* info,
+                                  kq_stream_t stream) {
+  return accum_cov_impl("kq_accum_cov", A, n, d, lda, C, ldc, alpha, accumulate, ws, ws_bytes, info, stream, 0);
+}
+
+extern "C" size_t kq_accum_cov_blocks_workspace_size(int64_t n, int64_t d, int64_t k) {
+  if (k < 256 || k % 256 || d % k) return 0;
+  return accum_ws_size(n, d, k);
+}
+
+extern "C" kq_status kq_accum_cov_blocks(const uint16_t* A, int64_t n, int64_t d, int64_t lda, int64_t k, float* C,
+                                         int64_t ldc, float alpha, int accumulate, void* ws, size_t ws_bytes,
+                                         int32_t* info, kq_stream_t stream) {
+  if (k < 256 || k % 256 || d % k)
+    return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_accum_cov_blocks: k must be a multiple of 256 dividing d");
+  return accum_cov_impl("kq_accum_cov_blocks", A, n, d, lda, C, ldc, alpha, accumulate, ws, ws_bytes, info, stream,
+                        k);
 }

@@ -32,13 +32,14 @@ class BitResult:
 class LayerQuantizer:
     """Device buffers for one (d_out, d_in) layer and the calls that fill them."""
 
-    def __init__(self, d_out, d_in, device="cuda", block=128, gemm_mode=K.KQ_GEMM_FP32):
+    def __init__(self, d_out, d_in, device="cuda", block=128, gemm_mode=K.KQ_GEMM_FP32, full_hg=True):
         self.d_out, self.d_in, self.block, self.gemm_mode = d_out, d_in, block, gemm_mode
         dev = torch.device(device)
         self.device = dev
         f32 = dict(dtype=torch.float32, device=dev)
         self.H_X = torch.empty((d_in, d_in), **f32)
-        self.H_G = torch.empty((d_out, d_out), **f32)
+        self.H_G = torch.empty((d_out, d_out), **f32) if full_hg else None
+        self.perm = None
         self.Wp = torch.empty((d_out, d_in), **f32)
         self.Uc = torch.empty((d_in, d_in), **f32)
         self.dead = torch.zeros(d_in, dtype=torch.uint8, device=dev)
@@ -77,9 +78,29 @@ class LayerQuantizer:
     def sensitivity(self, stream=None):
         K.kq_sensitivity(self.H_X, self.H_G, self.sens, stream)
 
+    def hg_permutation(self, G, k, n_total=None, stream=None):
+        """The H_G-informed factor P_G of the output rotation V = T P_G:
+        output channels ranked by descending gradient energy diag(H_G)
+        (ties: lower index) and dealt round-robin to d_out / k blocks
+        (kq_channel_energy, kq_balance_permutation).  rotate() then applies
+        P_G before T."""
+        n_total = G.shape[0] if n_total is None else n_total
+        energy = torch.empty(self.d_out, dtype=torch.float32, device=self.device)
+        K.kq_channel_energy(G, energy, 1.0 / n_total, None, self.info, stream)
+        self.perm = torch.empty(self.d_out, dtype=torch.int64, device=self.device)
+        K.kq_balance_permutation(energy, k, self.perm, stream)
+
     def rotate(self, W, T_in: K.RHT, T_out: K.RHT, stream=None):
-        """W' = V W U^T, H_X' = U H_X U^T, H_G' = V H_G V^T (in the layer's buffers)."""
-        self.Wp.copy_(W)
+        """W' = V W U^T, H_X' = U H_X U^T, H_G' = V H_G V^T (in the layer's
+        buffers), V = T_out, or T_out P_G after hg_permutation()."""
+        if self.perm is not None:
+            K.kq_gather(W, self.Wp, self.perm, None, self.info, stream)
+            tmp = torch.empty_like(self.H_G)
+            K.kq_gather(self.H_G, tmp, self.perm, self.perm, self.info, stream)
+            self.H_G.copy_(tmp)
+            del tmp
+        else:
+            self.Wp.copy_(W)
         K.kq_rotate(self.Wp, K.KQ_AXIS_COLS, T_in, False, stream)
         K.kq_rotate(self.Wp, K.KQ_AXIS_ROWS, T_out, False, stream)
         K.kq_rotate(self.H_X, K.KQ_AXIS_COLS, T_in, False, stream)
@@ -129,6 +150,93 @@ class LayerQuantizer:
 
     def check(self, where="kronq"):
         K.check_info(self.info, where)
+
+
+class BlockwiseLayerQuantizer(LayerQuantizer):
+    """One layer whose output side never forms the full d_out x d_out H_G.
+
+    KronQ review, Limitations (second limitation: BiIP holds the full H_G, a
+    transient peak of memory) and the research thread's "Sparks" (blockwise
+    H_G); KronQ paper page, Abstract (1) (the output rotation uses the
+    gradient covariance).  Only the k x k diagonal blocks of H_G are formed
+    (kq_accum_cov_blocks: d_out k floats), the output rotation is block
+    diagonal, V = (I kron T_k) P_G, so that V H_G V^T stays block diagonal
+    and is rotated block by block, and the loss is that of the block-diagonal
+    H_G (kq_kron_loss_blocks).  With balanced=True, P_G is the permutation
+    dealing output channels to blocks by descending gradient energy
+    (kq_channel_energy, kq_balance_permutation): it needs a transient
+    column-permuted copy of G (kq_gather); balanced=False takes P_G = I.
+    The input side and the solver are those of LayerQuantizer.
+    """
+
+    def __init__(self, d_out, d_in, k, balanced=True, device="cuda", block=128, gemm_mode=K.KQ_GEMM_FP32):
+        if d_out % k or k % 256:
+            raise ValueError("k must be a multiple of 256 dividing d_out")
+        self.k, self.balanced = k, balanced
+        super().__init__(d_out, d_in, device, block, gemm_mode, full_hg=False)   # H_G never formed
+        dev = self.device
+        self.H_Gb = torch.empty((d_out, k), dtype=torch.float32, device=dev)
+        self.energy = torch.empty(d_out, dtype=torch.float32, device=dev)
+        self.perm = torch.arange(d_out, dtype=torch.int64, device=dev)
+
+    def statistics(self, X, G, n_total=None, accumulate=False, stream=None):
+        if accumulate:
+            raise ValueError("the blockwise output side takes all calibration tokens in one call")
+        n_total = X.shape[0] if n_total is None else n_total
+        alpha = 1.0 / n_total if n_total else 0.0
+        ws = self.workspace(max(K.kq_accum_cov_workspace_size(X.shape[0], self.d_in),
+                                K.kq_accum_cov_blocks_workspace_size(G.shape[0], self.d_out, self.k)))
+        K.kq_accum_cov(X, self.H_X, alpha, False, ws, self.info, stream)
+        if self.balanced:
+            K.kq_channel_energy(G, self.energy, alpha, None, self.info, stream)
+            K.kq_balance_permutation(self.energy, self.k, self.perm, stream)
+            Gp = torch.empty_like(G)                           # transient, the size of G
+            K.kq_gather(G, Gp, None, self.perm, self.info, stream)
+            K.kq_accum_cov_blocks(Gp, self.k, self.H_Gb, alpha, False, ws, self.info, stream)
+            del Gp
+        else:
+            K.kq_accum_cov_blocks(G, self.k, self.H_Gb, alpha, False, ws, self.info, stream)
+
+    def sensitivity(self, stream=None):
+        K.kq_sensitivity_blocks(self.H_X, self.H_Gb, self.sens, stream)
+
+    def rotate(self, W, T_in: K.RHT, T_k: K.RHT, stream=None):
+        """W' = (I kron T_k) P_G W U^T, H_X' = U H_X U^T, each H_G block T_k B T_k^T."""
+        k = self.k
+        if self.balanced:
+            K.kq_gather(W, self.Wp, self.perm, None, self.info, stream)
+        else:
+            self.Wp.copy_(W)
+        K.kq_rotate(self.Wp, K.KQ_AXIS_COLS, T_in, False, stream)
+        for b in range(self.d_out // k):
+            K.kq_rotate(self.Wp[b * k:(b + 1) * k], K.KQ_AXIS_ROWS, T_k, False, stream)
+        K.kq_rotate(self.H_X, K.KQ_AXIS_COLS, T_in, False, stream)
+        K.kq_rotate(self.H_X, K.KQ_AXIS_ROWS, T_in, False, stream)
+        for b in range(self.d_out // k):
+            Hb = self.H_Gb[b * k:(b + 1) * k]
+            K.kq_rotate(Hb, K.KQ_AXIS_COLS, T_k, False, stream)
+            K.kq_rotate(Hb, K.KQ_AXIS_ROWS, T_k, False, stream)
+
+    def loss(self, res: BitResult, stream=None):
+        ws = self.workspace(K.kq_kron_loss_blocks_workspace_size(self.d_out, self.d_in, self.k))
+        K.kq_kron_loss_blocks(self.Wp, res.W_hat, self.H_X, self.H_Gb, res.loss, ws, stream)
+
+    def loss_all(self, results, stream=None):
+        for r in results:
+            self.loss(r, stream)
+
+    def unrotate_output(self, M, T_k: K.RHT, out, stream=None):
+        """out = P_G^T (I kron T_k)^T M for M [d_out, cols] (M is overwritten):
+        takes rotated output rows back to the original channel order."""
+        k = self.k
+        for b in range(self.d_out // k):
+            K.kq_rotate(M[b * k:(b + 1) * k], K.KQ_AXIS_ROWS, T_k, True, stream)
+        if self.balanced:
+            inv = torch.empty_like(self.perm)
+            inv.scatter_(0, self.perm, torch.arange(self.d_out, dtype=torch.int64, device=self.device))
+            K.kq_gather(M, out, inv, None, self.info, stream)
+        else:
+            out.copy_(M)
 
 
 def quantize_from_host(lq: LayerQuantizer, host_layers, T_in, T_out, settings, results, host_outputs,
