@@ -63,6 +63,9 @@ def parse():
     ap.add_argument("--configs", default="layer512,mlp_up11008,mlp_down11008,down28672",
                     help="other workloads reported per layer (comma list; empty for none)")
     ap.add_argument("--no-diag", action="store_true", help="skip the untimed per-kernel-class diagnostics")
+    ap.add_argument("--act-order", action="store_true",
+                    help="solve the columns in descending order of the H_X' diagonal (results returned in the "
+                         "original order)")
     a = ap.parse_args()
     a.warmup = max(a.warmup, 3)
     return a
@@ -273,7 +276,7 @@ def run_kronq(a):
 
     T_in, T_out = dev_rht(Ti), dev_rht(To)
     gemm_mode = P.KQ_GEMM_3XTF32 if a.gemm == "3xtf32" else P.KQ_GEMM_FP32
-    lq = LayerQuantizer(spec.d_out, spec.d_in, dev, gemm_mode=gemm_mode)
+    lq = LayerQuantizer(spec.d_out, spec.d_in, dev, gemm_mode=gemm_mode, act_order=a.act_order)
     results = [lq.alloc_result(b, g) for b, g in settings]
     stream = torch.cuda.current_stream()
 
@@ -443,7 +446,7 @@ def run_kronq(a):
         "config": {"workload": f"{a.workload}: W {spec.d_out}x{spec.d_in}, N={spec.n_tokens} tokens, "
                                f"{'+'.join('W%d' % b for b in bits)} {'per-channel' if not a.group else 'g%d' % a.group}",
                    "layers_per_rank_per_step": 1, "bit_widths": bits, "group": a.group,
-                   "trailing_update": a.gemm,
+                   "trailing_update": a.gemm, "column_order": "act-order" if a.act_order else "natural",
                    "l2": "inputs larger than L2 (X, G 2 GiB each); no flush"},
         "roofline": {"kernel": "kq_accum_cov (SYRK)", "bound": "tensor", "achieved": achieved, "peak": peak,
                      "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,

@@ -160,7 +160,7 @@ kq_status kq_accum_cov_blocks(const uint16_t* A, int64_t n, int64_t d, int64_t l
  *   descending energy[j] (ties: lower j); energy fp32 [d], perm int64 [d],
  *   both device; k divides d, d <= 65536.
  * kq_gather: out[i][j] = M[row_idx[i]][col_idx[j]] (either index array may
- *   be NULL: the identity) for rows x cols matrices of 2- or 4-byte elements
+ *   be NULL: the identity) for rows x cols matrices of 1-, 2- or 4-byte elements
  *   (ldm, ldo >= cols; out must not alias M); an index outside 0..rows-1 or
  *   0..cols-1 is skipped and reported as KQ_ERR_INVALID_ARG (index = row i).
  *   Row gather: P_G W (or P_G^T with the inverse permutation); both: P_G H
@@ -172,6 +172,16 @@ kq_status kq_channel_energy(const uint16_t* A, int64_t n, int64_t d, int64_t lda
 kq_status kq_balance_permutation(const float* energy, int64_t d, int64_t k, int64_t* perm, kq_stream_t stream);
 kq_status kq_gather(const void* M, int64_t ldm, int elem_bytes, const int64_t* row_idx, const int64_t* col_idx,
                     int64_t rows, int64_t cols, void* out, int64_t ldo, int32_t* info, kq_stream_t stream);
+
+/* kq_act_order_permutation - the solver's column order by descending
+ * Hessian diagonal ("A Unified Hessian-Guided Framework for Post-Training
+ * Quantization", block-LDL rounding: like GPTQ, blocks with larger traces
+ * are quantized first).  perm[q] = the column of rank q by descending
+ * H[j][j], ties to the lower j; H fp32 [n, n] (ldh >= n), perm int64 [n],
+ * both device.  The act-order solve is kq_gather of W's columns and of H's
+ * rows and columns by perm, kq_chol_inv and kq_quantize_layer on those, and
+ * kq_gather of W_hat and the codes back with the inverse permutation. */
+kq_status kq_act_order_permutation(const float* H, int64_t n, int64_t ldh, int64_t* perm, kq_stream_t stream);
 
 /* --------------------------------------------------------------------------
  * kq_sensitivity - trace sensitivity (step a3).

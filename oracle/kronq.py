@@ -46,7 +46,7 @@ __all__ = [
     "allocate_bits", "budget_units", "quantize_linear",
     "pack_codes", "unpack_codes", "dequantize_layer", "reverted_apply",
     "balance_permutation", "permutation_matrix", "hg_blockwise", "hg_lowrank", "block_rht_matrix",
-    "blockwise_kron_loss", "weight_cv",
+    "blockwise_kron_loss", "weight_cv", "act_order_permutation", "quantize_layer_act_order",
 ]
 
 
@@ -649,3 +649,42 @@ def weight_cv(W, axis):
     W = np.asarray(W, dtype=np.float64)
     norms = np.linalg.norm(W, axis=1 if axis == "out" else 0)
     return float(np.std(norms) / np.mean(norms))
+
+
+# ---------------------------------------------------------------------------
+# Act-order: columns quantized in descending order of the Hessian diagonal
+# ---------------------------------------------------------------------------
+# "A Unified Hessian-Guided Framework for Post-Training Quantization",
+# block-LDL rounding section: like GPTQ, the blocks are sorted before the
+# solve so that those with the larger Fisher traces are quantized first.  For
+# the column-wise solver here a column's trace is its diagonal entry of
+# H_X'.  Reading: ties go to the lower index; the solve runs on the permuted
+# W and H, and its dequantized weights and codes are returned in the original
+# column order; a grouped grid then covers consecutive columns of the
+# quantization order (group g = original columns perm[g*group:(g+1)*group]).
+
+def act_order_permutation(H):
+    """perm[q] = the column of rank q by descending H[j, j] (ties: lower j)."""
+    d = np.asarray(H).diagonal()
+    return np.array(sorted(range(len(d)), key=lambda j: (-float(d[j]), j)), dtype=np.int64)
+
+
+def quantize_layer_act_order(W, H, bits, group=0, block=128, damp_frac=0.01):
+    """Blocked OBS in act-order: permute W's columns and H's rows and columns
+    by act_order_permutation(H), take the damped Cholesky factor of the
+    permuted H, solve, and scatter codes and W_hat back to the original
+    column order.  Returns (QuantResult in the original order with the
+    solver's grid arrays, perm, Uc of the permuted H)."""
+    W = np.asarray(W, dtype=np.float64)
+    H = np.asarray(H, dtype=np.float64)
+    perm = act_order_permutation(H)
+    Hp = H[np.ix_(perm, perm)]
+    Uc, dead, _ = chol_inv(Hp, damp_frac)
+    q = quantize_layer(W[:, perm], Uc, bits, group, block, dead)
+    codes = np.empty_like(q.codes)
+    W_hat = np.empty_like(q.W_hat)
+    V = np.empty_like(q.V)
+    codes[:, perm] = q.codes
+    W_hat[:, perm] = q.W_hat
+    V[:, perm] = q.V
+    return QuantResult(codes, q.scales, q.zeros, W_hat, V), perm, Uc

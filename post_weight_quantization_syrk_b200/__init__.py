@@ -12,7 +12,7 @@ from ._lib import (  # noqa: F401
     kq_quantize_layer_multi, kq_reverted_matvec, kq_reverted_matvec_workspace_size, kq_set_wait_limit_ns, KQ_WAIT_LIMIT_DEFAULT_NS,
     kq_solver_timing, kq_accum_cov_blocks, kq_accum_cov_blocks_workspace_size, kq_channel_energy,
     kq_balance_permutation, kq_gather, kq_sensitivity_blocks, kq_kron_loss_blocks,
-    kq_kron_loss_blocks_workspace_size,
+    kq_kron_loss_blocks_workspace_size, kq_act_order_permutation,
     kq_quantize_layer_multi_workspace_size, kq_quantize_layer_workspace_size, kq_rotate, kq_sensitivity,
     kq_status_string, kq_version, load, new_info, workspace,
 )

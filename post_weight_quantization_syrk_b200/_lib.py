@@ -30,6 +30,7 @@ EXPORTS = (
     "kq_status_string", "kq_last_error", "kq_version", "kq_launch_count", "kq_set_wait_limit_ns",
     "kq_accum_cov_workspace_size", "kq_accum_cov", "kq_accum_cov_blocks_workspace_size", "kq_accum_cov_blocks",
     "kq_channel_energy_workspace_size", "kq_channel_energy", "kq_balance_permutation", "kq_gather",
+    "kq_act_order_permutation",
     "kq_pack_codes", "kq_reverted_matvec_workspace_size", "kq_reverted_matvec",
     "kq_sensitivity", "kq_sensitivity_blocks",
     "kq_rotate",
@@ -80,6 +81,7 @@ _SIGS = {
     "kq_channel_energy": (_i32, [_vp, _i64, _i64, _i64, _f32, _vp, _vp, _sz, _vp, _vp]),
     "kq_balance_permutation": (_i32, [_vp, _i64, _i64, _vp, _vp]),
     "kq_gather": (_i32, [_vp, _i64, _i32, _vp, _vp, _i64, _i64, _vp, _i64, _vp, _vp]),
+    "kq_act_order_permutation": (_i32, [_vp, _i64, _i64, _vp, _vp]),
     "kq_rotate": (_i32, [_vp, _i64, _i64, _i64, _i32, ctypes.POINTER(kq_rht), _i32, _vp]),
     "kq_chol_inv_workspace_size": (_sz, [_i64]),
     "kq_chol_inv": (_i32, [_vp, _i64, _i64, _f32, _vp, _i64, _vp, _vp, _sz, _vp, _vp]),
@@ -256,11 +258,20 @@ def kq_balance_permutation(energy, k, perm, stream=None):
            "kq_balance_permutation")
 
 
+def kq_act_order_permutation(H, perm, stream=None):
+    """perm int64 [n]: columns by descending diagonal of H (ties: lower index)."""
+    ldh = _mat(H, torch.float32, "H")
+    n = H.shape[0]
+    if perm.dtype != torch.int64 or perm.numel() < n or not perm.is_cuda:
+        raise TypeError("perm must be a CUDA int64 tensor of n elements")
+    _check(load().kq_act_order_permutation(_ptr(H), n, ldh, _ptr(perm), _stream(stream)), "kq_act_order_permutation")
+
+
 def kq_gather(M, out, row_idx=None, col_idx=None, info=None, stream=None):
     """out[i, j] = M[row_idx[i], col_idx[j]] (either index may be None) for
-    float32 or bf16 matrices of the same shape."""
-    if M.dtype != out.dtype or M.dtype not in (torch.float32, torch.bfloat16):
-        raise TypeError("M and out must both be float32 or both bf16")
+    float32, bf16 or uint8 matrices of the same shape."""
+    if M.dtype != out.dtype or M.dtype not in (torch.float32, torch.bfloat16, torch.uint8):
+        raise TypeError("M and out must have the same dtype: float32, bf16 or uint8")
     ldm = _mat(M, M.dtype, "M")
     ldo = _mat(out, out.dtype, "out")
     if M.shape != out.shape:

@@ -15,7 +15,9 @@
 //                           fixed order;
 //   kq_balance_permutation: perm[(q % nb) k + q / nb] = the channel of rank q,
 //                           the rank found by counting (deterministic);
-//   kq_gather:              out[i][j] = M[r(i)][c(j)] for 2- or 4-byte elements.
+//   kq_act_order_permutation: perm[q] = the column of rank q by descending
+//                           H[j][j] (ties: lower j), the solver's act-order;
+//   kq_gather:              out[i][j] = M[r(i)][c(j)] for 1-, 2- or 4-byte elements.
 #include <algorithm>
 
 #include "kq_internal.cuh"
@@ -50,16 +52,18 @@ __global__ void __launch_bounds__(256) energy_sum_kernel(const double* __restric
   out[j] = v;
 }
 
-// rank[j] = #{i : e[i] > e[j] or (e[i] == e[j] and i < j)}; one thread per
-// channel, the energies streamed through shared memory in tiles.
-__global__ void __launch_bounds__(256) balance_perm_kernel(const float* __restrict__ e, int64_t d, int64_t k,
-                                                           int64_t* __restrict__ perm) {
+// rank[j] = #{i : e[i] > e[j] or (e[i] == e[j] and i < j)} with e[j] at
+// e[j * stride]; one thread per channel, the values streamed through shared
+// memory in tiles.  Then perm[(rank % nb) k + rank / nb] = j (k == d: the
+// plain descending order).
+__global__ void __launch_bounds__(256) balance_perm_kernel(const float* __restrict__ e, int64_t stride, int64_t d,
+                                                           int64_t k, int64_t* __restrict__ perm) {
   __shared__ float tile[1024];
   const int64_t j = (int64_t)blockIdx.x * 256 + threadIdx.x;
-  const float ej = (j < d) ? e[j] : 0.f;
+  const float ej = (j < d) ? e[j * stride] : 0.f;
   int64_t rank = 0;
   for (int64_t i0 = 0; i0 < d; i0 += 1024) {
-    for (int u = threadIdx.x; u < 1024; u += 256) tile[u] = (i0 + u < d) ? e[i0 + u] : 0.f;
+    for (int u = threadIdx.x; u < 1024; u += 256) tile[u] = (i0 + u < d) ? e[(i0 + u) * stride] : 0.f;
     __syncthreads();
     const int lim = (int)std::min<int64_t>(1024, d - i0);
     for (int u = 0; u < lim; ++u) {
@@ -130,8 +134,20 @@ extern "C" kq_status kq_balance_permutation(const float* energy, int64_t d, int6
   if (d < 1 || d > 65536 || k < 1 || d % k)
     return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_balance_permutation: need 1 <= d <= 65536 and k dividing d");
   cudaStream_t st = (cudaStream_t)stream;
-  balance_perm_kernel<<<(unsigned)kq::cdiv(d, 256), 256, 0, st>>>(energy, d, k, perm);
+  balance_perm_kernel<<<(unsigned)kq::cdiv(d, 256), 256, 0, st>>>(energy, 1, d, k, perm);
   KQ_TRY(kq::launch_check("kq_balance_permutation"));
+  kq::clear_error();
+  return KQ_OK;
+}
+
+extern "C" kq_status kq_act_order_permutation(const float* H, int64_t n, int64_t ldh, int64_t* perm,
+                                              kq_stream_t stream) {
+  if (!H || !perm) return kq::fail(KQ_ERR_INVALID_ARG, "kq_act_order_permutation: NULL pointer");
+  if (n < 1 || n > 65536) return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_act_order_permutation: n outside 1..65536");
+  if (ldh < n) return kq::fail(KQ_ERR_INVALID_ARG, "kq_act_order_permutation: ldh < n");
+  cudaStream_t st = (cudaStream_t)stream;
+  balance_perm_kernel<<<(unsigned)kq::cdiv(n, 256), 256, 0, st>>>(H, ldh + 1, n, n, perm);
+  KQ_TRY(kq::launch_check("kq_act_order_permutation"));
   kq::clear_error();
   return KQ_OK;
 }
@@ -141,7 +157,8 @@ extern "C" kq_status kq_gather(const void* M, int64_t ldm, int elem_bytes, const
                                int32_t* info, kq_stream_t stream) {
   if (!M || !out || !info) return kq::fail(KQ_ERR_INVALID_ARG, "kq_gather: NULL pointer");
   if (rows < 0 || cols < 0 || ldm < cols || ldo < cols) return kq::fail(KQ_ERR_INVALID_ARG, "kq_gather: sizes");
-  if (elem_bytes != 2 && elem_bytes != 4) return kq::fail(KQ_ERR_INVALID_ARG, "kq_gather: elem_bytes must be 2 or 4");
+  if (elem_bytes != 1 && elem_bytes != 2 && elem_bytes != 4)
+    return kq::fail(KQ_ERR_INVALID_ARG, "kq_gather: elem_bytes must be 1, 2 or 4");
   if (rows == 0 || cols == 0) return KQ_OK;
   if (M == out) return kq::fail(KQ_ERR_INVALID_ARG, "kq_gather: out must not alias M");
   cudaStream_t st = (cudaStream_t)stream;
@@ -151,6 +168,9 @@ extern "C" kq_status kq_gather(const void* M, int64_t ldm, int elem_bytes, const
     gather_kernel<uint32_t><<<dim3(gx, gy), 256, 0, st>>>(static_cast<const uint32_t*>(M), ldm, row_idx,
                                                                        col_idx, rows, cols,
                                                                        static_cast<uint32_t*>(out), ldo, info);
+  else if (elem_bytes == 1)
+    gather_kernel<uint8_t><<<dim3(gx, gy), 256, 0, st>>>(static_cast<const uint8_t*>(M), ldm, row_idx, col_idx, rows,
+                                                         cols, static_cast<uint8_t*>(out), ldo, info);
   else
     gather_kernel<uint16_t><<<dim3(gx, gy), 256, 0, st>>>(static_cast<const uint16_t*>(M), ldm, row_idx,
                                                                        col_idx, rows, cols,

@@ -27,13 +27,21 @@ class BitResult:
     zeros: torch.Tensor
     W_hat: torch.Tensor
     loss: torch.Tensor      # fp64[1] device
+    # act-order: the solve's outputs in quantization order, and that order
+    # (codes and W_hat above are in the original column order; a grouped
+    # grid's group g covers original columns perm[g * group:(g + 1) * group])
+    codes_q: torch.Tensor = None
+    W_hat_q: torch.Tensor = None
+    perm: torch.Tensor = None
 
 
 class LayerQuantizer:
     """Device buffers for one (d_out, d_in) layer and the calls that fill them."""
 
-    def __init__(self, d_out, d_in, device="cuda", block=128, gemm_mode=K.KQ_GEMM_FP32, full_hg=True):
+    def __init__(self, d_out, d_in, device="cuda", block=128, gemm_mode=K.KQ_GEMM_FP32, full_hg=True,
+                 act_order=False):
         self.d_out, self.d_in, self.block, self.gemm_mode = d_out, d_in, block, gemm_mode
+        self.act_order = act_order
         dev = torch.device(device)
         self.device = dev
         f32 = dict(dtype=torch.float32, device=dev)
@@ -47,6 +55,13 @@ class LayerQuantizer:
         self.info = K.new_info(dev)
         self._ws = K.workspace(256, dev)
         self._ws_bytes = 256
+        if act_order:
+            # the solve's column order (descending diag H_X'), its inverse, and
+            # W' and H_X' permuted into it
+            self.perm_in = torch.empty(d_in, dtype=torch.int64, device=dev)
+            self.inv_in = torch.empty(d_in, dtype=torch.int64, device=dev)
+            self.Hq = torch.empty((d_in, d_in), **f32)
+            self.Wq = torch.empty((d_out, d_in), **f32)
 
     def workspace(self, nbytes):
         """One scratch buffer shared by the calls (they run in stream order)."""
@@ -58,12 +73,17 @@ class LayerQuantizer:
     def alloc_result(self, bits, group):
         ng = 1 if not group else -(-self.d_in // group)
         dev = self.device
-        return BitResult(bits, group,
-                         torch.empty((self.d_out, self.d_in), dtype=torch.uint8, device=dev),
-                         torch.empty((self.d_out, ng), dtype=torch.float32, device=dev),
-                         torch.empty((self.d_out, ng), dtype=torch.float32, device=dev),
-                         torch.empty((self.d_out, self.d_in), dtype=torch.float32, device=dev),
-                         torch.zeros(1, dtype=torch.float64, device=dev))
+        r = BitResult(bits, group,
+                      torch.empty((self.d_out, self.d_in), dtype=torch.uint8, device=dev),
+                      torch.empty((self.d_out, ng), dtype=torch.float32, device=dev),
+                      torch.empty((self.d_out, ng), dtype=torch.float32, device=dev),
+                      torch.empty((self.d_out, self.d_in), dtype=torch.float32, device=dev),
+                      torch.zeros(1, dtype=torch.float64, device=dev))
+        if self.act_order:
+            r.codes_q = torch.empty_like(r.codes)
+            r.W_hat_q = torch.empty_like(r.W_hat)
+            r.perm = self.perm_in
+        return r
 
     # -- steps -----------------------------------------------------------
     def statistics(self, X, G, n_total=None, accumulate=False, stream=None):
@@ -109,13 +129,37 @@ class LayerQuantizer:
         K.kq_rotate(self.H_G, K.KQ_AXIS_ROWS, T_out, False, stream)
 
     def factor(self, damp_frac=0.01, stream=None):
+        """Damped Cholesky factor of the inverse of H_X' (of the act-order
+        permuted H_X' when act_order; dead flags then in that order)."""
         ws = self.workspace(K.kq_chol_inv_workspace_size(self.d_in))
-        K.kq_chol_inv(self.H_X, damp_frac, self.Uc, self.dead, ws, self.info, stream)
+        H = self.H_X
+        if self.act_order:
+            K.kq_act_order_permutation(self.H_X, self.perm_in, stream)
+            K.kq_gather(self.H_X, self.Hq, self.perm_in, self.perm_in, self.info, stream)
+            # inverse permutation (index bookkeeping): inv[perm[i]] = i
+            self.inv_in.scatter_(0, self.perm_in, torch.arange(self.d_in, dtype=torch.int64, device=self.device))
+            H = self.Hq
+        K.kq_chol_inv(H, damp_frac, self.Uc, self.dead, ws, self.info, stream)
+
+    def _solve_input(self, stream=None):
+        """W' as the solver sees it: in act-order, its columns permuted."""
+        if not self.act_order:
+            return self.Wp
+        K.kq_gather(self.Wp, self.Wq, None, self.perm_in, self.info, stream)
+        return self.Wq
+
+    def _unpermute(self, r: BitResult, stream=None):
+        if self.act_order:
+            K.kq_gather(r.codes_q, r.codes, None, self.inv_in, self.info, stream)
+            K.kq_gather(r.W_hat_q, r.W_hat, None, self.inv_in, self.info, stream)
 
     def quantize(self, res: BitResult, stream=None):
         ws = self.workspace(K.kq_quantize_layer_workspace_size(self.d_out, self.d_in, self.block))
-        K.kq_quantize_layer(self.Wp, self.Uc, self.dead, res.bits, res.group, res.codes, res.scales, res.zeros,
-                            res.W_hat, self.block, self.gemm_mode, ws, self.info, stream)
+        Win = self._solve_input(stream)
+        codes, W_hat = (res.codes_q, res.W_hat_q) if self.act_order else (res.codes, res.W_hat)
+        K.kq_quantize_layer(Win, self.Uc, self.dead, res.bits, res.group, codes, res.scales, res.zeros,
+                            W_hat, self.block, self.gemm_mode, ws, self.info, stream)
+        self._unpermute(res, stream)
 
     def loss(self, res: BitResult, stream=None):
         ws = self.workspace(K.kq_kron_loss_workspace_size(self.d_out, self.d_in))
@@ -125,10 +169,14 @@ class LayerQuantizer:
         """Every setting of `results` in one call: the factor's operand split is
         shared and up to four settings are solved side by side."""
         ws = self.workspace(K.kq_quantize_layer_multi_workspace_size(self.d_out, self.d_in, self.block, len(results)))
-        K.kq_quantize_layer_multi(self.Wp, self.Uc, self.dead, [(r.bits, r.group) for r in results],
-                                  [r.codes for r in results], [r.scales for r in results],
-                                  [r.zeros for r in results], [r.W_hat for r in results], self.block,
-                                  self.gemm_mode, ws, self.info, stream)
+        Win = self._solve_input(stream)
+        q = self.act_order
+        K.kq_quantize_layer_multi(Win, self.Uc, self.dead, [(r.bits, r.group) for r in results],
+                                  [r.codes_q if q else r.codes for r in results], [r.scales for r in results],
+                                  [r.zeros for r in results], [r.W_hat_q if q else r.W_hat for r in results],
+                                  self.block, self.gemm_mode, ws, self.info, stream)
+        for r in results:
+            self._unpermute(r, stream)
 
     def loss_all(self, results, stream=None):
         """Every result's Kronecker loss in one call (the split of the smaller Hessian is shared)."""

@@ -139,6 +139,45 @@ def test_host_validation_without_gpu():
     assert s == 1
 
 
+def test_output_side_entry_points_validate_without_gpu():
+    """The blockwise-H_G, permutation and act-order entry points reject bad
+    arguments before any CUDA call."""
+    lib = _raw()
+    NULL = ctypes.c_void_p(0)
+    fake = ctypes.c_void_p(0x10000)
+    # block size not a multiple of 256 dividing d
+    s = lib.kq_accum_cov_blocks(fake, 10, 1024, 1024, 300, fake, 300, ctypes.c_float(1.0), 0, NULL, 0, fake, NULL)
+    assert s == 2 and b"multiple of 256" in lib.kq_last_error()
+    s = lib.kq_accum_cov_blocks(fake, 10, 768, 768, 512, fake, 512, ctypes.c_float(1.0), 0, NULL, 0, fake, NULL)
+    assert s == 2
+    s = lib.kq_accum_cov_blocks(fake, 10, 1024, 1024, 256, fake, 128, ctypes.c_float(1.0), 0, NULL, 0, fake, NULL)
+    assert s == 1                           # ldc < k
+    assert P.kq_accum_cov_blocks_workspace_size(1 << 18, 1000, 256) == 0
+    assert P.kq_accum_cov_blocks_workspace_size(1 << 18, 4096, 512) > 0
+    s = lib.kq_sensitivity_blocks(fake, 8, 8, fake, 1000, 256, 256, fake, NULL)
+    assert s == 1                           # k does not divide d_out
+    s = lib.kq_kron_loss_blocks(fake, 8, fake, 8, 512, 8, fake, 8, fake, 256, 256, fake, fake, 8, NULL)
+    assert s == 4                           # workspace too small
+    s = lib.kq_kron_loss_blocks(fake, 8, fake, 8, 500, 8, fake, 8, fake, 256, 256, fake, fake, 1 << 30, NULL)
+    assert s == 1                           # k does not divide d_out
+    s = lib.kq_channel_energy(fake, 10, 8, 8, ctypes.c_float(1.0), fake, fake, 8, fake, NULL)
+    assert s == 4
+    s = lib.kq_balance_permutation(fake, 12, 5, fake, NULL)
+    assert s == 2
+    s = lib.kq_balance_permutation(NULL, 12, 4, fake, NULL)
+    assert s == 1
+    s = lib.kq_act_order_permutation(fake, 0, 8, fake, NULL)
+    assert s == 2
+    s = lib.kq_act_order_permutation(fake, 16, 8, fake, NULL)
+    assert s == 1                           # ldh < n
+    s = lib.kq_gather(fake, 8, 3, NULL, NULL, 4, 8, ctypes.c_void_p(0x20000), 8, fake, NULL)
+    assert s == 1 and b"elem_bytes" in lib.kq_last_error()
+    s = lib.kq_gather(fake, 8, 4, NULL, NULL, 4, 8, fake, 8, fake, NULL)
+    assert s == 1                           # out aliases M
+    s = lib.kq_gather(fake, 4, 4, NULL, NULL, 4, 8, ctypes.c_void_p(0x20000), 8, fake, NULL)
+    assert s == 1                           # ldm < cols
+
+
 def test_workspace_sizes():
     assert P.kq_chol_inv_workspace_size(4096) >= 2 * 4096 * 4096 * 8
     assert P.kq_quantize_layer_workspace_size(4096, 4096) >= 4096 * 128 * 4

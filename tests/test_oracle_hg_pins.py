@@ -152,3 +152,63 @@ def test_hg_informed_rotation_orthogonal_function_and_loss():
         assert np.isclose(O.kron_loss(Wp, What, HXp, HGp), O.kron_loss(W, back, HX, HG), rtol=1e-10)
     spread = lambda M: np.std(np.diag(M)) / np.mean(np.diag(M))
     assert spread(Vk @ Pm @ HG @ Pm.T @ Vk.T) < 0.8 * spread(Vk @ HG @ Vk.T)
+
+
+# --------------------------------------------------------------- act-order
+
+def test_act_order_permutation_hand_values():
+    H = np.diag([1.0, 5.0, 3.0, 5.0, 0.5])
+    assert O.act_order_permutation(H).tolist() == [1, 3, 2, 0, 4]
+
+
+def test_act_order_identity_when_already_sorted():
+    """With the diagonal already descending the act-order solve is the
+    natural-order solve."""
+    rng = np.random.default_rng(21)
+    d_out, d_in = 6, 10
+    A = rng.standard_normal((d_in, 3 * d_in))
+    H = A @ A.T / (3 * d_in)
+    order = np.argsort(-np.diag(H), kind="stable")
+    H = H[np.ix_(order, order)]
+    W = rng.normal(0, 0.02, (d_out, d_in))
+    q, perm, _ = O.quantize_layer_act_order(W, H, 3, 0, 4)
+    assert perm.tolist() == list(range(d_in))
+    Uc, dead, _ = O.chol_inv(H)
+    ref = O.quantize_layer(W, Uc, 3, 0, 4, dead)
+    assert np.array_equal(q.codes, ref.codes) and np.array_equal(q.W_hat, ref.W_hat)
+
+
+def test_act_order_invariant_to_the_input_column_order():
+    """Act-order depends on the diagonal, not on where a column sits: solving
+    a layer whose columns were shuffled (W[:, s], H[s][:, s]) gives the same
+    weights, shuffled the same way (distinct diagonal entries)."""
+    rng = np.random.default_rng(22)
+    d_out, d_in = 5, 12
+    A = rng.standard_normal((d_in, 4 * d_in)) * np.exp(rng.normal(0, 1, d_in))[:, None]
+    H = A @ A.T / (4 * d_in)
+    W = rng.normal(0, 0.02, (d_out, d_in))
+    s = rng.permutation(d_in)
+    q1, p1, _ = O.quantize_layer_act_order(W, H, 2, 0, 4)
+    q2, p2, _ = O.quantize_layer_act_order(W[:, s], H[np.ix_(s, s)], 2, 0, 4)
+    assert np.array_equal(s[p2], p1)
+    assert np.allclose(q2.W_hat, q1.W_hat[:, s], rtol=0, atol=1e-15)
+    assert np.array_equal(q2.codes, q1.codes[:, s])
+
+
+def test_act_order_least_squares_in_the_permuted_order():
+    """The OBS property holds in the quantization order: after the solve, the
+    last column's pre-rounding value equals W0 + (W0_p - W_hat_p) H_pr H_rr^-1
+    for p = all earlier columns in act-order (damped H)."""
+    rng = np.random.default_rng(23)
+    d_out, d_in = 3, 7
+    A = rng.standard_normal((d_in, 3 * d_in)) * np.exp(rng.normal(0, 1, d_in))[:, None]
+    H = A @ A.T / (3 * d_in)
+    W = rng.normal(0, 0.02, (d_out, d_in))
+    q, perm, _ = O.quantize_layer_act_order(W, H, 3, 0, 128)
+    Hd, _, _ = O.damp_and_dead(H[np.ix_(perm, perm)])
+    Wp = W[:, perm]
+    What_p = q.W_hat[:, perm]
+    p, r = np.arange(d_in - 1), np.array([d_in - 1])
+    cur = Wp[:, r] + (Wp[:, p] - What_p[:, p]) @ Hd[np.ix_(p, r)] @ np.linalg.inv(Hd[np.ix_(r, r)])
+    scale, zero = q.scales[:, 0].astype(np.float64), q.zeros[:, 0].astype(np.float64)
+    assert np.allclose(cur[:, 0] / scale + zero, q.V[:, perm[-1]], atol=1e-9)
