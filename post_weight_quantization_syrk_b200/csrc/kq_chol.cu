@@ -166,6 +166,7 @@ __global__ void __launch_bounds__(256) potrf_kernel(const double* __restrict__ A
   double* Rb = Cb + 32;          // leaf broadcast: row j of R, two buffers of 16
   const int t = threadIdx.x, warp = t / 32, lane = t % 32;
   const int fr = lane / 4, fc = lane % 4;
+  kq::pdl_wait();   // the block was last updated by the previous kernel of the chain
   {
     // all 16 loads of a thread in flight before any is used
     double v[16];
@@ -287,6 +288,7 @@ __global__ void __launch_bounds__(256) potrf_kernel(const double* __restrict__ A
     }
     __syncthreads();
   }
+  kq::pdl_trigger();   // the panel step may be scheduled now; it waits for this grid's stores
   for (int idx = t; idx < NB * NB; idx += 256) Dinv[idx] = Xs[(idx / NB) * SP + idx % NB];
 }
 
@@ -318,6 +320,7 @@ __global__ void __launch_bounds__(256) step_a_kernel(const double* __restrict__ 
   const bool panel = (int64_t)blockIdx.x < tp;
   const int64_t r0 = k0 + NB + (int64_t)blockIdx.x * 128;
   const int64_t c0 = ((int64_t)blockIdx.x - tp) * 128;
+  kq::pdl_wait();   // Dinv comes from the diagonal factorisation just before
 #pragma unroll
   for (int u = 0; u < 8; ++u) {   // Dinv: 64 rows x 32 chunks
     const int id = u * 256 + t, row = id / 32, cc = id % 32;
@@ -460,6 +463,7 @@ __global__ void __launch_bounds__(256, 2) step_b_kernel(double* __restrict__ A, 
     opB = X + k0 * ld + cb * TBN;
   }
   const int t = threadIdx.x;
+  kq::pdl_wait();
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
 #pragma unroll
@@ -662,12 +666,15 @@ extern "C" kq_status kq_chol_inv(const float* H, int64_t n, int64_t ldh, float d
     const int kb = (int)std::min<int64_t>(NB, n - k0);
     double* Dk = w.Dinv + b * NB * NB;
     double* Pt = w.Pt + (b & 1) * NB * ld;
-    potrf_kernel<<<1, 256, kPotrfSmem, s1>>>(w.A, ld, n, k0, kb, Dk, info);
-    KQ_TRY(kq::launch_check("kq_chol_inv potrf"));
+    // the chain potrf -> step a -> (kNext) -> potrf runs as programmatic
+    // dependents on s1: each kernel is scheduled while its predecessor
+    // finishes and waits for it (griddepcontrol.wait) before reading
+    KQ_TRY(kq::launch_ex("kq_chol_inv potrf", b > 0, potrf_kernel, dim3(1), dim3(256), kPotrfSmem, s1, w.A, ld, n,
+                         k0, kb, Dk, info));
     const int64_t tp = kq::cdiv(n - k0 - kb, 128);   // > 0 only when kb == 64
     const int64_t xt = kq::cdiv(k0 + kb, 128);
-    step_a_kernel<<<(unsigned)(tp + xt), 256, kStepASmem, s1>>>(w.A, w.X, Pt, ld, k0, tp, Dk);
-    KQ_TRY(kq::launch_check("kq_chol_inv step a"));
+    KQ_TRY(kq::launch_ex("kq_chol_inv step a", true, step_a_kernel, dim3((unsigned)(tp + xt)), dim3(256), kStepASmem,
+                         s1, w.A, w.X, Pt, ld, k0, tp, Dk));
     if (tp > 0) {
       const int64_t tr = kq::cdiv(n - k0 - NB, TBM), xcols = (k0 + NB) / TBN;
       KQ_TRY(kq::cuda_check(cudaEventRecord(ev_a, s1), "kq_chol_inv: record"));

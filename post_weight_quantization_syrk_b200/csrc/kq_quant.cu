@@ -104,20 +104,27 @@ struct InblockArgs {
   int32_t* info;
 };
 
-// Eight lanes share a row: lane L of a row group owns the 16 columns
-// 32 m + 4 L + t (m, t in 0..3), kept in registers.  Column j is quantized by
-// its owner, whose error e_j reaches the row's other lanes by one warp
-// shuffle; every lane then updates its own columns right of j.  This
-// interleaved ownership makes each lane's four float4 reads of Uc row j hit
-// distinct shared-memory banks.
-constexpr int LPR = 8;                  // lanes per row
+// LPR lanes share a row (LPR = 8 or 4): lane L of a row group owns the
+// 128 / LPR columns 4 LPR m + 4 L + t (t in 0..3, m in 0..32/LPR - 1), kept
+// in registers.  Column j is quantized by its owner, whose error e_j reaches
+// the row's other lanes by one warp shuffle; every lane then updates its own
+// columns right of j.  This interleaved ownership makes each lane's float4
+// reads of Uc row j hit distinct shared-memory banks (the row groups of a
+// warp read the same row: broadcast).  Fewer lanes per row mean fewer warps
+// repeating the per-column quantisation and shuffle (the latency-bound part)
+// for the same multiply-adds.
 constexpr int IB_THREADS = 256;
-constexpr int IB_ROWS = IB_THREADS / LPR;  // 32 rows per CTA
 constexpr int IB_SMEM = BLK * BLK * 4 + BLK * 4;
 
-__device__ __forceinline__ int col_of(int L, int r) { return 32 * (r >> 2) + 4 * L + (r & 3); }
+template <int LPR>
+__device__ __forceinline__ int col_of(int L, int r) { return 4 * LPR * (r >> 2) + 4 * L + (r & 3); }
 
+template <int LPR>
 __global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
+  constexpr int IB_ROWS = IB_THREADS / LPR;   // rows per CTA
+  constexpr int NR = BLK / LPR;               // columns (registers) per lane
+  constexpr int MB = NR / 4;                  // register blocks of 4 columns
+  constexpr int SPAN = 4 * LPR;               // columns per register block over the row group
   extern __shared__ float sm[];
   float* Us = sm;                 // [128][128]: Uc[i0 + j][i0 + k]
   float* inv_d = sm + BLK * BLK;  // 1 / Uc[i0 + j][i0 + j]
@@ -147,11 +154,11 @@ __global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
   asm volatile("cp.async.commit_group;" ::: "memory");
   kq::pdl_wait();
 
-  // this lane's 16 columns of the row
-  float w[16];
+  // this lane's columns of the row
+  float w[NR];
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    const int c = 32 * m + 4 * L;
+  for (int m = 0; m < MB; ++m) {
+    const int c = SPAN * m + 4 * L;
     float v[4] = {0.f, 0.f, 0.f, 0.f};
     if (row_ok) {
       if (c + 3 < bw && !a.dead) {
@@ -184,26 +191,26 @@ __global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
     zero = a.zeros[row * a.n_groups];
   }
   float inv_scale = 1.f / scale;
-  float qv[16], ev[16];
+  float qv[NR], ev[NR];
   const int gbase = lane & ~(LPR - 1);
 
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {
+  for (int m = 0; m < MB; ++m) {
 #pragma unroll 1
     for (int Lo = 0; Lo < LPR; ++Lo) {
 #pragma unroll
       for (int tt = 0; tt < 4; ++tt) {
-        const int j = 32 * m + 4 * Lo + tt;   // column quantized in this step
+        const int j = SPAN * m + 4 * Lo + tt;   // column quantized in this step
         if (j >= bw) break;
         if (a.group && tt == 0 && ((i0 + j) % a.group) == 0) {
           // group grid on the current values of columns [j, j + group): every
-          // lane folds its own columns in range, then the row's 8 lanes meet
+          // lane folds its own columns in range, then the row's lanes meet
           const int64_t lim = a.d_in - i0;
           const int gend = (int)((int64_t)(j + a.group) < lim ? (int64_t)(j + a.group) : lim);
           float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
-          for (int r = 0; r < 16; ++r) {
-            const int c = col_of(L, r);
+          for (int r = 0; r < NR; ++r) {
+            const int c = col_of<LPR>(L, r);
             if (c >= j && c < gend) {
               mn = fminf(mn, w[r]);
               mx = fmaxf(mx, w[r]);
@@ -234,11 +241,11 @@ __global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
         // columns left of j see Uc[j][c] = 0 (cleared above), so the update
         // runs over all of this lane's columns; column j itself is then set
         // to its final dequantized value by its owner
-        // register blocks m2 < m hold columns left of 32 m <= j: final, skipped
+        // register blocks m2 < m hold columns left of SPAN m <= j: final, skipped
         const float4* urow = reinterpret_cast<const float4*>(Us + j * BLK);
 #pragma unroll
-        for (int m2 = m; m2 < 4; ++m2) {
-          const float4 u = urow[8 * m2 + L];
+        for (int m2 = m; m2 < MB; ++m2) {
+          const float4 u = urow[LPR * m2 + L];
           const float uu[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
           for (int t2 = 0; t2 < 4; ++t2) w[4 * m2 + t2] = fmaf(-e, uu[t2], w[4 * m2 + t2]);
@@ -253,10 +260,10 @@ __global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
   }
 
   if (!row_ok) return;
-  // this lane's 16 columns: W_hat, codes, and the errors for the trailing update
+  // this lane's columns: W_hat, codes, and the errors for the trailing update
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    const int c = 32 * m + 4 * L;
+  for (int m = 0; m < MB; ++m) {
+    const int c = SPAN * m + 4 * L;
     if (c + 3 < bw) {
       *reinterpret_cast<float4*>(a.W_hat + row * a.ldwh + i0 + c) = make_float4(w[4 * m], w[4 * m + 1], w[4 * m + 2],
                                                                                w[4 * m + 3]);
@@ -288,6 +295,9 @@ __global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
     }
   }
 }
+
+// Lanes per row of the in-block recursion.
+constexpr int kLanesPerRow = 8;
 
 // Lazy trailing update, fp32 SIMT: dst[:, c0..] = src[:, c0..] - E Uc[i0:i0+bw, c0..].
 // 128x128 output tile per CTA, 256 threads, 8x8 each, K in chunks of 32.
@@ -498,8 +508,8 @@ kq_status enqueue_setting(const float* W, int64_t d_out, int64_t d_in, int64_t l
       return kq::launch_check("kq_quantize_layer grid");
     }));
   }
-  KQ_TRY(kq::cuda_check(cudaFuncSetAttribute(inblock_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, IB_SMEM),
-                        "kq_quantize_layer: smem attribute"));
+  KQ_TRY(kq::cuda_check(cudaFuncSetAttribute(inblock_kernel<kLanesPerRow>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             IB_SMEM), "kq_quantize_layer: smem attribute"));
   auto inblock = [&](int64_t i0, int64_t o0) -> kq_status {
     const int bw = (int)std::min<int64_t>(BLK, d_in - i0);
     const bool first = (i0 == 0);
@@ -531,8 +541,9 @@ kq_status enqueue_setting(const float* W, int64_t d_out, int64_t d_in, int64_t l
     // after the first block the previous kernel is this solve's own trailing
     // update, so the launch may overlap its tail (tensor-core mode)
     return timed(kClassInblock, 0.0, (double)d_out * bw * (tc ? 17.0 : 13.0), st, [&]() {
-      return kq::launch_ex("kq_quantize_layer inblock", tc && i0 > 0, inblock_kernel,
-                           dim3((unsigned)kq::cdiv(d_out, IB_ROWS)), dim3(IB_THREADS), IB_SMEM, st, a);
+      return kq::launch_ex("kq_quantize_layer inblock", tc && i0 > 0, inblock_kernel<kLanesPerRow>,
+                           dim3((unsigned)kq::cdiv(d_out, IB_THREADS / kLanesPerRow)), dim3(IB_THREADS), IB_SMEM, st,
+                           a);
     });
   };
   // W_hat[:, c0:c0+N] = src[:, c0:c0+N] - E[:, e0:e0+K] Uc[k0:k0+K, c0:c0+N]; the
