@@ -253,6 +253,10 @@ kq_status kq_rotate(float* M, int64_t rows, int64_t cols, int64_t ld, int axis,
  *   info      KQ_ERR_NOT_PD (index = column whose pivot failed),
  *             KQ_ERR_NONFINITE (index = row holding NaN/Inf).
  * Limits: 1 <= n <= 65536, 0 <= damp_frac.
+ * The serial diagonal chain runs on an internal high-priority stream of the
+ * library, one per (host thread, device, caller stream), forked from and
+ * joined back into `stream`; calls on different caller streams (each with
+ * its own workspace) run concurrently.
  * ------------------------------------------------------------------------ */
 size_t kq_chol_inv_workspace_size(int64_t n);
 kq_status kq_chol_inv(const float* H, int64_t n, int64_t ldh, float damp_frac,

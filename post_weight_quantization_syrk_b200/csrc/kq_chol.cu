@@ -551,28 +551,32 @@ struct CholWs {
   int64_t ld;
 };
 
-// The look-ahead needs a second stream and a few events per device; they are
-// created on first use by each host thread and kept for its lifetime.
+// The look-ahead needs a second stream and a few events per (device, caller
+// stream), so that factorisations enqueued on different caller streams keep
+// their chains apart and run concurrently; created on first use by each host
+// thread and kept for its lifetime.
 struct LookAhead {
   int device = -1;
+  cudaStream_t caller = nullptr;
   cudaStream_t s1 = nullptr;
   cudaEvent_t ev[4] = {};
 };
 
-kq_status look_ahead(LookAhead** out) {
-  thread_local LookAhead cache[16];
+kq_status look_ahead(cudaStream_t caller, LookAhead** out) {
+  thread_local LookAhead cache[32];
   int dev = 0;
   KQ_TRY(kq::cuda_check(cudaGetDevice(&dev), "kq_chol_inv: cudaGetDevice"));
   LookAhead* la = nullptr;
   for (auto& c : cache)
-    if (c.device == dev) la = &c;
+    if (c.device == dev && c.caller == caller) la = &c;
   if (!la) {
     for (auto& c : cache)
       if (c.device < 0) {
         la = &c;
         break;
       }
-    if (!la) return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_chol_inv: more than 16 devices");
+    if (!la) return kq::fail(KQ_ERR_UNSUPPORTED_SHAPE, "kq_chol_inv: more than 32 (device, stream) pairs");
+    la->caller = caller;
     int least = 0, greatest = 0;
     KQ_TRY(kq::cuda_check(cudaDeviceGetStreamPriorityRange(&least, &greatest), "kq_chol_inv: priority range"));
     KQ_TRY(kq::cuda_check(cudaStreamCreateWithPriority(&la->s1, cudaStreamNonBlocking, greatest),
@@ -654,7 +658,7 @@ extern "C" kq_status kq_chol_inv(const float* H, int64_t n, int64_t ldh, float d
   // step k+1 waits for kRest of step k (both update column block k+2), and
   // the transposed panel alternates between two buffers.
   LookAhead* la = nullptr;
-  KQ_TRY(look_ahead(&la));
+  KQ_TRY(look_ahead(st, &la));
   cudaStream_t s1 = la->s1;
   cudaEvent_t ev_fork = la->ev[0], ev_a = la->ev[1], ev_rest[2] = {la->ev[2], la->ev[3]};
   KQ_TRY(kq::cuda_check(cudaEventRecord(ev_fork, st), "kq_chol_inv: record"));

@@ -13,10 +13,12 @@ Order (KronQ paper page, Abstract; KronQ review, Method and Comparison):
     rotation of W and H_G, the blocked OBS solve at its allocated bit-width
     and its Kronecker loss.
 In pass 2 the linears of an input group start as soon as its factor is
-ready: the rotations of H_X and the Cholesky factorisations run on the
-caller's stream, each linear's rotations, solve and loss on a second
-stream, so the linears of one group overlap the factorisation of the next
-(the factorisations are a latency-bound chain).  GPU time is the elapsed
+ready: the rotation of H_X and the Cholesky factorisation of the widest
+input group (the down projection's, the longest) run on the caller's
+stream, those of the three 4096-wide groups one after another on a second
+factor stream beside it, and each linear's rotations, solve and loss on a
+third stream, so the factorisations overlap one another and the linears of
+the groups already factored (the factorisations are latency-bound chains).  GPU time is the elapsed
 time of pass 1 and of each block of pass 2, taken with CUDA events;
 generating the synthetic inputs is reported separately and is not part of
 it.  Phase seconds are each phase's own event time, summed over its calls
@@ -81,6 +83,8 @@ class ModelQuantizer:
         self.overlap = overlap
         self.ws = K.workspace(256, self.dev)        # calls on the caller's stream
         self.ws_lin = None                          # calls of the linears (their stream)
+        self.ws_fac = None                          # factorisations on the second factor stream
+        self.fac_stream = None
         self.phases = {k: Phase() for k in ("statistics", "sensitivity", "rotate", "chol_inv", "quantize", "loss")}
         self.gen_s = 0.0
         self.rank, self.world = rank, world
@@ -90,6 +94,12 @@ class ModelQuantizer:
         if nbytes > self.ws.numel():
             self.ws = K.workspace(nbytes, self.dev)
         return self.ws
+
+    def _ws_fac(self, nbytes):
+        # the second factor stream's workspace (its factorisations overlap the first's)
+        if self.ws_fac is None or nbytes > self.ws_fac.numel():
+            self.ws_fac = K.workspace(nbytes, self.dev)
+        return self.ws_fac
 
     def _ws_lin(self, nbytes):
         # allocated while the linears' stream is current, so that the caching
@@ -182,19 +192,32 @@ class ModelQuantizer:
             span = self._span_start()
             U = {g: self.make_rht(b, "in:" + g, INPUT_WIDTH[g]) for g in INPUT_WIDTH}
             Uc, dead, ready = {}, {}, {}
-            # caller's stream: per input group the rotation of H_X and its factor
-            for g in INPUT_WIDTH:
+            # per input group the rotation of H_X and its factor; the groups
+            # are independent, so the widest (the down projection's input,
+            # the longest factorisation) runs on the caller's stream while the
+            # others run one after another on a second factor stream
+            if self.overlap and self.fac_stream is None:
+                self.fac_stream = torch.cuda.Stream(device=dev)
+            fac = self.fac_stream if self.overlap else main
+            fork = torch.cuda.Event()
+            fork.record(main)
+            fac.wait_event(fork)
+            order = sorted(INPUT_WIDTH, key=lambda g: -INPUT_WIDTH[g])
+            for i, g in enumerate(order):
+                st = main if i == 0 else fac
                 H = HX.pop((b, g))
-                self._timed("rotate", lambda: (K.kq_rotate(H, K.KQ_AXIS_COLS, U[g]),
-                                               K.kq_rotate(H, K.KQ_AXIS_ROWS, U[g])))
-                n = H.shape[0]
-                Uc[g] = torch.empty_like(H)
-                dead[g] = torch.zeros(n, dtype=torch.uint8, device=dev)
-                ws = self._ws(K.kq_chol_inv_workspace_size(n))
-                self._timed("chol_inv", lambda: K.kq_chol_inv(H, self.damp, Uc[g], dead[g], ws, self.info))
+                with torch.cuda.stream(st):
+                    self._timed("rotate", lambda: (K.kq_rotate(H, K.KQ_AXIS_COLS, U[g]),
+                                                   K.kq_rotate(H, K.KQ_AXIS_ROWS, U[g])))
+                    n = H.shape[0]
+                    Uc[g] = torch.empty_like(H)
+                    dead[g] = torch.zeros(n, dtype=torch.uint8, device=dev)
+                    ws = self._ws(K.kq_chol_inv_workspace_size(n)) if i == 0 else \
+                        self._ws_fac(K.kq_chol_inv_workspace_size(n))
+                    self._timed("chol_inv", lambda: K.kq_chol_inv(H, self.damp, Uc[g], dead[g], ws, self.info))
                 HX[(b, g)] = H
                 ready[g] = torch.cuda.Event()
-                ready[g].record(main)
+                ready[g].record(st)
             # linears' stream: each linear once its group's factor is ready.
             # Everything allocated here belongs to this stream; what the
             # caller's stream allocated is freed only after the join below.
@@ -228,6 +251,10 @@ class ModelQuantizer:
                 done = torch.cuda.Event()
                 done.record(lin_stream)
                 main.wait_event(done)
+            if fac is not main:
+                fdone = torch.cuda.Event()
+                fdone.record(fac)
+                main.wait_event(fdone)
             self._span_end(span)
             for g in INPUT_WIDTH:
                 del HX[(b, g)]
