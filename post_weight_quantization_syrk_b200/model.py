@@ -12,14 +12,15 @@ Order (KronQ paper page, Abstract; KronQ review, Method and Comparison):
     share U and H_X, hence one damped Cholesky factor), then per linear the
     rotation of W and H_G, the blocked OBS solve at its allocated bit-width
     and its Kronecker loss.
-In pass 2 the linears of an input group start as soon as its factor is
-ready: the rotation of H_X and the Cholesky factorisation of the widest
-input group (the down projection's, the longest) run on the caller's
-stream, those of the three 4096-wide groups one after another on a second
-factor stream beside it, and each linear's rotations, solve and loss on a
-third stream, so the factorisations overlap one another and the linears of
-the groups already factored (the factorisations are latency-bound chains).  GPU time is the elapsed
-time of pass 1 and of each block of pass 2, taken with CUDA events;
+In pass 2 the weights of all blocks are generated first; then the rotation
+of H_X and the Cholesky factorisation of every input group run block after
+block on two factor streams (the widest group, the down projection's input
+and the longest factorisation, on the caller's stream, the three 4096-wide
+groups on a second stream beside it), and every linear's rotations, solve
+and loss run on a third stream as soon as its group's factor is ready, so
+the factorisations overlap one another and the linears of earlier blocks
+(the factorisations are latency-bound chains).  GPU time is the elapsed
+time of pass 1's blocks and of pass 2 as a whole, taken with CUDA events;
 generating the synthetic inputs is reported separately and is not part of
 it.  Phase seconds are each phase's own event time, summed over its calls
 (with the overlap they add up to more than the GPU time).  On several ranks
@@ -141,6 +142,36 @@ class ModelQuantizer:
         e1.record()
         self._spans.append((e0, e1))
 
+    def _linears(self, b, weights, U, Uc, dead, ready, HX, HG, alloc, results, lin_stream, dev):
+        """Rotations of W and H_G, solve and loss of block b's linears on the
+        linears' stream, each after its input group's factor."""
+        with torch.cuda.stream(lin_stream):
+            for lin in LINEARS:
+                g = INPUT_OF[lin]
+                lin_stream.wait_event(ready[(b, g)])
+                d_out, d_in = SHAPE[lin]
+                V = self.make_rht(b, "out:" + lin, d_out)
+                W = weights[b][lin]
+                Hg = HG.pop((b, lin))
+                self._timed("rotate", lambda: (K.kq_rotate(W, K.KQ_AXIS_COLS, U[b][g]),
+                                               K.kq_rotate(W, K.KQ_AXIS_ROWS, V),
+                                               K.kq_rotate(Hg, K.KQ_AXIS_COLS, V),
+                                               K.kq_rotate(Hg, K.KQ_AXIS_ROWS, V)))
+                nb = alloc[(b, lin)]
+                codes = torch.empty((d_out, d_in), dtype=torch.uint8, device=dev)
+                scales = torch.empty((d_out, 1), dtype=torch.float32, device=dev)
+                zeros = torch.empty((d_out, 1), dtype=torch.float32, device=dev)
+                W_hat = torch.empty((d_out, d_in), dtype=torch.float32, device=dev)
+                loss = torch.zeros(1, dtype=torch.float64, device=dev)
+                ws = self._ws_lin(max(K.kq_quantize_layer_workspace_size(d_out, d_in),
+                                      K.kq_kron_loss_workspace_size(d_out, d_in)))
+                self._timed("quantize", lambda: K.kq_quantize_layer(W, Uc[(b, g)], dead[(b, g)], nb, 0, codes,
+                                                                     scales, zeros, W_hat, gemm_mode=self.gemm_mode,
+                                                                     ws=ws, info=self.info))
+                self._timed("loss", lambda: K.kq_kron_loss(W, W_hat, HX[(b, g)], Hg, loss, ws))
+                results[(b, lin)] = {"bits": nb, "loss": loss, "codes_bytes": codes.numel()}
+                del Hg, codes, W_hat
+
     def run(self):
         self._events, self._spans = [], []
         dev = self.dev
@@ -181,84 +212,59 @@ class ModelQuantizer:
         mine = [(b, lin) for b in self.blocks for lin in LINEARS]
 
         # ---------------- pass 2: BiIP, Cholesky, solver, loss (this rank's blocks)
+        # The weights of every block are generated first (untimed).  Then, in
+        # one timed span: the factor streams rotate every input group's H_X
+        # and factor it, block after block (the widest group on the caller's
+        # stream, the three 4096-wide ones on a second factor stream), while
+        # the linears' stream quantizes each block's linears as soon as their
+        # group's factor is ready; so the factorisations of later blocks
+        # overlap the linears of earlier ones.
         main = torch.cuda.current_stream(dev)
         lin_stream = torch.cuda.Stream(device=dev) if self.overlap else main
-        results = {}
+        if self.overlap and self.fac_stream is None:
+            self.fac_stream = torch.cuda.Stream(device=dev)
+        fac = self.fac_stream if self.overlap else main
+        weights = {}
         for b in self.blocks:
             t0 = time.perf_counter()
-            inp = self.make_inputs(b, stats_only=False)
+            weights[b] = self.make_inputs(b, stats_only=False)["W"]
             torch.cuda.synchronize()
             self.gen_s += time.perf_counter() - t0
-            span = self._span_start()
-            U = {g: self.make_rht(b, "in:" + g, INPUT_WIDTH[g]) for g in INPUT_WIDTH}
-            Uc, dead, ready = {}, {}, {}
-            # per input group the rotation of H_X and its factor; the groups
-            # are independent, so the widest (the down projection's input,
-            # the longest factorisation) runs on the caller's stream while the
-            # others run one after another on a second factor stream
-            if self.overlap and self.fac_stream is None:
-                self.fac_stream = torch.cuda.Stream(device=dev)
-            fac = self.fac_stream if self.overlap else main
-            fork = torch.cuda.Event()
-            fork.record(main)
-            fac.wait_event(fork)
-            order = sorted(INPUT_WIDTH, key=lambda g: -INPUT_WIDTH[g])
+        results = {}
+        U = {b: {g: self.make_rht(b, "in:" + g, INPUT_WIDTH[g]) for g in INPUT_WIDTH} for b in self.blocks}
+        Uc, dead, ready = {}, {}, {}
+        span = self._span_start()
+        fork = torch.cuda.Event()
+        fork.record(main)
+        fac.wait_event(fork)
+        order = sorted(INPUT_WIDTH, key=lambda g: -INPUT_WIDTH[g])
+        for b in self.blocks:
             for i, g in enumerate(order):
                 st = main if i == 0 else fac
-                H = HX.pop((b, g))
+                H = HX[(b, g)]
                 with torch.cuda.stream(st):
-                    self._timed("rotate", lambda: (K.kq_rotate(H, K.KQ_AXIS_COLS, U[g]),
-                                                   K.kq_rotate(H, K.KQ_AXIS_ROWS, U[g])))
+                    self._timed("rotate", lambda: (K.kq_rotate(H, K.KQ_AXIS_COLS, U[b][g]),
+                                                   K.kq_rotate(H, K.KQ_AXIS_ROWS, U[b][g])))
                     n = H.shape[0]
-                    Uc[g] = torch.empty_like(H)
-                    dead[g] = torch.zeros(n, dtype=torch.uint8, device=dev)
+                    Uc[(b, g)] = torch.empty_like(H)
+                    dead[(b, g)] = torch.zeros(n, dtype=torch.uint8, device=dev)
                     ws = self._ws(K.kq_chol_inv_workspace_size(n)) if i == 0 else \
                         self._ws_fac(K.kq_chol_inv_workspace_size(n))
-                    self._timed("chol_inv", lambda: K.kq_chol_inv(H, self.damp, Uc[g], dead[g], ws, self.info))
-                HX[(b, g)] = H
-                ready[g] = torch.cuda.Event()
-                ready[g].record(st)
-            # linears' stream: each linear once its group's factor is ready.
-            # Everything allocated here belongs to this stream; what the
-            # caller's stream allocated is freed only after the join below.
-            with torch.cuda.stream(lin_stream):
-                for lin in LINEARS:
-                    g = INPUT_OF[lin]
-                    lin_stream.wait_event(ready[g])
-                    d_out, d_in = SHAPE[lin]
-                    V = self.make_rht(b, "out:" + lin, d_out)
-                    W = inp["W"][lin]
-                    Hg = HG.pop((b, lin))
-                    self._timed("rotate", lambda: (K.kq_rotate(W, K.KQ_AXIS_COLS, U[g]),
-                                                   K.kq_rotate(W, K.KQ_AXIS_ROWS, V),
-                                                   K.kq_rotate(Hg, K.KQ_AXIS_COLS, V),
-                                                   K.kq_rotate(Hg, K.KQ_AXIS_ROWS, V)))
-                    nb = alloc[(b, lin)]
-                    codes = torch.empty((d_out, d_in), dtype=torch.uint8, device=dev)
-                    scales = torch.empty((d_out, 1), dtype=torch.float32, device=dev)
-                    zeros = torch.empty((d_out, 1), dtype=torch.float32, device=dev)
-                    W_hat = torch.empty((d_out, d_in), dtype=torch.float32, device=dev)
-                    loss = torch.zeros(1, dtype=torch.float64, device=dev)
-                    ws = self._ws_lin(max(K.kq_quantize_layer_workspace_size(d_out, d_in),
-                                          K.kq_kron_loss_workspace_size(d_out, d_in)))
-                    self._timed("quantize", lambda: K.kq_quantize_layer(W, Uc[g], dead[g], nb, 0, codes, scales,
-                                                                         zeros, W_hat, gemm_mode=self.gemm_mode,
-                                                                         ws=ws, info=self.info))
-                    self._timed("loss", lambda: K.kq_kron_loss(W, W_hat, HX[(b, g)], Hg, loss, ws))
-                    results[(b, lin)] = {"bits": nb, "loss": loss, "codes_bytes": codes.numel()}
-                    del Hg, codes, W_hat
-            if lin_stream is not main:
+                    self._timed("chol_inv", lambda: K.kq_chol_inv(H, self.damp, Uc[(b, g)], dead[(b, g)], ws,
+                                                                  self.info))
+                ready[(b, g)] = torch.cuda.Event()
+                ready[(b, g)].record(st)
+            if not self.overlap:
+                self._linears(b, weights, U, Uc, dead, ready, HX, HG, alloc, results, lin_stream, dev)
+        if self.overlap:
+            for b in self.blocks:
+                self._linears(b, weights, U, Uc, dead, ready, HX, HG, alloc, results, lin_stream, dev)
+        for st in (lin_stream, fac):
+            if st is not main:
                 done = torch.cuda.Event()
-                done.record(lin_stream)
+                done.record(st)
                 main.wait_event(done)
-            if fac is not main:
-                fdone = torch.cuda.Event()
-                fdone.record(fac)
-                main.wait_event(fdone)
-            self._span_end(span)
-            for g in INPUT_WIDTH:
-                del HX[(b, g)]
-            del inp, U, Uc, dead
+        self._span_end(span)
         torch.cuda.synchronize()
         K.check_info(self.info, "model quantization")
         for name, e0, e1 in self._events:
