@@ -156,9 +156,10 @@ __device__ __forceinline__ void store16(const double (&acc)[2][2][2], double* c,
     }
 }
 
-__global__ void __launch_bounds__(256) potrf_kernel(const double* __restrict__ A, int64_t ld, int64_t n, int64_t k0,
-                                                    int kb, double* __restrict__ Dinv, int32_t* info) {
-  extern __shared__ __align__(16) double psm[];
+// The factorisation of one diagonal block by all 256 threads of a CTA, with
+// psm at least kPotrfSmem bytes of shared memory (16-byte aligned).
+__device__ __forceinline__ void potrf_block(const double* __restrict__ A, int64_t ld, int64_t n, int64_t k0, int kb,
+                                            double* __restrict__ Dinv, int32_t* info, double* psm) {
   double* As = psm;              // [64][SP]
   double* Xs = psm + NB * SP;    // [64][SP]
   double* Ls = Xs + NB * SP;     // [16][SL]
@@ -166,7 +167,6 @@ __global__ void __launch_bounds__(256) potrf_kernel(const double* __restrict__ A
   double* Rb = Cb + 32;          // leaf broadcast: row j of R, two buffers of 16
   const int t = threadIdx.x, warp = t / 32, lane = t % 32;
   const int fr = lane / 4, fc = lane % 4;
-  kq::pdl_wait();   // the block was last updated by the previous kernel of the chain
   {
     // all 16 loads of a thread in flight before any is used
     double v[16];
@@ -290,6 +290,13 @@ __global__ void __launch_bounds__(256) potrf_kernel(const double* __restrict__ A
   }
   kq::pdl_trigger();   // the panel step may be scheduled now; it waits for this grid's stores
   for (int idx = t; idx < NB * NB; idx += 256) Dinv[idx] = Xs[(idx / NB) * SP + idx % NB];
+}
+
+__global__ void __launch_bounds__(256) potrf_kernel(const double* __restrict__ A, int64_t ld, int64_t n, int64_t k0,
+                                                    int kb, double* __restrict__ Dinv, int32_t* info) {
+  extern __shared__ __align__(16) double psm[];
+  kq::pdl_wait();   // the block was last updated by the previous kernel of the chain
+  potrf_block(A, ld, n, k0, kb, Dinv, info, psm);
 }
 
 
@@ -419,9 +426,15 @@ constexpr int SA = TBM + 4, SB = TBN + 4;   // padded k-row strides (doubles)
 constexpr size_t kStepBSmem = (size_t)NB * (SA + SB) * sizeof(double);   // 102 KB
 
 
+// With Dnext != NULL (kNext launches), CTA 0 (row tile 0 of column block
+// k+1, which holds the next diagonal block) goes on, once its tile is
+// stored, to factor that diagonal block and write its inverse factor to
+// Dnext: the next block step's diagonal factorisation without a launch of
+// its own.
 __global__ void __launch_bounds__(256, 2) step_b_kernel(double* __restrict__ A, double* __restrict__ X,
                                                        const double* __restrict__ Pt, int64_t ld, int64_t k0,
-                                                       int64_t tr, int part) {
+                                                       int64_t tr, int part, int64_t n, double* __restrict__ Dnext,
+                                                       int32_t* info) {
   extern __shared__ __align__(16) double sm[];
   double* As = sm;               // [64][SA]
   double* Bs = sm + NB * SA;     // [64][SB]
@@ -520,6 +533,10 @@ __global__ void __launch_bounds__(256, 2) step_b_kernel(double* __restrict__ A, 
     for (int ct = 0; ct < 4; ++ct)
       *reinterpret_cast<double2*>(C + (32 * wm + 8 * rt + fr) * ld + 32 * wn + 8 * ct + 2 * fc) =
           make_double2(acc[rt][ct][0], acc[rt][ct][1]);
+  if (Dnext && bid == 0) {
+    __syncthreads();   // the tile's stores are visible to the whole CTA; the operand smem is free
+    potrf_block(A, ld, n, base, (int)(n - base < NB ? n - base : NB), Dnext, info, sm);
+  }
 }
 
 
@@ -636,6 +653,7 @@ extern "C" kq_status kq_chol_inv(const float* H, int64_t n, int64_t ldh, float d
   ws_layout(n, &w, ws);
   const int64_t ld = w.ld;
   static_assert(kStepASmem <= 227 * 1024 && 2 * (kStepBSmem + 1024) <= 228 * 1024, "smem");
+  static_assert(kPotrfSmem <= kStepBSmem, "the fused diagonal factorisation reuses step b's shared memory");
   KQ_TRY(kq::cuda_check(cudaFuncSetAttribute(potrf_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPotrfSmem), "attr"));
   KQ_TRY(kq::cuda_check(cudaFuncSetAttribute(step_a_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStepASmem), "attr"));
   KQ_TRY(kq::cuda_check(cudaFuncSetAttribute(step_b_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStepBSmem), "attr"));
@@ -673,24 +691,27 @@ extern "C" kq_status kq_chol_inv(const float* H, int64_t n, int64_t ldh, float d
     // the chain potrf -> step a -> (kNext) -> potrf runs as programmatic
     // dependents on s1: each kernel is scheduled while its predecessor
     // finishes and waits for it (griddepcontrol.wait) before reading
-    KQ_TRY(kq::launch_ex("kq_chol_inv potrf", b > 0, potrf_kernel, dim3(1), dim3(256), kPotrfSmem, s1, w.A, ld, n,
-                         k0, kb, Dk, info));
+    // block 0's diagonal factorisation has a launch of its own; every later
+    // one is done by the previous step's kNext launch (CTA 0)
+    if (b == 0)
+      KQ_TRY(kq::launch_ex("kq_chol_inv potrf", false, potrf_kernel, dim3(1), dim3(256), kPotrfSmem, s1, w.A, ld, n,
+                           k0, kb, Dk, info));
     const int64_t tp = kq::cdiv(n - k0 - kb, 128);   // > 0 only when kb == 64
     const int64_t xt = kq::cdiv(k0 + kb, 128);
-    KQ_TRY(kq::launch_ex("kq_chol_inv step a", true, step_a_kernel, dim3((unsigned)(tp + xt)), dim3(256), kStepASmem,
+    KQ_TRY(kq::launch_ex("kq_chol_inv step a", b > 0, step_a_kernel, dim3((unsigned)(tp + xt)), dim3(256), kStepASmem,
                          s1, w.A, w.X, Pt, ld, k0, tp, Dk));
     if (tp > 0) {
       const int64_t tr = kq::cdiv(n - k0 - NB, TBM), xcols = (k0 + NB) / TBN;
       KQ_TRY(kq::cuda_check(cudaEventRecord(ev_a, s1), "kq_chol_inv: record"));
       KQ_TRY(kq::cuda_check(cudaStreamWaitEvent(st, ev_a, 0), "kq_chol_inv: wait"));
       step_b_kernel<<<(unsigned)step_b_ctas(tr, xcols, kRest), 256, kStepBSmem, st>>>(w.A, w.X, Pt, ld, k0, tr,
-                                                                                      kRest);
+                                                                                      kRest, n, nullptr, info);
       KQ_TRY(kq::launch_check("kq_chol_inv step b"));
       KQ_TRY(kq::cuda_check(cudaEventRecord(ev_rest[b & 1], st), "kq_chol_inv: record"));
       if (rest_pending)
         KQ_TRY(kq::cuda_check(cudaStreamWaitEvent(s1, ev_rest[(b - 1) & 1], 0), "kq_chol_inv: wait"));
-      step_b_kernel<<<(unsigned)step_b_ctas(tr, xcols, kNext), 256, kStepBSmem, s1>>>(w.A, w.X, Pt, ld, k0, tr,
-                                                                                      kNext);
+      step_b_kernel<<<(unsigned)step_b_ctas(tr, xcols, kNext), 256, kStepBSmem, s1>>>(
+          w.A, w.X, Pt, ld, k0, tr, kNext, n, w.Dinv + (b + 1) * NB * NB, info);
       KQ_TRY(kq::launch_check("kq_chol_inv step b"));
       rest_pending = true;
     }
