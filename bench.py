@@ -164,7 +164,7 @@ def run_layer_steps(P, LayerQuantizer, spec, settings, seed, dev, steps, warmup,
     T_in = P.RHT(Ti.n, Ti.log2_p, Ti.m, Ti.signs.to(dev), None if Ti.Qm is None else Ti.Qm.to(dev))
     T_out = P.RHT(To.n, To.log2_p, To.m, To.signs.to(dev), None if To.Qm is None else To.Qm.to(dev))
     lq = LayerQuantizer(spec.d_out, spec.d_in, dev, gemm_mode=gemm_mode)
-    results = [lq.alloc_result(b, g) for b, g in settings]
+    results = lq.alloc_results(settings)
     stream = torch.cuda.current_stream()
     names = ["syrk_x2", "sensitivity", "rotate", "chol_inv", "quantize", "loss"]
     per = {n: [] for n in names}
@@ -277,7 +277,7 @@ def run_kronq(a):
     T_in, T_out = dev_rht(Ti), dev_rht(To)
     gemm_mode = P.KQ_GEMM_3XTF32 if a.gemm == "3xtf32" else P.KQ_GEMM_FP32
     lq = LayerQuantizer(spec.d_out, spec.d_in, dev, gemm_mode=gemm_mode, act_order=a.act_order)
-    results = [lq.alloc_result(b, g) for b, g in settings]
+    results = lq.alloc_results(settings)
     stream = torch.cuda.current_stream()
 
     stage_events = []   # per timed step: [(name, start_event, end_event), ...]

@@ -59,6 +59,7 @@ struct Params {
   int64_t ldc;
   const float* src;
   int64_t ld_src;
+  int64_t src_rows;
   const uint8_t* dead;
   int dead_vec;    // `dead` 4-byte aligned: the mask read 4 columns at a time
   const float* other;
@@ -266,6 +267,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       for (int h = 0; h <= p.wide; ++h) {
         const int64_t gi = m0 + h * 128 + 32 * wq + lane;
         const bool row_ok = gi < p.M;
+        const int64_t si = p.src_rows ? gi % p.src_rows : gi;   // source row
 #pragma unroll 1
         for (int g0 = 0; g0 < 128; g0 += 64) {
           const int64_t gj0 = n0 + cbase + g0;
@@ -274,7 +276,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
                             !(p.epilogue == kEpiDot && !p.other_vec);
           float pre[64];
           if (fast && (p.epilogue == kEpiDot || p.epilogue == kEpiSubtract)) {
-            const float* sp = (p.epilogue == kEpiDot ? p.other + gi * p.ld_other : p.src + gi * p.ld_src) + gj0;
+            const float* sp = (p.epilogue == kEpiDot ? p.other + gi * p.ld_other : p.src + si * p.ld_src) + gj0;
 #pragma unroll
             for (int q = 0; q < 64; q += 4) {
               const float4 w = *reinterpret_cast<const float4*>(sp + q);
@@ -337,7 +339,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
                 if (p.epilogue == kEpiDot) {
                   dot += (double)v[q] * (double)p.other[gi * p.ld_other + j];
                 } else if (p.epilogue == kEpiSubtract) {
-                  const float sv = (p.dead && p.dead[j]) ? 0.f : p.src[gi * p.ld_src + j];
+                  const float sv = (p.dead && p.dead[j]) ? 0.f : p.src[si * p.ld_src + j];
                   p.C[gi * p.ldc + j] = sv - v[q];
                 } else if (p.epilogue == kEpiStoreSplit) {
                   const float b = tf32_round(v[q]);
@@ -493,6 +495,7 @@ kq_status gemm_3xtf32(const Gemm3xTF32& g, cudaStream_t st) {
   p.ldc = g.ldc;
   p.src = g.src;
   p.ld_src = g.ld_src;
+  p.src_rows = g.src_rows;
   p.dead = g.dead;
   p.dead_vec = (g.dead && aligned(g.dead, 4)) ? 1 : 0;
   p.other = g.other;

@@ -39,6 +39,8 @@ struct Gemm3xTF32 {
   int64_t ldc = 0;
   const float* src = nullptr;      // (m, n) at src[m * ld_src + n] (subtract)
   int64_t ld_src = 0;
+  int64_t src_rows = 0;            // > 0: row m of the source is row m % src_rows (stacked
+                                   // problems that share one source)
   const uint8_t* dead = nullptr;   // subtract: src column n reads as 0 when dead[n]
   const float* other = nullptr;    // (m, n) at other[m * ld_other + n] (dot)
   int64_t ld_other = 0;

@@ -24,6 +24,7 @@
 // (round half to even); errors e = (w - w_hat) * (1/Uc[j][j]).  The grid
 // itself (scale, zero) uses IEEE fp32 division.
 #include <algorithm>
+#include <cstdint>
 #include <vector>
 
 #include "kq_gemm.cuh"
@@ -50,11 +51,20 @@ __device__ __forceinline__ float load_w(const float* __restrict__ src, int64_t l
   return src[r * ld + c];
 }
 
-// Per-channel grid from the initial rotated rows (dead columns as zeros).
-// One warp per row.
+// The per-channel settings of a stacked solve: each fits its grid to the
+// same row minimum and maximum.
+struct GridSets {
+  int count;
+  float nl[4];
+  float* scales[4];
+  float* zeros[4];
+};
+
+// Per-channel grid from the initial rotated rows (dead columns as zeros),
+// for every per-channel setting of the solve from one read of W.  One warp
+// per row.
 __global__ void grid_rows_kernel(const float* __restrict__ W, int64_t ldw, int64_t d_out, int64_t d_in,
-                                 const uint8_t* __restrict__ dead, float nl, float* __restrict__ scales,
-                                 float* __restrict__ zeros, int32_t* info) {
+                                 const uint8_t* __restrict__ dead, GridSets gs, int32_t* info) {
   const int64_t r = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   if (r >= d_out) return;
@@ -73,35 +83,52 @@ __global__ void grid_rows_kernel(const float* __restrict__ W, int64_t ldw, int64
   finite = __all_sync(0xffffffffu, finite);
   if (lane == 0) {
     if (!finite) kq::report(info, KQ_ERR_NONFINITE, r);
-    float s, z;
-    fit_grid(mn, mx, nl, &s, &z);
-    scales[r] = s;
-    zeros[r] = z;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (i >= gs.count) break;
+      float sc, z;
+      fit_grid(mn, mx, gs.nl[i], &sc, &z);
+      gs.scales[i][r] = sc;
+      gs.zeros[i][r] = z;
+    }
   }
 }
+
+// Most settings of one layer solved as one stacked problem: their rows are
+// independent chains that share Uc, so setting s's rows follow setting
+// s - 1's in W_hat and in the errors, and every launch of the solve covers
+// all of them.
+constexpr int kMaxStack = 4;
+
+// The outputs and grid of one setting.
+struct SetArgs {
+  uint8_t* codes;
+  float* scales;
+  float* zeros;
+  int64_t n_groups;
+  int group;   // 0 = per channel
+  float nl;    // 2^bits - 1
+};
 
 struct InblockArgs {
   const float* src;  // W for the first block, W_hat afterwards
   int64_t ld_src;
+  int64_t src_set;   // setting s reads its rows at src + s * src_set (0: all read W)
   float* W_hat;
   int64_t ldwh;
+  int64_t wh_set;    // setting s's rows of W_hat start at W_hat + s * wh_set
   const float* Uc;
   int64_t lduc;
   const uint8_t* dead;  // applied only when src is W
   int64_t d_out, d_in, i0;
   int bw;      // block width (<= 128)
-  int group;   // 0 = per channel
-  float nl;
-  float* scales;
-  float* zeros;
-  int64_t n_groups;
-  uint8_t* codes;
   int64_t ldq;
-  float* ET;   // [128, d_out]: the block's errors, transposed (fp32 SIMT trailing update)
+  float* ET;   // [128, d_out]: the block's errors, transposed (fp32 SIMT trailing update; one setting)
   float* Eb;   // tf32 part of the errors (3xTF32 trailing update), or NULL:
-  float* Es;   // row r, column c of the block at [r * ldE + e_col0 + c]; remainder
+  float* Es;   // row r of setting s, column c of the block at [(s d_out + r) * ldE + e_col0 + c]; remainder
   int64_t ldE, e_col0;
   int32_t* info;
+  SetArgs set[kMaxStack];   // setting s = blockIdx.y
 };
 
 // LPR lanes share a row (LPR = 8 or 4): lane L of a row group owns the
@@ -130,10 +157,16 @@ __global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
   float* inv_d = sm + BLK * BLK;  // 1 / Uc[i0 + j][i0 + j]
   const int t = threadIdx.x;
   const int lane = t & 31, L = lane & (LPR - 1);
-  const int64_t row = (int64_t)blockIdx.x * IB_ROWS + t / LPR;
+  const int64_t row = (int64_t)blockIdx.x * IB_ROWS + t / LPR;   // row of the setting
   const bool row_ok = row < a.d_out;
   const int bw = a.bw;
   const int64_t i0 = a.i0;
+  // this CTA's setting (uniform over the CTA, so its control flow is too)
+  const int s = blockIdx.y;
+  const SetArgs S = s == 0 ? a.set[0] : s == 1 ? a.set[1] : s == 2 ? a.set[2] : a.set[3];
+  const float* __restrict__ src = a.src + s * a.src_set;
+  float* __restrict__ W_hat = a.W_hat + s * a.wh_set;
+  const int64_t erow = s * a.d_out + row;   // row of the stacked errors
   kq::pdl_trigger();
 
   // the block of Uc: 16 asynchronous 16-byte copies per thread, all in
@@ -162,11 +195,11 @@ __global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
     float v[4] = {0.f, 0.f, 0.f, 0.f};
     if (row_ok) {
       if (c + 3 < bw && !a.dead) {
-        const float4 q = *reinterpret_cast<const float4*>(a.src + row * a.ld_src + i0 + c);
+        const float4 q = *reinterpret_cast<const float4*>(src + row * a.ld_src + i0 + c);
         v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
       } else {
         for (int e = 0; e < 4; ++e)
-          if (c + e < bw) v[e] = load_w(a.src, a.ld_src, row, i0 + c + e, a.dead);
+          if (c + e < bw) v[e] = load_w(src, a.ld_src, row, i0 + c + e, a.dead);
       }
       if (!(isfinite(v[0]) && isfinite(v[1]) && isfinite(v[2]) && isfinite(v[3])))
         kq::report(a.info, KQ_ERR_NONFINITE, row);
@@ -186,9 +219,9 @@ __global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
   __syncthreads();
 
   float scale = 1.f, zero = 0.f;
-  if (!a.group && row_ok) {
-    scale = a.scales[row * a.n_groups];
-    zero = a.zeros[row * a.n_groups];
+  if (!S.group && row_ok) {
+    scale = S.scales[row * S.n_groups];
+    zero = S.zeros[row * S.n_groups];
   }
   float inv_scale = 1.f / scale;
   float qv[NR], ev[NR];
@@ -202,11 +235,11 @@ __global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
       for (int tt = 0; tt < 4; ++tt) {
         const int j = SPAN * m + 4 * Lo + tt;   // column quantized in this step
         if (j >= bw) break;
-        if (a.group && tt == 0 && ((i0 + j) % a.group) == 0) {
+        if (S.group && tt == 0 && ((i0 + j) % S.group) == 0) {
           // group grid on the current values of columns [j, j + group): every
           // lane folds its own columns in range, then the row's lanes meet
           const int64_t lim = a.d_in - i0;
-          const int gend = (int)((int64_t)(j + a.group) < lim ? (int64_t)(j + a.group) : lim);
+          const int gend = (int)((int64_t)(j + S.group) < lim ? (int64_t)(j + S.group) : lim);
           float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
           for (int r = 0; r < NR; ++r) {
@@ -221,12 +254,12 @@ __global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
             mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
           }
-          fit_grid(mn, mx, a.nl, &scale, &zero);
+          fit_grid(mn, mx, S.nl, &scale, &zero);
           inv_scale = 1.f / scale;
           if (row_ok && L == 0) {
-            const int64_t g = (i0 + j) / a.group;
-            a.scales[row * a.n_groups + g] = scale;
-            a.zeros[row * a.n_groups + g] = zero;
+            const int64_t g = (i0 + j) / S.group;
+            S.scales[row * S.n_groups + g] = scale;
+            S.zeros[row * S.n_groups + g] = zero;
           }
         }
         // every lane runs the owner's arithmetic on its own register 4m+tt;
@@ -234,7 +267,7 @@ __global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
         const int r = 4 * m + tt;
         const float x = w[r];
         const float v = fmaf(x, inv_scale, zero);
-        const float q = fminf(fmaxf(rintf(v), 0.f), a.nl);
+        const float q = fminf(fmaxf(rintf(v), 0.f), S.nl);
         const float wh = scale * (q - zero);
         const float e_own = (x - wh) * inv_d[j];
         const float e = __shfl_sync(0xffffffffu, e_own, gbase + Lo);
@@ -265,16 +298,16 @@ __global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
   for (int m = 0; m < MB; ++m) {
     const int c = SPAN * m + 4 * L;
     if (c + 3 < bw) {
-      *reinterpret_cast<float4*>(a.W_hat + row * a.ldwh + i0 + c) = make_float4(w[4 * m], w[4 * m + 1], w[4 * m + 2],
-                                                                               w[4 * m + 3]);
+      *reinterpret_cast<float4*>(W_hat + row * a.ldwh + i0 + c) = make_float4(w[4 * m], w[4 * m + 1], w[4 * m + 2],
+                                                                             w[4 * m + 3]);
       uchar4 qq = make_uchar4((unsigned char)qv[4 * m], (unsigned char)qv[4 * m + 1], (unsigned char)qv[4 * m + 2],
                               (unsigned char)qv[4 * m + 3]);
-      *reinterpret_cast<uchar4*>(a.codes + row * a.ldq + i0 + c) = qq;
+      *reinterpret_cast<uchar4*>(S.codes + row * a.ldq + i0 + c) = qq;
     } else {
       for (int e = 0; e < 4; ++e)
         if (c + e < bw) {
-          a.W_hat[row * a.ldwh + i0 + c + e] = w[4 * m + e];
-          a.codes[row * a.ldq + i0 + c + e] = (uint8_t)qv[4 * m + e];
+          W_hat[row * a.ldwh + i0 + c + e] = w[4 * m + e];
+          S.codes[row * a.ldq + i0 + c + e] = (uint8_t)qv[4 * m + e];
         }
     }
     if (a.Eb) {
@@ -287,8 +320,8 @@ __global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
         b[e] = __uint_as_float(bits);
         sm4[e] = ee - b[e];
       }
-      *reinterpret_cast<float4*>(a.Eb + row * a.ldE + a.e_col0 + c) = make_float4(b[0], b[1], b[2], b[3]);
-      *reinterpret_cast<float4*>(a.Es + row * a.ldE + a.e_col0 + c) = make_float4(sm4[0], sm4[1], sm4[2], sm4[3]);
+      *reinterpret_cast<float4*>(a.Eb + erow * a.ldE + a.e_col0 + c) = make_float4(b[0], b[1], b[2], b[3]);
+      *reinterpret_cast<float4*>(a.Es + erow * a.ldE + a.e_col0 + c) = make_float4(sm4[0], sm4[1], sm4[2], sm4[3]);
     } else {
       for (int e = 0; e < 4; ++e)
         if (c + e < bw) a.ET[(int64_t)(c + e) * a.d_out + row] = ev[4 * m + e];
@@ -428,8 +461,10 @@ struct QuantWs {
   int64_t ldu;
 };
 
-// Most settings kq_quantize_layer_multi solves side by side.
+// Most settings kq_quantize_layer_multi solves side by side (when their
+// outputs are not stacked); the workspace size serves both forms.
 constexpr int kMaxLanes = 4;
+static_assert(kMaxLanes == kMaxStack, "one workspace size for lanes and stacks");
 
 size_t quant_layout(int64_t d_out, int64_t d_in, int lanes, int lane, QuantWs* w, void* base) {
   const int64_t ldu = (d_in + 3) / 4 * 4;
@@ -445,6 +480,25 @@ size_t quant_layout(int64_t d_out, int64_t d_in, int lanes, int lane, QuantWs* w
     w->ldu = ldu;
   }
   return 2 * se * lanes + 2 * su;
+}
+
+// The workspace of a stacked solve of `count` settings: their errors as one
+// [count d_out, OUTER] matrix (tf32 part, then remainder), then the split of
+// Uc^T; the same size as `count` lanes side by side.
+size_t stack_layout(int64_t d_out, int64_t d_in, int count, QuantWs* w, void* base) {
+  const int64_t ldu = (d_in + 3) / 4 * 4;
+  const size_t se = kq::align_up((size_t)d_out * OUTER * sizeof(float), 256);
+  const size_t su = kq::align_up((size_t)d_in * ldu * sizeof(float), 256);
+  if (w && base) {
+    char* b = static_cast<char*>(base);
+    w->ET = reinterpret_cast<float*>(b);
+    w->Eb = w->ET;
+    w->Es = reinterpret_cast<float*>(b + se * count);
+    w->Ub = reinterpret_cast<float*>(b + 2 * se * count);
+    w->Us = reinterpret_cast<float*>(b + 2 * se * count + su);
+    w->ldu = ldu;
+  }
+  return 2 * se * count + 2 * su;
 }
 
 }  // namespace
@@ -488,23 +542,51 @@ kq_status check_args(const float* W, int64_t d_out, int64_t d_in, int64_t ldw, c
   return KQ_OK;
 }
 
-// Enqueues one checked setting on `st` with the workspace lane `w`; the tf32
-// split of Uc^T (3xTF32 mode) is formed here unless `split_uc` is false
-// (then it is already in the workspace, from an earlier setting).
-kq_status enqueue_setting(const float* W, int64_t d_out, int64_t d_in, int64_t ldw, const float* Uc, int64_t lduc,
-                          const uint8_t* dead_mask, int bits, int group, int gemm_mode, uint8_t* codes, int64_t ldq,
-                          float* scales, float* zeros, float* W_hat, int64_t ldwh, const QuantWs& w, int32_t* info,
-                          cudaStream_t st, bool split_uc) {
+// One setting as the caller passes it.
+struct SetOut {
+  int bits, group;
+  uint8_t* codes;
+  float* scales;
+  float* zeros;
+};
+
+// Enqueues `count` (<= kMaxStack) checked settings on `st` as one stacked
+// solve: setting i's rows of W_hat start at W_hat + i d_out ldwh, its
+// errors at row i d_out of the workspace's E, and every launch covers all
+// the settings (M = count d_out in the trailing updates, whose first
+// super-block reads W for every setting).  The tf32 split of Uc^T (3xTF32
+// mode) is formed here unless `split_uc` is false (then it is already in the
+// workspace).  The fp32 SIMT mode solves one setting per call (count == 1).
+kq_status enqueue_stacked(const float* W, int64_t d_out, int64_t d_in, int64_t ldw, const float* Uc, int64_t lduc,
+                          const uint8_t* dead_mask, int count, const SetOut* so, int gemm_mode, int64_t ldq,
+                          float* W_hat, int64_t ldwh, const QuantWs& w, int32_t* info, cudaStream_t st,
+                          bool split_uc) {
   const bool tc = (gemm_mode == KQ_GEMM_3XTF32);
+  if (count < 1 || count > kMaxStack || (!tc && count != 1))
+    return kq::fail(KQ_ERR_INVALID_ARG, "kq_quantize_layer: a stacked solve of %d settings", count);
   if (tc && split_uc) KQ_TRY(kq::split_tf32(Uc, lduc, nullptr, 0, d_in, d_in, w.Ub, w.Us, w.ldu, true, st));
+  const int64_t M = count * d_out;
+  const int64_t wh_set = d_out * ldwh;
 
-  const float nl = (float)((1 << bits) - 1);
-  const int64_t n_groups = group ? kq::cdiv(d_in, group) : 1;
-
-  if (!group) {
+  SetArgs sets[kMaxStack] = {};
+  GridSets gs = {};
+  for (int i = 0; i < count; ++i) {
+    sets[i].codes = so[i].codes;
+    sets[i].scales = so[i].scales;
+    sets[i].zeros = so[i].zeros;
+    sets[i].group = so[i].group;
+    sets[i].n_groups = so[i].group ? kq::cdiv(d_in, so[i].group) : 1;
+    sets[i].nl = (float)((1 << so[i].bits) - 1);
+    if (!so[i].group) {
+      gs.nl[gs.count] = sets[i].nl;
+      gs.scales[gs.count] = so[i].scales;
+      gs.zeros[gs.count] = so[i].zeros;
+      ++gs.count;
+    }
+  }
+  if (gs.count) {
     KQ_TRY(timed(kClassGrid, 0.0, 4.0 * d_out * d_in, st, [&]() -> kq_status {
-      grid_rows_kernel<<<(unsigned)kq::cdiv(d_out, 8), 256, 0, st>>>(W, ldw, d_out, d_in, dead_mask, nl, scales,
-                                                                     zeros, info);
+      grid_rows_kernel<<<(unsigned)kq::cdiv(d_out, 8), 256, 0, st>>>(W, ldw, d_out, d_in, dead_mask, gs, info);
       return kq::launch_check("kq_quantize_layer grid");
     }));
   }
@@ -513,11 +595,13 @@ kq_status enqueue_setting(const float* W, int64_t d_out, int64_t d_in, int64_t l
   auto inblock = [&](int64_t i0, int64_t o0) -> kq_status {
     const int bw = (int)std::min<int64_t>(BLK, d_in - i0);
     const bool first = (i0 == 0);
-    InblockArgs a;
+    InblockArgs a = {};
     a.src = first ? W : W_hat;
     a.ld_src = first ? ldw : ldwh;
+    a.src_set = first ? 0 : wh_set;
     a.W_hat = W_hat;
     a.ldwh = ldwh;
+    a.wh_set = wh_set;
     a.Uc = Uc;
     a.lduc = lduc;
     a.dead = first ? dead_mask : nullptr;
@@ -525,12 +609,6 @@ kq_status enqueue_setting(const float* W, int64_t d_out, int64_t d_in, int64_t l
     a.d_in = d_in;
     a.i0 = i0;
     a.bw = bw;
-    a.group = group;
-    a.nl = nl;
-    a.scales = scales;
-    a.zeros = zeros;
-    a.n_groups = n_groups;
-    a.codes = codes;
     a.ldq = ldq;
     a.ET = w.ET;
     a.Eb = tc ? w.Eb : nullptr;
@@ -538,19 +616,21 @@ kq_status enqueue_setting(const float* W, int64_t d_out, int64_t d_in, int64_t l
     a.ldE = OUTER;
     a.e_col0 = i0 - o0;
     a.info = info;
+    for (int i = 0; i < count; ++i) a.set[i] = sets[i];
     // after the first block the previous kernel is this solve's own trailing
     // update, so the launch may overlap its tail (tensor-core mode)
-    return timed(kClassInblock, 0.0, (double)d_out * bw * (tc ? 17.0 : 13.0), st, [&]() {
+    return timed(kClassInblock, 0.0, (double)M * bw * (tc ? 17.0 : 13.0), st, [&]() {
       return kq::launch_ex("kq_quantize_layer inblock", tc && i0 > 0, inblock_kernel<kLanesPerRow>,
-                           dim3((unsigned)kq::cdiv(d_out, IB_THREADS / kLanesPerRow)), dim3(IB_THREADS), IB_SMEM, st,
-                           a);
+                           dim3((unsigned)kq::cdiv(d_out, IB_THREADS / kLanesPerRow), (unsigned)count),
+                           dim3(IB_THREADS), IB_SMEM, st, a);
     });
   };
-  // W_hat[:, c0:c0+N] = src[:, c0:c0+N] - E[:, e0:e0+K] Uc[k0:k0+K, c0:c0+N]; the
-  // source is W (dead columns as zeros) while those columns are still untouched.
+  // W_hat[:, c0:c0+N] = src[:, c0:c0+N] - E[:, e0:e0+K] Uc[k0:k0+K, c0:c0+N] over
+  // the stacked rows; the source is W (dead columns as zeros, row r of every
+  // setting reading W's row r mod d_out) while those columns are untouched.
   auto update = [&](int64_t c0, int64_t N, int64_t e0, int64_t k0, int64_t K, bool from_w) -> kq_status {
     kq::Gemm3xTF32 g;
-    g.M = d_out;
+    g.M = M;
     g.N = N;
     g.K = K;
     g.a_big = w.Eb;
@@ -567,10 +647,11 @@ kq_status enqueue_setting(const float* W, int64_t d_out, int64_t d_in, int64_t l
     g.ldc = ldwh;
     g.src = (from_w ? W : W_hat) + c0;
     g.ld_src = from_w ? ldw : ldwh;
+    g.src_rows = from_w ? d_out : 0;
     g.dead = from_w && dead_mask ? dead_mask + c0 : nullptr;
     g.info = info;
     g.pdl = true;   // always follows this solve's in-block kernel
-    return timed(kClassUpdate, 2.0 * d_out * N * K, 0.0, st, [&]() { return kq::gemm_3xtf32(g, st); });
+    return timed(kClassUpdate, 2.0 * M * N * K, 0.0, st, [&]() { return kq::gemm_3xtf32(g, st); });
   };
   if (!tc) {
     for (int64_t i0 = 0; i0 < d_in; i0 += BLK) {
@@ -652,9 +733,10 @@ extern "C" kq_status kq_quantize_layer(const float* W, int64_t d_out, int64_t d_
   if (!ws || !kq::aligned(ws, 256) || ws_bytes < kq_quantize_layer_workspace_size(d_out, d_in, block))
     return kq::fail(KQ_ERR_WORKSPACE, "kq_quantize_layer: workspace too small or not 256-byte aligned");
   QuantWs w;
-  quant_layout(d_out, d_in, 1, 0, &w, ws);
-  return enqueue_setting(W, d_out, d_in, ldw, Uc, lduc, dead_mask, bits, group, gemm_mode, codes, ldq, scales, zeros,
-                         W_hat, ldwh, w, info, (cudaStream_t)stream, true);
+  stack_layout(d_out, d_in, 1, &w, ws);
+  const SetOut so = {bits, group, codes, scales, zeros};
+  return enqueue_stacked(W, d_out, d_in, ldw, Uc, lduc, dead_mask, 1, &so, gemm_mode, ldq, W_hat, ldwh, w, info,
+                         (cudaStream_t)stream, true);
 }
 
 extern "C" kq_status kq_quantize_layer_multi(const float* W, int64_t d_out, int64_t d_in, int64_t ldw,
@@ -675,19 +757,39 @@ extern "C" kq_status kq_quantize_layer_multi(const float* W, int64_t d_out, int6
   }
   if (!ws || !kq::aligned(ws, 256))
     return kq::fail(KQ_ERR_WORKSPACE, "kq_quantize_layer_multi: workspace NULL or not 256-byte aligned");
-  // side by side when the workspace holds a lane per setting (up to
-  // kMaxLanes), else one after the other in a single lane
+  cudaStream_t st = (cudaStream_t)stream;
+  std::vector<SetOut> so(count);
+  for (int i = 0; i < count; ++i) so[i] = SetOut{bits[i], group[i], codes[i], scales[i], zeros[i]};
+  // Stacked when the settings' W_hat buffers follow one another (setting i
+  // at W_hat[0] + i d_out ldwh) and the trailing updates run on the tensor
+  // cores: up to kMaxStack settings per solve, every launch covering all
+  // of them.
+  bool stacked = gemm_mode == KQ_GEMM_3XTF32 && (int64_t)std::min(count, kMaxStack) * d_out <= INT32_MAX;
+  for (int i = 1; i < count && stacked; ++i) stacked = (W_hat[i] == W_hat[0] + (int64_t)i * d_out * ldwh);
+  if (stacked) {
+    int per = std::min(count, kMaxStack);
+    while (per > 1 && ws_bytes < stack_layout(d_out, d_in, per, nullptr, nullptr)) --per;
+    if (ws_bytes < stack_layout(d_out, d_in, per, nullptr, nullptr))
+      return kq::fail(KQ_ERR_WORKSPACE, "kq_quantize_layer_multi: workspace too small");
+    QuantWs sw;
+    stack_layout(d_out, d_in, per, &sw, ws);
+    for (int i0 = 0; i0 < count; i0 += per)
+      KQ_TRY(enqueue_stacked(W, d_out, d_in, ldw, Uc, lduc, dead_mask, std::min(per, count - i0), so.data() + i0,
+                             gemm_mode, ldq, W_hat[i0], ldwh, sw, info, st, i0 == 0));
+    return KQ_OK;
+  }
+  // otherwise side by side when the workspace holds a lane per setting (up
+  // to kMaxLanes), else one after the other in a single lane
   int lanes = std::min(count, kMaxLanes);
   if (ws_bytes < quant_layout(d_out, d_in, lanes, 0, nullptr, nullptr)) lanes = 1;
   if (ws_bytes < quant_layout(d_out, d_in, lanes, 0, nullptr, nullptr))
     return kq::fail(KQ_ERR_WORKSPACE, "kq_quantize_layer_multi: workspace too small");
   QuantWs w[kMaxLanes];
   for (int l = 0; l < lanes; ++l) quant_layout(d_out, d_in, lanes, l, &w[l], ws);
-  cudaStream_t st = (cudaStream_t)stream;
   if (lanes == 1) {
     for (int i = 0; i < count; ++i)
-      KQ_TRY(enqueue_setting(W, d_out, d_in, ldw, Uc, lduc, dead_mask, bits[i], group[i], gemm_mode, codes[i], ldq,
-                             scales[i], zeros[i], W_hat[i], ldwh, w[0], info, st, i == 0));
+      KQ_TRY(enqueue_stacked(W, d_out, d_in, ldw, Uc, lduc, dead_mask, 1, &so[i], gemm_mode, ldq, W_hat[i], ldwh, w[0],
+                             info, st, i == 0));
     return KQ_OK;
   }
   Lanes* L = nullptr;
@@ -701,8 +803,8 @@ extern "C" kq_status kq_quantize_layer_multi(const float* W, int64_t d_out, int6
   kq_status first = KQ_OK;
   for (int i = 0; i < count && first == KQ_OK; ++i) {
     const int l = i % lanes;
-    first = enqueue_setting(W, d_out, d_in, ldw, Uc, lduc, dead_mask, bits[i], group[i], gemm_mode, codes[i], ldq,
-                            scales[i], zeros[i], W_hat[i], ldwh, w[l], info, l ? L->s[l - 1] : st, false);
+    first = enqueue_stacked(W, d_out, d_in, ldw, Uc, lduc, dead_mask, 1, &so[i], gemm_mode, ldq, W_hat[i], ldwh, w[l],
+                            info, l ? L->s[l - 1] : st, false);
   }
   // the join is enqueued even after a failed launch, so that the caller's
   // stream is ordered after everything that did get enqueued

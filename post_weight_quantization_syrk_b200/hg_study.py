@@ -130,7 +130,7 @@ def run_layer(name, n_tokens, ks, dev, recipe="pages"):
             before_rotate(lq)
         lq.rotate(W, T_in, T_o)
         lq.factor(0.01)
-        res = [lq.alloc_result(b, g) for b, g in settings]
+        res = lq.alloc_results(settings)
         lq.quantize_all(res)
         lq.loss_all(res)
         e.record()

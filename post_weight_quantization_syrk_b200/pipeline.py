@@ -70,20 +70,32 @@ class LayerQuantizer:
             self._ws_bytes = nbytes
         return self._ws
 
-    def alloc_result(self, bits, group):
+    def alloc_result(self, bits, group, solve_out=None):
+        """Buffers of one setting; `solve_out` (d_out x d_in fp32), if given,
+        becomes the buffer the solve writes W_hat into."""
         ng = 1 if not group else -(-self.d_in // group)
         dev = self.device
+        q = self.act_order
         r = BitResult(bits, group,
                       torch.empty((self.d_out, self.d_in), dtype=torch.uint8, device=dev),
                       torch.empty((self.d_out, ng), dtype=torch.float32, device=dev),
                       torch.empty((self.d_out, ng), dtype=torch.float32, device=dev),
+                      solve_out if solve_out is not None and not q else
                       torch.empty((self.d_out, self.d_in), dtype=torch.float32, device=dev),
                       torch.zeros(1, dtype=torch.float64, device=dev))
-        if self.act_order:
+        if q:
             r.codes_q = torch.empty_like(r.codes)
-            r.W_hat_q = torch.empty_like(r.W_hat)
+            r.W_hat_q = solve_out if solve_out is not None else torch.empty_like(r.W_hat)
             r.perm = self.perm_in
         return r
+
+    def alloc_results(self, settings):
+        """Buffers of several settings, the W_hat the solve writes stacked in
+        one [count, d_out, d_in] tensor: kq_quantize_layer_multi then solves
+        the settings as one problem (their rows are independent chains that
+        share U_c)."""
+        stack = torch.empty((len(settings), self.d_out, self.d_in), dtype=torch.float32, device=self.device)
+        return [self.alloc_result(b, g, stack[i]) for i, (b, g) in enumerate(settings)]
 
     # -- steps -----------------------------------------------------------
     def statistics(self, X, G, n_total=None, accumulate=False, stream=None):
@@ -167,7 +179,8 @@ class LayerQuantizer:
 
     def quantize_all(self, results, stream=None):
         """Every setting of `results` in one call: the factor's operand split is
-        shared and up to four settings are solved side by side."""
+        shared, and up to four settings are solved as one stacked problem
+        (results from alloc_results) or else side by side."""
         ws = self.workspace(K.kq_quantize_layer_multi_workspace_size(self.d_out, self.d_in, self.block, len(results)))
         Win = self._solve_input(stream)
         q = self.act_order
@@ -191,7 +204,7 @@ class LayerQuantizer:
         self.rotate(W, T_in, T_out, stream)
         self.factor(damp_frac, stream)
         if results is None:
-            results = [self.alloc_result(b, g) for b, g in settings]
+            results = self.alloc_results(settings)
         self.quantize_all(results, stream)
         self.loss_all(results, stream)
         return results

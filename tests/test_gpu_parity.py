@@ -452,6 +452,14 @@ def test_multi_entry_points_match_single_calls(P, rotated_small, gemm_mode):
         return res
 
     one, many, seq = outputs(), outputs(), outputs()
+    # the same settings with their W_hat stacked in one buffer: solved as one
+    # problem (four settings, then the fifth), or one at a time when the
+    # workspace holds one setting
+    stk, stk1 = outputs(), outputs()
+    for outs in (stk, stk1):
+        buf = torch.empty((len(settings), d_out, d_in), device="cuda")
+        for i, o in enumerate(outs):
+            outs[i] = (o[0], o[1], o[2], buf[i], o[4])
     info = _info()
     for (b, g), (c, s, z, wh, l) in zip(settings, one):
         P.kq_quantize_layer(lq.Wp, lq.Uc, lq.dead, b, g, c, s, z, wh, gemm_mode=mode, info=info)
@@ -463,9 +471,64 @@ def test_multi_entry_points_match_single_calls(P, rotated_small, gemm_mode):
     P.kq_quantize_layer_multi(lq.Wp, lq.Uc, lq.dead, settings, [o[0] for o in seq], [o[1] for o in seq],
                               [o[2] for o in seq], [o[3] for o in seq], gemm_mode=mode, ws=ws1, info=info)
     P.kq_kron_loss_multi(lq.Wp, [o[3] for o in seq], lq.H_X, lq.H_G, [o[4] for o in seq])
+    P.kq_quantize_layer_multi(lq.Wp, lq.Uc, lq.dead, settings, [o[0] for o in stk], [o[1] for o in stk],
+                              [o[2] for o in stk], [o[3] for o in stk], gemm_mode=mode, info=info)
+    P.kq_kron_loss_multi(lq.Wp, [o[3] for o in stk], lq.H_X, lq.H_G, [o[4] for o in stk])
+    P.kq_quantize_layer_multi(lq.Wp, lq.Uc, lq.dead, settings, [o[0] for o in stk1], [o[1] for o in stk1],
+                              [o[2] for o in stk1], [o[3] for o in stk1], gemm_mode=mode, ws=ws1, info=info)
+    P.kq_kron_loss_multi(lq.Wp, [o[3] for o in stk1], lq.H_X, lq.H_G, [o[4] for o in stk1])
     torch.cuda.synchronize()
     assert _info_code(info)[0] == 0
-    for a, b, c in zip(one, many, seq):
-        for x, y, z in zip(a, b, c):
+    for a, *rest in zip(one, many, seq, stk, stk1):
+        for k, x in enumerate(a):
+            for r in rest:
+                assert torch.equal(x, r[k])
+
+
+@pytest.mark.parametrize("d_out,d_in", [(200, 260), (33, 136)])
+def test_stacked_solve_ragged_rows(P, d_out, d_in):
+    """Settings stacked in one solve (M = count d_out rows in every trailing
+    update, the first super-block reading W's row r mod d_out) against one
+    call per setting, bit for bit, at row counts that leave partial CTAs and
+    tiles, with dead columns; a non-finite weight is reported with its row in
+    W."""
+    rng = np.random.default_rng(d_out + d_in)
+    W = torch.from_numpy(rng.normal(0, 0.02, (d_out, d_in)).astype(np.float32)).cuda()
+    H = torch.from_numpy(_spd(d_in, 5, 1.0)).cuda()
+    dead = torch.zeros(d_in, dtype=torch.uint8, device="cuda")
+    dead[[3, d_in - 2]] = 1
+    H[3, :] = 0
+    H[:, 3] = 0
+    H[d_in - 2, :] = 0
+    H[:, d_in - 2] = 0
+    Uc = torch.empty_like(H)
+    info = _info()
+    P.kq_chol_inv(H, 0.01, Uc, dead, None, info)
+    settings = [(2, 0), (3, 32), (4, 0)]
+
+    def outputs(stacked):
+        buf = torch.empty((len(settings), d_out, d_in), device="cuda") if stacked else None
+        res = []
+        for i, (b, g) in enumerate(settings):
+            ng = 1 if not g else -(-d_in // g)
+            res.append((torch.empty((d_out, d_in), dtype=torch.uint8, device="cuda"),
+                        torch.empty((d_out, ng), device="cuda"), torch.empty((d_out, ng), device="cuda"),
+                        buf[i] if stacked else torch.empty((d_out, d_in), device="cuda")))
+        return res
+
+    one, stk = outputs(False), outputs(True)
+    for (b, g), (c, s_, z, wh) in zip(settings, one):
+        P.kq_quantize_layer(W, Uc, dead, b, g, c, s_, z, wh, gemm_mode=P.KQ_GEMM_3XTF32, info=info)
+    P.kq_quantize_layer_multi(W, Uc, dead, settings, *[[o[k] for o in stk] for k in range(4)],
+                              gemm_mode=P.KQ_GEMM_3XTF32, info=info)
+    torch.cuda.synchronize()
+    assert _info_code(info)[0] == 0
+    for a, b in zip(one, stk):
+        for x, y in zip(a, b):
             assert torch.equal(x, y)
-            assert torch.equal(x, z)
+    bad = W.clone()
+    bad[d_out - 1, d_in // 2] = float("inf")
+    info = _info()
+    P.kq_quantize_layer_multi(bad, Uc, dead, settings, *[[o[k] for o in stk] for k in range(4)],
+                              gemm_mode=P.KQ_GEMM_3XTF32, info=info)
+    assert _info_code(info) == (7, d_out - 1)
