@@ -309,7 +309,14 @@ kq_status kq_quantize_layer(const float* W, int64_t d_out, int64_t d_in, int64_t
  * layer (the same W, Uc and dead mask; bit-width bits[i] and group group[i]
  * into codes[i], scales[i], zeros[i], W_hat[i]).  The 3xTF32 operand split
  * of Uc is formed once for all settings (KronQ paper page, authors' reply:
- * one set of statistics serves every bit-width).  With a workspace of
+ * one set of statistics serves every bit-width).  Stacked outputs: in
+ * 3xTF32 mode, when W_hat[i] == W_hat[0] + i * d_out * ldwh for every i
+ * (one [count, d_out, ldwh] buffer), up to 4 settings are solved as ONE
+ * problem of count * d_out rows (the rows are independent chains that share
+ * Uc): each in-block launch covers every setting's rows, each trailing
+ * update is one product with M = count * d_out, and the per-channel grids
+ * come from one pass over W; settings beyond 4 form further such solves.
+ * Otherwise, with a workspace of
  * kq_quantize_layer_multi_workspace_size(d_out, d_in, block, count) bytes
  * up to 4 settings are solved side by side: setting i runs on lane i % 4,
  * lane 0 being `stream` and the others internal streams of the library
@@ -317,7 +324,8 @@ kq_status kq_quantize_layer(const float* W, int64_t d_out, int64_t d_in, int64_t
  * forked from and joined back into `stream` by events, so all the work is
  * still ordered on `stream` as one call.  With a smaller workspace of at
  * least kq_quantize_layer_workspace_size bytes the settings run one after
- * the other on `stream`.  The results are the same either way, bit for bit.
+ * the other on `stream` (stacked outputs: one stacked solve per setting).
+ * The results are the same in every form, bit for bit.
  * The pointer arrays are HOST arrays of device pointers, read during the
  * call; no two settings may share an output buffer.  Errors as
  * kq_quantize_layer; count >= 1; every setting is validated before any
