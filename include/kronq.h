@@ -482,8 +482,14 @@ kq_status kq_allocate_bits(const double* sens, const int64_t* n_params, int n_la
  *   kq_quantize_layer writes.  T_in (order d_in) / T_out (order d_out) as
  *   for kq_rotate; NULL means the identity (the plain dequantized matvec).
  *   X fp32 [batch, d_in] (ldx >= d_in), Y fp32 [batch, d_out] (ldy >=
- *   d_out; 16-byte aligned with ldy % 4 == 0 when T_out is given).
- *   ws: kq_reverted_matvec_workspace_size(d_in, batch) bytes.
+ *   d_out; 16-byte aligned with ldy % 4 == 0 when T_out is given);
+ *   d_in <= 2^24 (KQ_ERR_UNSUPPORTED_SHAPE above).
+ *   ws: kq_reverted_matvec_workspace_size(d_in, batch) bytes (U x is formed
+ *   there; without T_in an X that is 16-byte aligned with ldx % 4 == 0 is
+ *   read in place).  Kernels: for bits in {2, 3, 4, 8} a row-tiled matvec
+ *   (x staged per chunk in shared memory and read once per CTA, the next
+ *   chunk's x and packed words in flight while one is summed, each code
+ *   decoded once for all vectors); other widths one warp per row.
  * ------------------------------------------------------------------------ */
 kq_status kq_pack_codes(const uint8_t* codes, int64_t rows, int64_t cols, int64_t ldq, int bits,
                         uint32_t* packed, int64_t ldp, int32_t* info, kq_stream_t stream);

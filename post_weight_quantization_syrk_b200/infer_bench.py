@@ -7,9 +7,11 @@ the same packed matvec without rotations.
 For each layer shape of the 7B model (4-bit, per-channel grid) and batch 1
 and 8, it cycles through 24 distinct packed layers (more bytes than L2, so
 the weights stream from HBM as in decode) and reports the CUDA-event time per
-kq_reverted_matvec call, issued back to back from Python: at batch 1 the
+kq_reverted_matvec call, issued back to back from Python (at batch 1 the
 plain call is bound by the host's launch rate, so its time is an upper bound
-of the device time.  The rotation parameters are seeded synthetic draws.
+of the device time), and the device time per call with the 24 calls captured
+in one CUDA graph and replayed.  The rotation parameters are seeded synthetic
+draws.
 """
 import torch
 
@@ -52,10 +54,29 @@ def main(shapes=((4096, 4096), (11008, 4096), (4096, 11008)), batches=(1, 8), n_
                 e1.record()
                 torch.cuda.synchronize()
                 us[name] = e0.elapsed_time(e1) / n * 1e3
+                # device time: the calls of one pass over the layers as a CUDA graph
+                side = torch.cuda.Stream()
+                side.wait_stream(torch.cuda.current_stream())
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.stream(side):
+                    with torch.cuda.graph(graph, stream=side):
+                        for i in range(n_layers):
+                            P.kq_reverted_matvec(layers[i], bits, scales, zeros, 0, a, b, X, Y, ws)
+                torch.cuda.current_stream().wait_stream(side)
+                graph.replay()
+                torch.cuda.synchronize()
+                e0.record()
+                for _ in range(10):
+                    graph.replay()
+                e1.record()
+                torch.cuda.synchronize()
+                us[name + "_dev"] = e0.elapsed_time(e1) / (10 * n_layers) * 1e3
+                del graph
             gb = d_out * d_in * bits / 8 / 1e9
-            print(f"{d_out}x{d_in} {bits}-bit batch {batch}: reverted {us['reverted']:.2f} us, plain "
-                  f"{us['plain']:.2f} us, weights {gb * 1e3:.1f} MB -> plain {gb / (us['plain'] * 1e-6):.0f} GB/s, "
-                  f"overhead {us['reverted'] - us['plain']:.2f} us", flush=True)
+            print(f"{d_out}x{d_in} {bits}-bit batch {batch}: reverted {us['reverted']:.2f} us "
+                  f"(device {us['reverted_dev']:.2f}), plain {us['plain']:.2f} us (device {us['plain_dev']:.2f}, "
+                  f"{gb / (us['plain_dev'] * 1e-6):.0f} GB/s of packed weights), weights {gb * 1e3:.1f} MB, "
+                  f"rotation overhead on the device {us['reverted_dev'] - us['plain_dev']:.2f} us", flush=True)
         del layers
         torch.cuda.empty_cache()
 

@@ -60,6 +60,10 @@ def test_pack_codes_reports_a_code_outside_the_width(P):
     (2, 64, 64, 128, 8),     # powers of two
     (4, 128, 200, 384, 3),   # ragged row count
     (3, 0, 40, 100, 2),      # d_in not a multiple of 32 (ragged last chunk)
+    (3, 0, 96, 2496, 8),     # several 1024-column chunks of x, ragged last tile
+    (8, 128, 72, 1312, 3),   # 8-bit codes, grouped, ragged last group
+    (2, 32, 4864, 1056, 4),  # enough rows for four rows per warp
+    (5, 0, 36, 70, 2),       # a width the row-tiled kernel does not take
 ])
 def test_reverted_matvec_matches_oracle(P, bits, group, d_out, d_in, batch):
     rng = np.random.default_rng(bits * 1000 + d_in + batch)
