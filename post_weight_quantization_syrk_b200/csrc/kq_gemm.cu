@@ -60,6 +60,7 @@ struct Params {
   const float* src;
   int64_t ld_src;
   int64_t src_rows;
+  int trigger_early;
   const uint8_t* dead;
   int dead_vec;    // `dead` 4-byte aligned: the mask read 4 columns at a time
   const float* other;
@@ -152,6 +153,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
   // CTAs per SM and would pile onto the SMs this grid leaves idle (measured
   // 17 % slower at d_out = 4096); it starts as these CTAs exit instead.
   pdl_wait();
+  if (p.trigger_early) pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -496,6 +498,7 @@ kq_status gemm_3xtf32(const Gemm3xTF32& g, cudaStream_t st) {
   p.src = g.src;
   p.ld_src = g.ld_src;
   p.src_rows = g.src_rows;
+  p.trigger_early = g.trigger_early ? 1 : 0;
   p.dead = g.dead;
   p.dead_vec = (g.dead && aligned(g.dead, 4)) ? 1 : 0;
   p.other = g.other;

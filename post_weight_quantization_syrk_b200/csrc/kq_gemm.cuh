@@ -49,6 +49,9 @@ struct Gemm3xTF32 {
   // Launched as a programmatic dependent of the previous kernel on the
   // stream, which must be a kernel of the same call (see pdl_wait).
   bool pdl = false;
+  // Let the next kernel on the stream be scheduled as soon as this grid has
+  // started (its own griddepcontrol.wait still waits for this grid's stores).
+  bool trigger_early = false;
 };
 
 // Output tiles of an M x N x K product as launched (`partial` holds 8 per

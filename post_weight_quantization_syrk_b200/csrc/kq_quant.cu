@@ -651,6 +651,10 @@ kq_status enqueue_stacked(const float* W, int64_t d_out, int64_t d_in, int64_t l
     g.dead = from_w && dead_mask ? dead_mask + c0 : nullptr;
     g.info = info;
     g.pdl = true;   // always follows this solve's in-block kernel
+    // with stacked settings the next in-block kernel may be scheduled early
+    // (it copies its block of Uc, which no kernel of the solve writes, while
+    // this product drains; measured 2.72 -> 2.67 ms for three attn4096 solves)
+    g.trigger_early = count > 1;
     return timed(kClassUpdate, 2.0 * M * N * K, 0.0, st, [&]() { return kq::gemm_3xtf32(g, st); });
   };
   if (!tc) {
