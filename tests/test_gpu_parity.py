@@ -485,12 +485,12 @@ def test_multi_entry_points_match_single_calls(P, rotated_small, gemm_mode):
                 assert torch.equal(x, r[k])
 
 
-@pytest.mark.parametrize("d_out,d_in", [(200, 260), (33, 136), (2500, 260)])
+@pytest.mark.parametrize("d_out,d_in", [(200, 260), (33, 136), (3400, 260)])
 def test_stacked_solve_ragged_rows(P, d_out, d_in):
     """Settings stacked in one solve (M = count d_out rows in every trailing
     update, the first super-block reading W's row r mod d_out) against one
     call per setting, bit for bit, at row counts that leave partial CTAs and
-    tiles, with dead columns (3 x 2500 rows: several CTAs per SM); a
+    tiles, with dead columns (3 x 3400 rows: three CTAs per SM); a
     non-finite weight is reported with its row in W."""
     rng = np.random.default_rng(d_out + d_in)
     W = torch.from_numpy(rng.normal(0, 0.02, (d_out, d_in)).astype(np.float32)).cuda()
