@@ -415,9 +415,17 @@ __device__ __forceinline__ void rect_index(int64_t l, int64_t* ti, int64_t* tj) 
 // other's arithmetic.
 enum StepBPart { kAll = 0, kNext = 1, kRest = 2 };
 
-int64_t step_b_ctas(int64_t tr, int64_t xcols, int part) {
-  if (part == kNext) return tr + xcols;
-  if (part == kRest) return tr * tr + (tr - 1) * xcols;
+// Order from which the bulk update runs every second block step (K = 128):
+// measured 42.4 -> 37.3 ms at n = 11008, 3.20 -> 3.37 ms at n = 4096 (bound
+// by the diagonal chain, which the two-step form lengthens a little).
+constexpr int64_t kTwoStepMinN = 8192;
+
+// CTAs of a launch: kNext covers `ncols` Cholesky column tiles and the
+// substitution row tile 0; kRest the Cholesky tiles right of column tile 0
+// and `xtiles` substitution row tiles.
+int64_t step_b_ctas(int64_t tr, int64_t xcols, int part, int ncols, int64_t xtiles) {
+  if (part == kNext) return tr * ncols + xcols;
+  if (part == kRest) return tr * tr + xtiles * xcols;
   return tr * (tr + 1) + tr * xcols;
 }
 
@@ -431,20 +439,34 @@ constexpr size_t kStepBSmem = (size_t)NB * (SA + SB) * sizeof(double);   // 102 
 // stored, to factor that diagonal block and write its inverse factor to
 // Dnext: the next block step's diagonal factorisation without a launch of
 // its own.
+// Depth: the update is over `kdepth` (64 or 128) panel rows, Pt rows 0 ..
+// kdepth - 1 from `Pt` and the inverse rows from X row xk0 (128: the bulk
+// update of two block steps at once, both panels in adjacent buffers).  A
+// kNext launch covers `ncols` (1 or 2) Cholesky column tiles and stores the
+// first `xrows` (64 or 128) rows of its substitution tile; a kRest launch's
+// substitution tiles start at row base + xoff.
 __global__ void __launch_bounds__(256, 2) step_b_kernel(double* __restrict__ A, double* __restrict__ X,
                                                        const double* __restrict__ Pt, int64_t ld, int64_t k0,
                                                        int64_t tr, int part, int64_t n, double* __restrict__ Dnext,
-                                                       int32_t* info) {
+                                                       int32_t* info, int kdepth, int64_t xk0, int ncols, int xrows,
+                                                       int64_t xoff) {
   extern __shared__ __align__(16) double sm[];
   double* As = sm;               // [64][SA]
   double* Bs = sm + NB * SA;     // [64][SB]
   const int64_t base = k0 + NB;
   const int64_t xcols = base / TBN;
   const int64_t bid = blockIdx.x;
-  int64_t ti = -1, tj = 0, rb = 0, cb = 0;   // Cholesky tile (ti, tj), or substitution tile (rb, cb)
+  int64_t ti = -1, tj = 0, xrow0 = 0, cb = 0;   // Cholesky tile (ti, tj), or substitution tile (rows xrow0.., cb)
+  int store_rows = TBM;
   if (part == kNext) {
-    if (bid < tr) ti = bid;
-    else cb = bid - tr;
+    if (bid < tr * ncols) {
+      ti = bid % tr;
+      tj = bid / tr;
+    } else {
+      cb = bid - tr * ncols;
+      xrow0 = base;
+      store_rows = xrows;
+    }
   } else if (part == kRest) {
     if (bid < tr * tr) {
       int64_t q = (int64_t)sqrt((double)bid);
@@ -453,13 +475,13 @@ __global__ void __launch_bounds__(256, 2) step_b_kernel(double* __restrict__ A, 
       ti = q;
       tj = bid - q * q + 1;
     } else {
-      rb = 1 + (bid - tr * tr) / xcols;
+      xrow0 = base + xoff + ((bid - tr * tr) / xcols) * TBM;
       cb = (bid - tr * tr) % xcols;
     }
   } else {
     if (bid < tr * (tr + 1)) rect_index(bid, &ti, &tj);
     else {
-      rb = (bid - tr * (tr + 1)) / xcols;
+      xrow0 = base + ((bid - tr * (tr + 1)) / xcols) * TBM;
       cb = (bid - tr * (tr + 1)) % xcols;
     }
   }
@@ -471,31 +493,35 @@ __global__ void __launch_bounds__(256, 2) step_b_kernel(double* __restrict__ A, 
     opA = Pt + base + ti * TBM;
     opB = Pt + base + tj * TBN;
   } else {
-    C = X + (base + rb * TBM) * ld + cb * TBN;
-    opA = Pt + base + rb * TBM;
-    opB = X + k0 * ld + cb * TBN;
+    C = X + xrow0 * ld + cb * TBN;
+    opA = Pt + xrow0;
+    opB = X + xk0 * ld + cb * TBN;
   }
   const int t = threadIdx.x;
-  kq::pdl_wait();
-#pragma unroll
-  for (int g = 0; g < 4; ++g) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int id = u * 256 + t;
-      const int kk = 16 * g + id / 64, cc = id % 64;
-      cp_async16(As + kk * SA + 2 * cc, opA + kk * ld + 2 * cc);
-    }
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int id = u * 256 + t;
-      const int kk = 16 * g + id / 32, cc = id % 32;
-      cp_async16(Bs + kk * SB + 2 * cc, opB + kk * ld + 2 * cc);
-    }
-    cp_commit();
-  }
   const int warp = t / 32, lane = t % 32;
   const int wm = warp / 2, wn = warp % 2;
   const int fr = lane / 4, fc = lane % 4;
+  kq::pdl_wait();
+  // operands of the 64-deep half h of the update, in four 16-deep groups
+  auto stage = [&](int h) {
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int id = u * 256 + t;
+        const int kk = 16 * g + id / 64, cc = id % 64;
+        cp_async16(As + kk * SA + 2 * cc, opA + (64 * h + kk) * ld + 2 * cc);
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int id = u * 256 + t;
+        const int kk = 16 * g + id / 32, cc = id % 32;
+        cp_async16(Bs + kk * SB + 2 * cc, opB + (64 * h + kk) * ld + 2 * cc);
+      }
+      cp_commit();
+    }
+  };
+  stage(0);
   double acc[4][4][2];
 #pragma unroll
   for (int rt = 0; rt < 4; ++rt)
@@ -506,33 +532,44 @@ __global__ void __launch_bounds__(256, 2) step_b_kernel(double* __restrict__ A, 
       acc[rt][ct][0] = v.x;
       acc[rt][ct][1] = v.y;
     }
+#pragma unroll 1
+  for (int h = 0; h < kdepth / NB; ++h) {
+    if (h > 0) {
+      __syncthreads();   // every warp is done with the previous half's operands
+      stage(h);
+    }
 #pragma unroll
-  for (int g = 0; g < 4; ++g) {
-    if (g == 0) cp_wait<3>();
-    else if (g == 1) cp_wait<2>();
-    else if (g == 2) cp_wait<1>();
-    else cp_wait<0>();
-    __syncthreads();
+    for (int g = 0; g < 4; ++g) {
+      if (g == 0) cp_wait<3>();
+      else if (g == 1) cp_wait<2>();
+      else if (g == 2) cp_wait<1>();
+      else cp_wait<0>();
+      __syncthreads();
 #pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      const int k = 16 * g + 4 * ks + fc;
-      double a[4], b[4];
+      for (int ks = 0; ks < 4; ++ks) {
+        const int k = 16 * g + 4 * ks + fc;
+        double a[4], b[4];
 #pragma unroll
-      for (int rt = 0; rt < 4; ++rt) a[rt] = -As[k * SA + 32 * wm + 8 * rt + fr];
+        for (int rt = 0; rt < 4; ++rt) a[rt] = -As[k * SA + 32 * wm + 8 * rt + fr];
 #pragma unroll
-      for (int ct = 0; ct < 4; ++ct) b[ct] = Bs[k * SB + 32 * wn + 8 * ct + fr];
+        for (int ct = 0; ct < 4; ++ct) b[ct] = Bs[k * SB + 32 * wn + 8 * ct + fr];
 #pragma unroll
-      for (int rt = 0; rt < 4; ++rt)
+        for (int rt = 0; rt < 4; ++rt)
 #pragma unroll
-        for (int ct = 0; ct < 4; ++ct) dmma_acc(acc[rt][ct][0], acc[rt][ct][1], a[rt], b[ct]);
+          for (int ct = 0; ct < 4; ++ct) dmma_acc(acc[rt][ct][0], acc[rt][ct][1], a[rt], b[ct]);
+      }
     }
   }
+  // a substitution tile of a kNext launch may store only its first rows
+  // (warps 0-3 hold rows 0-63)
+  if (32 * wm < store_rows) {
 #pragma unroll
-  for (int rt = 0; rt < 4; ++rt)
+    for (int rt = 0; rt < 4; ++rt)
 #pragma unroll
-    for (int ct = 0; ct < 4; ++ct)
-      *reinterpret_cast<double2*>(C + (32 * wm + 8 * rt + fr) * ld + 32 * wn + 8 * ct + 2 * fc) =
-          make_double2(acc[rt][ct][0], acc[rt][ct][1]);
+      for (int ct = 0; ct < 4; ++ct)
+        *reinterpret_cast<double2*>(C + (32 * wm + 8 * rt + fr) * ld + 32 * wn + 8 * ct + 2 * fc) =
+            make_double2(acc[rt][ct][0], acc[rt][ct][1]);
+  }
   if (Dnext && bid == 0) {
     __syncthreads();   // the tile's stores are visible to the whole CTA; the operand smem is free
     potrf_block(A, ld, n, base, (int)(n - base < NB ? n - base : NB), Dnext, info, sm);
@@ -618,7 +655,7 @@ size_t ws_layout(int64_t n, CholWs* w, void* base) {
   };
   size_t oA = take((size_t)ld * ld * sizeof(double));
   size_t oX = take((size_t)ld * ld * sizeof(double));
-  size_t oP = take((size_t)2 * NB * ld * sizeof(double));   // two buffers (look-ahead)
+  size_t oP = take((size_t)4 * NB * ld * sizeof(double));   // four buffers (look-ahead, two-step bulk updates)
   size_t oD = take((size_t)nblk * NB * NB * sizeof(double));
   size_t oL = take(sizeof(double));
   if (w && base) {
@@ -665,7 +702,7 @@ extern "C" kq_status kq_chol_inv(const float* H, int64_t n, int64_t ldh, float d
   KQ_TRY(kq::launch_check("kq_chol_inv damp"));
   identity_kernel<<<1184, 256, 0, st>>>(w.X, n, ld);
   KQ_TRY(kq::launch_check("kq_chol_inv identity"));
-  KQ_TRY(kq::cuda_check(cudaMemsetAsync(w.Pt, 0, (size_t)2 * NB * ld * sizeof(double), st), "kq_chol_inv memset"));
+  KQ_TRY(kq::cuda_check(cudaMemsetAsync(w.Pt, 0, (size_t)4 * NB * ld * sizeof(double), st), "kq_chol_inv memset"));
 
   // Cholesky of the reversed matrix and the inverse of its factor, formed
   // together.  Block step k: factor diagonal block k (potrf), form its panel
@@ -682,12 +719,21 @@ extern "C" kq_status kq_chol_inv(const float* H, int64_t n, int64_t ldh, float d
   KQ_TRY(kq::cuda_check(cudaEventRecord(ev_fork, st), "kq_chol_inv: record"));
   KQ_TRY(kq::cuda_check(cudaStreamWaitEvent(s1, ev_fork, 0), "kq_chol_inv: wait"));
   const int64_t nblk = kq::cdiv(n, NB);
-  bool rest_pending = false;
+  // From kTwoStepMinN on, the bulk update runs every second block step over
+  // both steps' panels (K = 128): an even step e's kNext covers column blocks
+  // e+1 and e+2 and the substitution rows of both; the odd step o = e+1's
+  // kNext covers column block o+1 and the substitution rows of block o+1
+  // only; its kRest applies both panels to column blocks >= o+2 and to the
+  // substitution rows from block o+2 on.  That halves the passes over the
+  // trailing matrix, the bound of the bulk update for the large layers.
+  const bool two_step = n >= kTwoStepMinN;
+  bool rest_pending = false;   // a kRest that the next kNext must wait for
+  int pending_ev = 0;
   for (int64_t b = 0; b < nblk; ++b) {
     const int64_t k0 = b * NB;
     const int kb = (int)std::min<int64_t>(NB, n - k0);
     double* Dk = w.Dinv + b * NB * NB;
-    double* Pt = w.Pt + (b & 1) * NB * ld;
+    double* Pt = w.Pt + (b & 3) * NB * ld;
     // the chain potrf -> step a -> (kNext) -> potrf runs as programmatic
     // dependents on s1: each kernel is scheduled while its predecessor
     // finishes and waits for it (griddepcontrol.wait) before reading
@@ -701,19 +747,37 @@ extern "C" kq_status kq_chol_inv(const float* H, int64_t n, int64_t ldh, float d
     KQ_TRY(kq::launch_ex("kq_chol_inv step a", b > 0, step_a_kernel, dim3((unsigned)(tp + xt)), dim3(256), kStepASmem,
                          s1, w.A, w.X, Pt, ld, k0, tp, Dk));
     if (tp > 0) {
-      const int64_t tr = kq::cdiv(n - k0 - NB, TBM), xcols = (k0 + NB) / TBN;
-      KQ_TRY(kq::cuda_check(cudaEventRecord(ev_a, s1), "kq_chol_inv: record"));
-      KQ_TRY(kq::cuda_check(cudaStreamWaitEvent(st, ev_a, 0), "kq_chol_inv: wait"));
-      step_b_kernel<<<(unsigned)step_b_ctas(tr, xcols, kRest), 256, kStepBSmem, st>>>(w.A, w.X, Pt, ld, k0, tr,
-                                                                                      kRest, n, nullptr, info);
+      const int64_t base = k0 + NB;
+      const int64_t tr = kq::cdiv(n - base, TBM), xcols = base / TBN;
+      const bool odd = (b & 1) != 0;
+      const bool do_rest = !two_step || odd;
+      if (do_rest) {
+        // this step's panel alone, or (two-step) the previous step's and this one's
+        const int kdepth = two_step ? 2 * NB : NB;
+        const double* Pr = two_step ? w.Pt + ((b - 1) & 3) * NB * ld : Pt;
+        const int64_t xk0 = two_step ? k0 - NB : k0;
+        const int64_t xoff = two_step ? NB : TBM;
+        const int64_t xtiles = std::max<int64_t>(0, kq::cdiv(n - base - xoff, TBM));
+        KQ_TRY(kq::cuda_check(cudaEventRecord(ev_a, s1), "kq_chol_inv: record"));
+        KQ_TRY(kq::cuda_check(cudaStreamWaitEvent(st, ev_a, 0), "kq_chol_inv: wait"));
+        step_b_kernel<<<(unsigned)step_b_ctas(tr, xcols, kRest, 1, xtiles), 256, kStepBSmem, st>>>(
+            w.A, w.X, Pr, ld, k0, tr, kRest, n, nullptr, info, kdepth, xk0, 1, TBM, xoff);
+        KQ_TRY(kq::launch_check("kq_chol_inv step b"));
+        KQ_TRY(kq::cuda_check(cudaEventRecord(ev_rest[b & 1], st), "kq_chol_inv: record"));
+      }
+      if (rest_pending) {
+        KQ_TRY(kq::cuda_check(cudaStreamWaitEvent(s1, ev_rest[pending_ev], 0), "kq_chol_inv: wait"));
+        rest_pending = false;
+      }
+      const int ncols = (two_step && !odd && base + NB < n) ? 2 : 1;
+      const int xrows = (two_step && odd) ? NB : TBM;
+      step_b_kernel<<<(unsigned)step_b_ctas(tr, xcols, kNext, ncols, 0), 256, kStepBSmem, s1>>>(
+          w.A, w.X, Pt, ld, k0, tr, kNext, n, w.Dinv + (b + 1) * NB * NB, info, NB, k0, ncols, xrows, 0);
       KQ_TRY(kq::launch_check("kq_chol_inv step b"));
-      KQ_TRY(kq::cuda_check(cudaEventRecord(ev_rest[b & 1], st), "kq_chol_inv: record"));
-      if (rest_pending)
-        KQ_TRY(kq::cuda_check(cudaStreamWaitEvent(s1, ev_rest[(b - 1) & 1], 0), "kq_chol_inv: wait"));
-      step_b_kernel<<<(unsigned)step_b_ctas(tr, xcols, kNext), 256, kStepBSmem, s1>>>(
-          w.A, w.X, Pt, ld, k0, tr, kNext, n, w.Dinv + (b + 1) * NB * NB, info);
-      KQ_TRY(kq::launch_check("kq_chol_inv step b"));
-      rest_pending = true;
+      if (do_rest) {
+        rest_pending = true;
+        pending_ev = (int)(b & 1);
+      }
     }
   }
   KQ_TRY(kq::cuda_check(cudaEventRecord(ev_fork, s1), "kq_chol_inv: record"));
