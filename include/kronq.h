@@ -257,10 +257,10 @@ kq_status kq_rotate(float* M, int64_t rows, int64_t cols, int64_t ld, int axis,
  * library, one per (host thread, device, caller stream), forked from and
  * joined back into `stream`; calls on different caller streams (each with
  * its own workspace) run concurrently.  Blocked in 64 columns; from
- * n = 8192 on, the bulk trailing update runs every second block step over
- * both steps' panels (rank 128).  The workspace holds the padded fp64
+ * n = 8192 on, the bulk trailing update runs once every four block steps
+ * over their four panels (rank 256).  The workspace holds the padded fp64
  * matrix and its inverse (2 ld^2 doubles, ld = n rounded up to 128, + 128),
- * four panel buffers (4 * 64 * ld doubles) and the diagonal blocks'
+ * eight panel buffers (8 * 64 * ld doubles) and the diagonal blocks'
  * inverse factors (ceil(n/64) * 64^2 doubles).
  * ------------------------------------------------------------------------ */
 size_t kq_chol_inv_workspace_size(int64_t n);

@@ -415,16 +415,21 @@ __device__ __forceinline__ void rect_index(int64_t l, int64_t* ti, int64_t* tj) 
 // other's arithmetic.
 enum StepBPart { kAll = 0, kNext = 1, kRest = 2 };
 
-// Order from which the bulk update runs every second block step (K = 128):
-// measured 42.4 -> 37.3 ms at n = 11008, 3.20 -> 3.37 ms at n = 4096 (bound
-// by the diagonal chain, which the two-step form lengthens a little).
-constexpr int64_t kTwoStepMinN = 8192;
+// Block steps per bulk update (D, K = 64 D) by order: the bulk update of
+// the large orders is bound by its passes over the trailing matrix, which D
+// divides; at n = 4096 the diagonal chain bounds the factorisation (3.24 ms
+// at D = 1, 3.37 at D = 2, 3.45 at D = 4).  Measured on one B200:
+// n = 11008 42.4 / 37.2 / 35.4 ms and n = 28672 581 (D = 2) / 537 ms
+// (D = 4).
+constexpr int64_t kMultiStepMinN = 8192;
+constexpr int kMaxSteps = 4;
+int bulk_steps(int64_t n) { return n >= kMultiStepMinN ? kMaxSteps : 1; }
 
-// CTAs of a launch: kNext covers `ncols` Cholesky column tiles and the
-// substitution row tile 0; kRest the Cholesky tiles right of column tile 0
+// CTAs of a launch: kNext covers `ncols` Cholesky column tiles and `xtiles`
+// substitution row tiles; kRest the Cholesky tiles right of column tile 0
 // and `xtiles` substitution row tiles.
 int64_t step_b_ctas(int64_t tr, int64_t xcols, int part, int ncols, int64_t xtiles) {
-  if (part == kNext) return tr * ncols + xcols;
+  if (part == kNext) return tr * ncols + xtiles * xcols;
   if (part == kRest) return tr * tr + xtiles * xcols;
   return tr * (tr + 1) + tr * xcols;
 }
@@ -439,12 +444,13 @@ constexpr size_t kStepBSmem = (size_t)NB * (SA + SB) * sizeof(double);   // 102 
 // stored, to factor that diagonal block and write its inverse factor to
 // Dnext: the next block step's diagonal factorisation without a launch of
 // its own.
-// Depth: the update is over `kdepth` (64 or 128) panel rows, Pt rows 0 ..
-// kdepth - 1 from `Pt` and the inverse rows from X row xk0 (128: the bulk
-// update of two block steps at once, both panels in adjacent buffers).  A
-// kNext launch covers `ncols` (1 or 2) Cholesky column tiles and stores the
-// first `xrows` (64 or 128) rows of its substitution tile; a kRest launch's
-// substitution tiles start at row base + xoff.
+// Depth: the update is over `kdepth` (64 D) panel rows, Pt rows 0 ..
+// kdepth - 1 from `Pt` and the inverse rows from X row xk0 (D > 1: the bulk
+// update of D block steps at once, their panels in adjacent buffers).  A
+// kNext launch covers `ncols` Cholesky column tiles and the first `xrows`
+// substitution rows from `base` (ceil(xrows / 128) row tiles, the last one
+// stored in part); a kRest launch's substitution tiles start at row
+// base + xoff.
 __global__ void __launch_bounds__(256, 2) step_b_kernel(double* __restrict__ A, double* __restrict__ X,
                                                        const double* __restrict__ Pt, int64_t ld, int64_t k0,
                                                        int64_t tr, int part, int64_t n, double* __restrict__ Dnext,
@@ -463,9 +469,10 @@ __global__ void __launch_bounds__(256, 2) step_b_kernel(double* __restrict__ A, 
       ti = bid % tr;
       tj = bid / tr;
     } else {
-      cb = bid - tr * ncols;
-      xrow0 = base;
-      store_rows = xrows;
+      const int64_t x = bid - tr * ncols, rt = x / xcols;
+      cb = x % xcols;
+      xrow0 = base + rt * TBM;
+      store_rows = (int)std::min<int64_t>(TBM, xrows - rt * TBM);
     }
   } else if (part == kRest) {
     if (bid < tr * tr) {
@@ -655,7 +662,7 @@ size_t ws_layout(int64_t n, CholWs* w, void* base) {
   };
   size_t oA = take((size_t)ld * ld * sizeof(double));
   size_t oX = take((size_t)ld * ld * sizeof(double));
-  size_t oP = take((size_t)4 * NB * ld * sizeof(double));   // four buffers (look-ahead, two-step bulk updates)
+  size_t oP = take((size_t)2 * kMaxSteps * NB * ld * sizeof(double));   // 2 D panel buffers
   size_t oD = take((size_t)nblk * NB * NB * sizeof(double));
   size_t oL = take(sizeof(double));
   if (w && base) {
@@ -702,7 +709,8 @@ extern "C" kq_status kq_chol_inv(const float* H, int64_t n, int64_t ldh, float d
   KQ_TRY(kq::launch_check("kq_chol_inv damp"));
   identity_kernel<<<1184, 256, 0, st>>>(w.X, n, ld);
   KQ_TRY(kq::launch_check("kq_chol_inv identity"));
-  KQ_TRY(kq::cuda_check(cudaMemsetAsync(w.Pt, 0, (size_t)4 * NB * ld * sizeof(double), st), "kq_chol_inv memset"));
+  KQ_TRY(kq::cuda_check(cudaMemsetAsync(w.Pt, 0, (size_t)2 * kMaxSteps * NB * ld * sizeof(double), st),
+                        "kq_chol_inv memset"));
 
   // Cholesky of the reversed matrix and the inverse of its factor, formed
   // together.  Block step k: factor diagonal block k (potrf), form its panel
@@ -719,21 +727,26 @@ extern "C" kq_status kq_chol_inv(const float* H, int64_t n, int64_t ldh, float d
   KQ_TRY(kq::cuda_check(cudaEventRecord(ev_fork, st), "kq_chol_inv: record"));
   KQ_TRY(kq::cuda_check(cudaStreamWaitEvent(s1, ev_fork, 0), "kq_chol_inv: wait"));
   const int64_t nblk = kq::cdiv(n, NB);
-  // From kTwoStepMinN on, the bulk update runs every second block step over
-  // both steps' panels (K = 128): an even step e's kNext covers column blocks
-  // e+1 and e+2 and the substitution rows of both; the odd step o = e+1's
-  // kNext covers column block o+1 and the substitution rows of block o+1
-  // only; its kRest applies both panels to column blocks >= o+2 and to the
-  // substitution rows from block o+2 on.  That halves the passes over the
-  // trailing matrix, the bound of the bulk update for the large layers.
-  const bool two_step = n >= kTwoStepMinN;
+  // Bulk updates of D block steps (D = bulk_steps(n)): the steps form groups
+  // [g0, g0 + D); step k's kNext updates column blocks k+1 .. g0+D and their
+  // substitution rows (D = 1: column block k+1 and the rows of blocks k+1,
+  // k+2), so the diagonal chain never waits for a bulk update inside the
+  // group; the group's last step's kRest applies the group's D panels
+  // (K = 64 D) to the column blocks and substitution rows beyond.  Every
+  // (panel, block) pair is updated exactly once, before the block is
+  // factored or read as a panel.  The panels of two groups alternate in 2 D
+  // buffers, so a group's panels stay until its kRest has read them (the
+  // next group's first kNext waits for that kRest, and every later panel
+  // step follows that kNext on the chain's stream).
+  const int D = bulk_steps(n);
   bool rest_pending = false;   // a kRest that the next kNext must wait for
   int pending_ev = 0;
   for (int64_t b = 0; b < nblk; ++b) {
     const int64_t k0 = b * NB;
     const int kb = (int)std::min<int64_t>(NB, n - k0);
     double* Dk = w.Dinv + b * NB * NB;
-    double* Pt = w.Pt + (b & 3) * NB * ld;
+    double* Pt = w.Pt + (b % (2 * D)) * NB * ld;
+    const int p = (int)(b % D);   // position in the group
     // the chain potrf -> step a -> (kNext) -> potrf runs as programmatic
     // dependents on s1: each kernel is scheduled while its predecessor
     // finishes and waits for it (griddepcontrol.wait) before reading
@@ -749,19 +762,17 @@ extern "C" kq_status kq_chol_inv(const float* H, int64_t n, int64_t ldh, float d
     if (tp > 0) {
       const int64_t base = k0 + NB;
       const int64_t tr = kq::cdiv(n - base, TBM), xcols = base / TBN;
-      const bool odd = (b & 1) != 0;
-      const bool do_rest = !two_step || odd;
+      const bool do_rest = (p == D - 1);
       if (do_rest) {
-        // this step's panel alone, or (two-step) the previous step's and this one's
-        const int kdepth = two_step ? 2 * NB : NB;
-        const double* Pr = two_step ? w.Pt + ((b - 1) & 3) * NB * ld : Pt;
-        const int64_t xk0 = two_step ? k0 - NB : k0;
-        const int64_t xoff = two_step ? NB : TBM;
+        // the group's D panels (D = 1: this step's alone)
+        const int64_t g0 = b - (D - 1);
+        const double* Pr = w.Pt + (g0 % (2 * D)) * NB * ld;
+        const int64_t xoff = D == 1 ? TBM : NB;
         const int64_t xtiles = std::max<int64_t>(0, kq::cdiv(n - base - xoff, TBM));
         KQ_TRY(kq::cuda_check(cudaEventRecord(ev_a, s1), "kq_chol_inv: record"));
         KQ_TRY(kq::cuda_check(cudaStreamWaitEvent(st, ev_a, 0), "kq_chol_inv: wait"));
         step_b_kernel<<<(unsigned)step_b_ctas(tr, xcols, kRest, 1, xtiles), 256, kStepBSmem, st>>>(
-            w.A, w.X, Pr, ld, k0, tr, kRest, n, nullptr, info, kdepth, xk0, 1, TBM, xoff);
+            w.A, w.X, Pr, ld, k0, tr, kRest, n, nullptr, info, D * NB, g0 * NB, 1, TBM, xoff);
         KQ_TRY(kq::launch_check("kq_chol_inv step b"));
         KQ_TRY(kq::cuda_check(cudaEventRecord(ev_rest[b & 1], st), "kq_chol_inv: record"));
       }
@@ -769,10 +780,13 @@ extern "C" kq_status kq_chol_inv(const float* H, int64_t n, int64_t ldh, float d
         KQ_TRY(kq::cuda_check(cudaStreamWaitEvent(s1, ev_rest[pending_ev], 0), "kq_chol_inv: wait"));
         rest_pending = false;
       }
-      const int ncols = (two_step && !odd && base + NB < n) ? 2 : 1;
-      const int xrows = (two_step && odd) ? NB : TBM;
-      step_b_kernel<<<(unsigned)step_b_ctas(tr, xcols, kNext, ncols, 0), 256, kStepBSmem, s1>>>(
-          w.A, w.X, Pt, ld, k0, tr, kNext, n, w.Dinv + (b + 1) * NB * NB, info, NB, k0, ncols, xrows, 0);
+      // column blocks b+1 .. g0+D (those that exist) and their substitution rows
+      const int64_t ahead = D == 1 ? 1 : D - p;
+      const int ncols = (int)std::min<int64_t>(ahead, kq::cdiv(n - base, NB));
+      const int64_t xrows = D == 1 ? TBM : std::min<int64_t>(ahead * NB, n - base);
+      const int64_t nxt = kq::cdiv(xrows, TBM);
+      step_b_kernel<<<(unsigned)step_b_ctas(tr, xcols, kNext, ncols, nxt), 256, kStepBSmem, s1>>>(
+          w.A, w.X, Pt, ld, k0, tr, kNext, n, w.Dinv + (b + 1) * NB * NB, info, NB, k0, ncols, (int)xrows, 0);
       KQ_TRY(kq::launch_check("kq_chol_inv step b"));
       if (do_rest) {
         rest_pending = true;
