@@ -210,6 +210,38 @@ def test_chol_inv_parity(P, n, seed):
     assert np.array_equal(dead.cpu().numpy().astype(bool), dref)
 
 
+def test_chol_inv_grouped_bulk_update_residual(P):
+    """From n = 8192 the bulk update runs once every four block steps; at
+    n = 8200 (129 blocks of 64, the last one 8 wide) the last group of steps
+    is incomplete.  A residual pin of the whole factor in fp64, for the first
+    64, the last 64 and 64 random columns j: ||(Uc^T Uc (H + lambda I) - I) e_j||
+    <= 2e-6 (H from 4n samples, so the exact factor rounded to fp32 leaves
+    about 1e-7)."""
+    n = 8200
+    g = torch.Generator(device="cuda")
+    g.manual_seed(41)
+    A = torch.randn((n, 4 * n), device="cuda", generator=g)
+    H = (A @ A.T) / (4 * n)
+    del A
+    Uc = torch.empty_like(H)
+    info = _info()
+    P.kq_chol_inv(H, 0.01, Uc, None, None, info)
+    torch.cuda.synchronize()
+    assert _info_code(info)[0] == 0
+    lam = 0.01 * float(torch.diagonal(H).double().mean())
+    rng = np.random.default_rng(43)
+    S = np.unique(np.r_[np.arange(64), np.arange(n - 64, n), rng.choice(n, 64, replace=False)])
+    St = torch.from_numpy(S).cuda()
+    Hs = torch.triu(H.double())[:, St] + torch.triu(H.double(), 1).T[:, St]   # columns of the symmetric H
+    Hs[St, torch.arange(len(S), device="cuda")] += lam
+    U = Uc.double()
+    R = U.T @ (U @ Hs)
+    R[St, torch.arange(len(S), device="cuda")] -= 1.0
+    r = torch.linalg.vector_norm(R, dim=0).cpu().numpy()
+    assert float(torch.tril(Uc, -1).abs().max()) == 0.0
+    assert r.max() <= 2e-6, (float(r.max()), int(S[int(np.argmax(r))]))
+
+
 def test_chol_inv_dead_columns_and_errors(P):
     H = _spd(150, 9)
     H[[3, 77, 149], :] = 0
@@ -485,13 +517,14 @@ def test_multi_entry_points_match_single_calls(P, rotated_small, gemm_mode):
                 assert torch.equal(x, r[k])
 
 
-@pytest.mark.parametrize("d_out,d_in", [(200, 260), (33, 136), (3400, 260)])
+@pytest.mark.parametrize("d_out,d_in", [(200, 260), (33, 136), (3400, 260), (200, 1300)])
 def test_stacked_solve_ragged_rows(P, d_out, d_in):
     """Settings stacked in one solve (M = count d_out rows in every trailing
     update, the first super-block reading W's row r mod d_out) against one
     call per setting, bit for bit, at row counts that leave partial CTAs and
-    tiles, with dead columns (3 x 3400 rows: three CTAs per SM); a
-    non-finite weight is reported with its row in W."""
+    tiles, with dead columns (3 x 3400 rows: three CTAs per SM; 1300
+    columns: the K = 1024 update after the first super-block reads W too);
+    a non-finite weight is reported with its row in W."""
     rng = np.random.default_rng(d_out + d_in)
     W = torch.from_numpy(rng.normal(0, 0.02, (d_out, d_in)).astype(np.float32)).cuda()
     H = torch.from_numpy(_spd(d_in, 5, 1.0)).cuda()
