@@ -140,13 +140,19 @@ struct InblockArgs {
 // warp read the same row: broadcast).  Fewer lanes per row mean fewer warps
 // repeating the per-column quantisation and shuffle (the latency-bound part)
 // for the same multiply-adds.
-constexpr int IB_THREADS = 256;
+// Threads per CTA of the in-block kernel (4 rows per warp): 224 (28 rows)
+// below kStackedRows rows, so that 4096 rows make 147 CTAs on 147 SMs
+// (measured 1.46 -> 1.38 ms for one attn4096 solve); 256 (32 rows) for
+// larger stacked solves, where 441 CTAs of 28 rows measured slower than 384
+// of 32 (1.30 against 1.05 ms for the 32 in-block launches of three
+// attn4096 settings).
+constexpr int kStackedRows = 2 * 148 * 32;
 constexpr int IB_SMEM = BLK * BLK * 4 + BLK * 4;
 
 template <int LPR>
 __device__ __forceinline__ int col_of(int L, int r) { return 4 * LPR * (r >> 2) + 4 * L + (r & 3); }
 
-template <int LPR>
+template <int LPR, int IB_THREADS>
 __global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
   constexpr int IB_ROWS = IB_THREADS / LPR;   // rows per CTA
   constexpr int NR = BLK / LPR;               // columns (registers) per lane
@@ -174,8 +180,9 @@ __global__ void __launch_bounds__(IB_THREADS) inblock_kernel(InblockArgs a) {
   // No kernel of the solve writes Uc, so the copies may start before the
   // previous kernel (a trailing update) has finished.
 #pragma unroll
-  for (int u = 0; u < BLK * (BLK / 4) / IB_THREADS; ++u) {
+  for (int u = 0; u < (BLK * (BLK / 4) + IB_THREADS - 1) / IB_THREADS; ++u) {
     const int idx = t + IB_THREADS * u;
+    if (idx >= BLK * (BLK / 4)) break;
     const int j = idx / (BLK / 4), k = 4 * (idx % (BLK / 4));
     // chunks wholly below the diagonal (k + 3 < j) are zero-filled: only the
     // upper triangle of Uc is the factor
@@ -590,8 +597,11 @@ kq_status enqueue_stacked(const float* W, int64_t d_out, int64_t d_in, int64_t l
       return kq::launch_check("kq_quantize_layer grid");
     }));
   }
-  KQ_TRY(kq::cuda_check(cudaFuncSetAttribute(inblock_kernel<kLanesPerRow>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             IB_SMEM), "kq_quantize_layer: smem attribute"));
+  const bool stacked_rows = M >= kStackedRows;
+  auto ib_kernel = stacked_rows ? inblock_kernel<kLanesPerRow, 256> : inblock_kernel<kLanesPerRow, 224>;
+  const int ib_threads = stacked_rows ? 256 : 224;
+  KQ_TRY(kq::cuda_check(cudaFuncSetAttribute(ib_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, IB_SMEM),
+                        "kq_quantize_layer: smem attribute"));
   auto inblock = [&](int64_t i0, int64_t o0) -> kq_status {
     const int bw = (int)std::min<int64_t>(BLK, d_in - i0);
     const bool first = (i0 == 0);
@@ -620,9 +630,9 @@ kq_status enqueue_stacked(const float* W, int64_t d_out, int64_t d_in, int64_t l
     // after the first block the previous kernel is this solve's own trailing
     // update, so the launch may overlap its tail (tensor-core mode)
     return timed(kClassInblock, 0.0, (double)M * bw * (tc ? 17.0 : 13.0), st, [&]() {
-      return kq::launch_ex("kq_quantize_layer inblock", tc && i0 > 0, inblock_kernel<kLanesPerRow>,
-                           dim3((unsigned)kq::cdiv(d_out, IB_THREADS / kLanesPerRow), (unsigned)count),
-                           dim3(IB_THREADS), IB_SMEM, st, a);
+      return kq::launch_ex("kq_quantize_layer inblock", tc && i0 > 0, ib_kernel,
+                           dim3((unsigned)kq::cdiv(d_out, ib_threads / kLanesPerRow), (unsigned)count),
+                           dim3(ib_threads), IB_SMEM, st, a);
     });
   };
   // W_hat[:, c0:c0+N] = src[:, c0:c0+N] - E[:, e0:e0+K] Uc[k0:k0+K, c0:c0+N] over
