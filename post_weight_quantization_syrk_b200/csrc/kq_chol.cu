@@ -747,11 +747,11 @@ extern "C" kq_status kq_chol_inv(const float* H, int64_t n, int64_t ldh, float d
     double* Dk = w.Dinv + b * NB * NB;
     double* Pt = w.Pt + (b % (2 * D)) * NB * ld;
     const int p = (int)(b % D);   // position in the group
-    // the chain potrf -> step a -> (kNext) -> potrf runs as programmatic
+    // The chain potrf -> step a -> kNext -> step a ... runs as programmatic
     // dependents on s1: each kernel is scheduled while its predecessor
-    // finishes and waits for it (griddepcontrol.wait) before reading
-    // block 0's diagonal factorisation has a launch of its own; every later
-    // one is done by the previous step's kNext launch (CTA 0)
+    // finishes and waits for it (griddepcontrol.wait) before reading.
+    // Block 0's diagonal factorisation has a launch of its own; every later
+    // one is done by the previous step's kNext launch (its CTA 0).
     if (b == 0)
       KQ_TRY(kq::launch_ex("kq_chol_inv potrf", false, potrf_kernel, dim3(1), dim3(256), kPotrfSmem, s1, w.A, ld, n,
                            k0, kb, Dk, info));
