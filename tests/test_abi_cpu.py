@@ -185,6 +185,20 @@ def test_workspace_sizes():
     assert P.kq_chol_inv_workspace_size(0) == 0
 
 
+def test_chol_inv_workspace_holds_what_the_header_lists():
+    """kq_chol_inv's workspace as its header documents it: the padded fp64
+    matrix and its inverse (2 ld^2 doubles, ld = n rounded up to 128, + 128),
+    eight panel buffers (8 * 64 * ld doubles) and the diagonal blocks'
+    inverse factors (ceil(n/64) * 64^2 doubles), each rounded up to 256
+    bytes, plus one double."""
+    def up(x):
+        return -(-x // 256) * 256
+    for n in (1, 63, 64, 1000, 4096, 8200, 11008, 28672):
+        ld = -(-n // 128) * 128 + 128
+        want = up(ld * ld * 8) * 2 + up(8 * 64 * ld * 8) + up(-(-n // 64) * 64 * 64 * 8) + up(8)
+        assert P.kq_chol_inv_workspace_size(n) == want, n
+
+
 def test_multi_workspace_sizes():
     """One lane per setting up to four lanes; one lane is the single-setting size."""
     one = P.kq_quantize_layer_workspace_size(4096, 4096)
