@@ -477,8 +477,8 @@ def run_kronq(a):
 # 262144 x 4096, from one ncu capture of dram__bytes_read.sum and
 # dram__bytes_write.sum; valid only for the kernel sources it was taken on
 # (their hashes), else the bench reports null.
-SYRK_TRAFFIC = {"attn4096": 5.00e9}
-SYRK_SOURCE_SHA = {"kq_syrk.cu": "a457aac871c196f3", "kq_tc.cuh": "91f487fc41a449d7"}
+SYRK_TRAFFIC = {"attn4096": 5.09e9}
+SYRK_SOURCE_SHA = {"kq_syrk.cu": "3634edf2f04853fc", "kq_tc.cuh": "91f487fc41a449d7"}
 
 
 def syrk_traffic(workload):
